@@ -1,0 +1,315 @@
+"""Pins of the CPU oracle against what the pages and the mathematics fix.
+
+Each test checks the oracle against something other than itself: a library routine, exact
+rational arithmetic, a closed form, an invariant of the definition, or brute force.
+"""
+import itertools
+import json
+import math
+import os
+from fractions import Fraction
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import rtp_oracle as O
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+# ----------------------------------------------------------------------------- bf16 rounding
+def _bf16_exact(x: float) -> float:
+    """Round-to-nearest-even to 8 significant bits with exact rationals."""
+    if x == 0 or not math.isfinite(x):
+        return x
+    f = Fraction(x)
+    sign = -1 if f < 0 else 1
+    a = abs(f)
+    e = 0
+    while a >= 2:
+        a /= 2
+        e += 1
+    while a < 1:
+        a *= 2
+        e -= 1
+    e = max(e, -126)                       # subnormal spacing 2^-133
+    q = Fraction(2) ** (e - 7)
+    n = abs(f) / q
+    fl = n.numerator // n.denominator
+    rem = n - fl
+    if rem > Fraction(1, 2) or (rem == Fraction(1, 2) and fl % 2 == 1):
+        fl += 1
+    return sign * float(fl * q)
+
+
+def test_bf16_round_matches_torch_on_float32_inputs():
+    rng = np.random.default_rng(0)
+    x = np.concatenate([rng.standard_normal(20000) * 10.0 ** rng.integers(-30, 30, 20000),
+                        rng.standard_normal(1000) * 1e-39]).astype(np.float32)
+    ref = torch.from_numpy(x).to(torch.bfloat16).to(torch.float64).numpy()
+    np.testing.assert_array_equal(O.bf16_round(x.astype(np.float64)), ref)
+
+
+def test_bf16_round_matches_exact_rationals_on_float64_inputs():
+    rng = np.random.default_rng(1)
+    xs = list(rng.standard_normal(3000) * 10.0 ** rng.integers(-12, 12, 3000))
+    # exact ties: odd multiples of half a bf16 spacing
+    for k in range(1, 200, 2):
+        xs.append(1.0 + k * 2.0 ** -8)
+        xs.append(-(3.0 + k * 2.0 ** -7))
+    xs += [2.0 ** -130 * 1.37, -(2.0 ** -128) * 1.5]     # bf16 subnormal range
+    got = O.bf16_round(np.array(xs))
+    for x, g in zip(xs, got):
+        assert g == _bf16_exact(float(x)), x
+
+
+# ----------------------------------------------------------------------------- RoPE, eq. (1)-(2)
+def test_rope_theta_decreasing_and_endpoints():
+    th = O.rope_theta(128, 1e6)
+    assert th[0] == 1.0
+    assert np.all(np.diff(th) < 0)
+    assert math.isclose(th[-1], 1e6 ** (-126 / 128), rel_tol=1e-15)
+
+
+def test_rope_matches_complex_rotation():
+    """Each pair (i, i+64) is the complex number x_i + j x_{i+64} times exp(j m theta_i)."""
+    rng = np.random.default_rng(2)
+    x = rng.standard_normal((5, 128))
+    pos = np.array([0, 1, 17, 4095, 1048575])
+    th = 1e6 ** (-np.arange(64) * 2.0 / 128)
+    z = (x[:, :64] + 1j * x[:, 64:]) * np.exp(1j * pos[:, None] * th[None, :])
+    ref = np.concatenate([z.real, z.imag], axis=1)
+    np.testing.assert_allclose(O.rope_rotate(x, pos), ref, rtol=0, atol=1e-12)
+
+
+def test_rope_identity_and_orthogonality():
+    rng = np.random.default_rng(3)
+    x = rng.standard_normal((7, 128))
+    np.testing.assert_array_equal(O.rope_rotate(x, np.zeros(7)), x)
+    y = O.rope_rotate(x, np.arange(7) * 1000 + 5)
+    np.testing.assert_allclose(np.linalg.norm(y, axis=1), np.linalg.norm(x, axis=1), rtol=1e-13)
+
+
+def test_rope_score_depends_only_on_offset_eq2():
+    """Eq. (2): q_m^T k_n = sum_i [a_i cos(theta_i D) + b_i sin(theta_i D)], D = m - n."""
+    rng = np.random.default_rng(4)
+    q, k = rng.standard_normal(128), rng.standard_normal(128)
+    th = O.rope_theta(128, 1e6)
+    qa, qb, ka, kb = q[:64], q[64:], k[:64], k[64:]
+    a = qa * ka + qb * kb
+    b = qa * kb - qb * ka
+    for m, n in [(10, 3), (5000, 4999), (1_000_000, 123), (77, 77)]:
+        got = O.rope_rotate(q, m) @ O.rope_rotate(k, n)
+        closed = np.sum(a * np.cos(th * (m - n)) + b * np.sin(th * (m - n)))
+        assert abs(got - closed) < 1e-9 * np.linalg.norm(q) * np.linalg.norm(k)
+        for c in (1, 1000, 65536):
+            sh = O.rope_rotate(q, m + c) @ O.rope_rotate(k, n + c)
+            assert abs(sh - got) < 1e-9 * np.linalg.norm(q) * np.linalg.norm(k)
+
+
+# ----------------------------------------------------------------------------- eq. (4)
+def test_index_keys_selector_weight_reduces_to_columns():
+    """With W^K = [I_16; 0] the projection of a bf16 key is its first 16 channels, exactly."""
+    rng = np.random.default_rng(5)
+    k = O.bf16_round(rng.standard_normal((50, 128)))
+    W = np.zeros((128, 16))
+    W[:16, :16] = np.eye(16)
+    np.testing.assert_array_equal(O.index_keys(k, W), k[:, :16])
+    # a permuting selector catches a transposed operand
+    W2 = np.zeros((128, 16))
+    perm = rng.permutation(128)[:16]
+    W2[perm, np.arange(16)] = 1.0
+    np.testing.assert_array_equal(O.index_keys(k, W2), k[:, perm])
+
+
+def test_index_scores_match_torch_and_bilinear_form():
+    """s = (W^Q q)^T (W^K k) equals q^T (W^Q^T W^K) k before rounding and torch's matmul."""
+    rng = np.random.default_rng(6)
+    q = rng.standard_normal(128)
+    k = rng.standard_normal((40, 128))
+    Wq = rng.standard_normal((128, 16)) / 11.3
+    Wk = rng.standard_normal((128, 16)) / 11.3
+    s = O.index_scores(O.index_query(q, Wq), k @ Wk)
+    bil = k @ (Wk @ Wq.T) @ q
+    np.testing.assert_allclose(s, bil, rtol=1e-12, atol=1e-12)
+    tq = torch.from_numpy(q) @ torch.from_numpy(Wq)
+    tk = torch.from_numpy(k) @ torch.from_numpy(Wk)
+    np.testing.assert_allclose(s, (tk @ tq).numpy(), rtol=1e-12, atol=1e-12)
+
+
+# ----------------------------------------------------------------------------- eq. (5): Top-P
+def test_topp_hand_worked_example():
+    """Scores {0, 0, ln2, ln8}: masses {1/8, 1/8, 1/4, 1}, T = 3/2; bins 0, 0, 85, 255
+    (256 ln2/ln8 = 85.33). p=0.9 -> C_0 = 1.5 >= 1.35 is the first bin from the top that
+    reaches pT, so b* = 0 (all); p=0.8 -> C_85 = 1.25 >= 1.2 -> {2, 3}; p=0.6 -> C_255 = 1 ->
+    {3}."""
+    s = np.array([0.0, 0.0, math.log(2.0), math.log(8.0)])
+    sel = O.topp_histogram(s, 0.9)
+    assert list(sel.bins) == [0, 0, 85, 255]
+    np.testing.assert_allclose(sel.T, 1.5, rtol=1e-15)
+    assert sel.bstar == 0 and sel.mask.all()
+    sel = O.topp_histogram(s, 0.8)
+    assert sel.bstar == 85 and list(np.nonzero(sel.mask)[0]) == [2, 3]
+    sel = O.topp_histogram(s, 0.6)
+    assert sel.bstar == 255 and list(np.nonzero(sel.mask)[0]) == [3]
+    assert list(np.nonzero(O.topp_exact(s, 0.8))[0]) == [2, 3]
+    assert list(np.nonzero(O.topp_exact(s, 0.6))[0]) == [3]
+
+
+def _brute_minimal_set(s, p):
+    """Minimal-cardinality subsets with mass >= p * total, by enumeration."""
+    w = np.exp(s - s.max())
+    T = w.sum()
+    N = len(s)
+    for k in range(1, N + 1):
+        best = None
+        for comb in itertools.combinations(range(N), k):
+            m = w[list(comb)].sum()
+            if m >= p * T and (best is None or m > best[0]):
+                best = (m, comb)
+        if best is not None:
+            return k, best[0]
+    return N, T
+
+
+@pytest.mark.parametrize("seed", range(12))
+def test_topp_exact_is_minimal_set_by_enumeration(seed):
+    rng = np.random.default_rng(100 + seed)
+    N = int(rng.integers(1, 13))
+    s = rng.standard_normal(N) * rng.uniform(0.1, 4.0)
+    p = float(rng.uniform(0.3, 0.99))
+    k, best_mass = _brute_minimal_set(s, p)
+    ex = O.topp_exact(s, p)
+    assert ex.sum() == k
+    w = np.exp(s - s.max())
+    assert math.isclose(w[ex].sum(), best_mass, rel_tol=1e-12)
+
+
+@pytest.mark.parametrize("seed", range(40))
+def test_topp_histogram_invariants(seed):
+    """S_exact is a subset of S; extra tokens all sit in bin b*; mass(S) >= p; bins above b*
+    hold less than p of the mass (b* is maximal); exact top-p agrees with a full sort."""
+    rng = np.random.default_rng(200 + seed)
+    N = int(rng.integers(2, 5000 if seed % 4 == 0 else 64))
+    s = rng.standard_normal(N) * rng.uniform(0.2, 6.0)
+    if seed % 5 == 1:                                     # a planted run
+        s[: max(1, N // 20)] += rng.uniform(2, 8)
+    if seed % 7 == 2:                                     # heavy ties
+        s = np.round(s)
+    p = float(rng.choice([0.5, 0.8, 0.9, 0.95, 0.99]))
+    sel = O.topp_histogram(s, p)
+    ex = O.topp_exact(s, p)
+    w = np.exp(s - s.max())
+    T = w.sum()
+    assert np.all(sel.mask[ex])
+    extra = sel.mask & ~ex
+    if not sel.select_all:
+        assert np.all(sel.bins[extra] == sel.bstar)
+        above = w[sel.bins > sel.bstar].sum()
+        assert above < p * T * (1 + 1e-12)
+    assert w[sel.mask].sum() >= p * T * (1 - 1e-12)
+    # the exact set is a prefix of the order by (score desc, index asc)
+    order = np.lexsort((np.arange(N), -s))
+    k = int(ex.sum())
+    assert set(order[:k]) == set(np.nonzero(ex)[0])
+    assert w[order[: k - 1]].sum() < p * T * (1 + 1e-12) or k == 1
+
+
+def test_topp_special_cases():
+    s = np.full(10, 3.25)
+    assert O.topp_histogram(s, 0.9).mask.all()            # all scores equal -> all
+    rng = np.random.default_rng(7)
+    s = rng.standard_normal(100)
+    assert O.topp_histogram(s, 1.0).mask.all()            # p >= 1 -> all
+    assert O.topp_exact(s, 1.0).all()
+    s = np.zeros(100)
+    s[37] = 100.0                                          # one dominant token -> its bin only
+    sel = O.topp_histogram(s, 0.9)
+    assert sel.bstar == 255 and list(np.nonzero(sel.mask)[0]) == [37]
+    sel = O.topp_histogram(np.array([1.5]), 0.9)           # N = 1
+    assert sel.mask.all()
+    with pytest.raises(ValueError):
+        O.topp_histogram(np.array([]), 0.9)
+
+
+def test_bins_linear_over_min_max():
+    s = np.linspace(-3.0, 5.0, 257)                        # exactly on the 256 bin edges
+    b = O.score_bins(s, -3.0, 5.0)
+    assert b[0] == 0 and b[-1] == 255
+    assert np.all(b[:-1] == np.arange(256))
+
+
+# ----------------------------------------------------------------------------- attention
+def _rope_complex(x, pos, base=1e6):
+    th = base ** (-np.arange(64) * 2.0 / 128)
+    z = (x[..., :64] + 1j * x[..., 64:]) * np.exp(1j * np.asarray(pos)[..., None] * th)
+    return np.concatenate([z.real, z.imag], axis=-1)
+
+
+def test_attend_matches_torch_sdpa():
+    rng = np.random.default_rng(8)
+    q = rng.standard_normal(128)
+    K = rng.standard_normal((300, 128))
+    V = rng.standard_normal((300, 128))
+    ref = torch.nn.functional.scaled_dot_product_attention(
+        torch.from_numpy(q)[None, None, None, :], torch.from_numpy(K)[None, None],
+        torch.from_numpy(V)[None, None])[0, 0, 0].numpy()
+    np.testing.assert_allclose(O.attend(q, K, V), ref, rtol=1e-12, atol=1e-12)
+    np.testing.assert_array_equal(O.attend(q, K[3:4], V[3:4]), V[3])
+
+
+def test_layer_reduces_to_dense_attention():
+    """p = 1 (retrieval) and window >= N (local) make the layer dense softmax attention over all
+    N RoPE'd, bf16-stored keys; compared with torch SDPA and a complex-number RoPE."""
+    rng = np.random.default_rng(9)
+    B, Hq, Hkv, N = 2, 4, 2, 300
+    q_pre = O.bf16_round(rng.standard_normal((B, Hq, 128)))
+    kp = O.bf16_round(rng.standard_normal((B, Hkv, N, 128)))
+    vv = O.bf16_round(rng.standard_normal((B, Hkv, N, 128)))
+    wq = rng.standard_normal((Hq, 128, 16)) / 11.3
+    wk = rng.standard_normal((Hkv, 128, 16)) / 11.3
+    res = O.decode_layer(q_pre, wq, wk, lambda b, g: kp[b, g], lambda b, g: vv[b, g],
+                         np.array([True, False]), [N, N], 1.0, sinks=4, window=N)
+    for b in range(B):
+        for h in range(Hq):
+            g = h // 2
+            K = O.bf16_round(_rope_complex(kp[b, g], np.arange(N)))
+            q = _rope_complex(q_pre[b, h], N - 1)
+            ref = torch.nn.functional.scaled_dot_product_attention(
+                torch.from_numpy(q)[None, None, None], torch.from_numpy(K)[None, None],
+                torch.from_numpy(vv[b, g])[None, None])[0, 0, 0].numpy()
+            np.testing.assert_allclose(res[(b, h)].out, ref, rtol=1e-10, atol=1e-12)
+            assert res[(b, h)].count == N
+
+
+def test_local_positions_bruteforce():
+    for N in range(1, 40):
+        for sinks in range(0, 6):
+            for window in range(1, 12):
+                ref = [n for n in range(N) if n < sinks or n >= N - window]
+                got = O.local_positions(N, sinks, window)
+                assert list(got) == ref, (N, sinks, window)
+
+
+def test_single_token_cache():
+    """N = 1: the only token is selected and the output is its value row."""
+    rng = np.random.default_rng(10)
+    kp = O.bf16_round(rng.standard_normal((1, 128)))
+    vv = O.bf16_round(rng.standard_normal((1, 128)))
+    r = O.retrieval_head(rng.standard_normal(128), rng.standard_normal((128, 16)), kp, vv,
+                         rng.standard_normal((128, 16)), 0.9)
+    assert r.count == 1
+    np.testing.assert_array_equal(r.out, vv[0])
+    r = O.local_head(rng.standard_normal(128), kp, vv, 4, 256)
+    np.testing.assert_array_equal(r.out, vv[0])
+
+
+def test_page_constants():
+    """Constants the pages fix: r = 16, p = 0.9, 256 bins of fp32 mass = 1 KB per head."""
+    with open(os.path.join(GOLDEN, "page_constants.json")) as f:
+        c = json.load(f)
+    assert c["idx_dim"] == O.IDX_DIM
+    assert c["n_bins"] == O.N_BINS
+    assert c["hist_bytes_per_head"] == O.N_BINS * 4
+    assert c["top_p"] == 0.9
