@@ -1,0 +1,30 @@
+"""Builds librtp.so (sm_100a) in-tree with nvcc."""
+from __future__ import annotations
+
+import os
+import subprocess
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+NVCC_FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-O3", "-lineinfo", "-std=c++17",
+              "-shared", "-Xcompiler", "-fPIC", "--expt-relaxed-constexpr"]
+
+
+def nvcc() -> str:
+    for c in (os.environ.get("NVCC"), "/usr/local/cuda/bin/nvcc", "nvcc"):
+        if c and (os.path.sep not in c or os.path.exists(c)):
+            return c
+    return "nvcc"
+
+
+def build(verbose: bool = False, extra_flags=()) -> str:
+    out = os.path.join(HERE, "librtp.so")
+    src = os.path.join(HERE, "csrc", "rtp_api.cu")
+    cmd = [nvcc(), *NVCC_FLAGS, *extra_flags, "-o", out, src]
+    if verbose:
+        print(" ".join(cmd))
+    subprocess.run(cmd, check=True)
+    return out
+
+
+if __name__ == "__main__":
+    print(build(verbose=True))

@@ -218,7 +218,11 @@ def _group_layout(w: Workload, layer: int, b: int, kvh: int) -> GroupLayout:
             targets.append(("diff", list(range(16)), list(rng.uniform(0.5, 1.5, size=16))))
     else:
         raise ValueError(w.kind)
-    starts = _place(rng, [n for n, _ in specs], max(N - 1, 1))
+    avail = max(N - 1, 0)
+    total = sum(n for n, _ in specs)
+    if total > avail:                      # short sequence: shrink the runs to fit
+        specs = [(int(n * avail // total), s) for n, s in specs]
+    starts = _place(rng, [n for n, _ in specs], max(avail, 1))
     W = w.w_kidx(layer)[kvh].astype(np.float64)          # [128][16]
     WtW = W.T @ W
     clusters = []

@@ -1,0 +1,131 @@
+"""GPU parity of the CUDA path against the CPU oracle, through the C ABI (needs a B200)."""
+import dataclasses
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import rtp_oracle as O
+from synth import gen, workloads
+
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda"
+
+
+def _parity():
+    import parity
+    return parity
+
+
+def test_gpu_fill_matches_numpy_stream():
+    from synth.gpu import LayerFiller
+    w = workloads.workload(1)
+    f = LayerFiller(w, 0, DEV)
+    k, v = f.fill(np.array([37]), 300)
+    k = k.view(torch.int16).cpu().numpy().view(np.uint16)
+    v = v.view(torch.int16).cpu().numpy().view(np.uint16)
+    for g in range(w.Hkv):
+        np.testing.assert_array_equal(k[0, :, g], w.kpre_bits(0, 0, g, 37, 337))
+        np.testing.assert_array_equal(v[0, :, g], w.v_bits(0, 0, g, 37, 337))
+    c = w.group_layout(0, 0, 0).clusters[0]                    # a planted run
+    k, _ = f.fill(np.array([c.start - 3]), c.length + 6)
+    k = k.view(torch.int16).cpu().numpy().view(np.uint16)
+    np.testing.assert_array_equal(k[0, :, 0], w.kpre_bits(0, 0, 0, c.start - 3, c.start + c.length + 3))
+
+
+def test_append_matches_oracle_rows():
+    P = _parity()
+    w = workloads.workload(1)
+    q, wq, wk = P.layer_inputs(w, 0, DEV)
+    N = int(w.seq_lens[0])
+    lay = P.make_layer(w, 0, DEV)
+    P.fill_layer(w, 0, lay, wk, [N], chunk=1000, device=DEV)   # ragged chunks
+    torch.cuda.synchronize()
+    assert lay.status() == 0
+    kp = P.bits_to_f64(w.kpre_bits(0, 0, 0, 0, N))
+    vv = P.bits_to_f64(w.v_bits(0, 0, 0, 0, N))
+    k_ref, v_ref, i_ref = O.append_rows(kp, vv, w.w_kidx(0)[0], np.arange(N), w.rope_base)
+    k_gpu = lay.k_ret[0, :N].double().cpu().numpy()
+    i_gpu = lay.idx[0, :N].double().cpu().numpy()
+    v_gpu = lay.v_ret[0, :N].double().cpu().numpy()
+    np.testing.assert_array_equal(v_gpu, v_ref)
+    # RoPE and the projection run in double on both sides: equal bf16 except, at most, values
+    # within one bf16 spacing of a rounding tie
+    for got, ref in ((k_gpu, k_ref), (i_gpu, i_ref)):
+        mism = got != ref
+        assert mism.mean() < 1e-5, mism.sum()
+        if mism.any():
+            ulp = np.ldexp(1.0, np.frexp(ref[mism])[1] - 8)
+            assert np.all(np.abs(got[mism] - ref[mism]) <= ulp)
+    # local ring of KV head 1: row n < sinks -> n; else sinks + (n - sinks) % window
+    kp1 = P.bits_to_f64(w.kpre_bits(0, 0, 1, 0, N))
+    pos = O.local_positions(N, w.sinks, w.window)
+    rows = np.where(pos < w.sinks, pos, w.sinks + (pos - w.sinks) % w.window)
+    k_ref1 = O.bf16_round(O.rope_rotate(kp1[pos], pos, w.rope_base))
+    got1 = lay.k_loc[0, 0].double().cpu().numpy()[rows]
+    assert (got1 != k_ref1).mean() < 1e-5
+
+
+@pytest.mark.parametrize("p", [0.9, 0.5, 0.99, 1.0])
+def test_tiny_layer_parity(p):
+    rep = _parity().run_layer_parity(workload_index=1, layer=0, p=p)
+    assert rep["max_abs"] <= 1e-2
+
+
+def _small(G=4, Hkv=2, B=1, seq=(4096,), sinks=4, window=256, ret=(True, False), kind="mix",
+           lam=(1.65, 2.05)):
+    w = workloads.workload(1)
+    return dataclasses.replace(w, B=B, Hq=G * Hkv, Hkv=Hkv, seq_lens=np.array(seq),
+                               sinks=sinks, window=window,
+                               ret_mask=np.array([list(ret)], bool), kind=kind,
+                               lam_conc=lam[0], lam_diff=lam[1])
+
+
+@pytest.mark.parametrize("G", [1, 2, 4, 8])
+def test_group_sizes(G):
+    w = _small(G=G, seq=(3000,))
+    _parity().run_layer_parity(w=w, layer=0)
+
+
+def test_ragged_batch_and_edge_lengths():
+    """N = 1, N < sinks, N around sinks + window, ragged lengths in one batch."""
+    w = _small(B=6, Hkv=2, seq=(1, 3, 259, 260, 261, 5000), kind="needle")
+    _parity().run_layer_parity(w=w, layer=0)
+
+
+def test_dense_reduction_on_gpu():
+    """p = 1 and window >= N: every head attends every token."""
+    w = _small(seq=(2000,), window=4096)
+    rep = _parity().run_layer_parity(w=w, layer=0, p=1.0)
+    for e in rep["heads"]:
+        assert e["count"] == 2000
+
+
+def test_all_retrieval_and_all_local_layers():
+    _parity().run_layer_parity(w=_small(ret=(True, True), seq=(5000,)), layer=0)
+    _parity().run_layer_parity(w=_small(ret=(False, False), seq=(5000,)), layer=0)
+
+
+def test_device_status_on_bad_seq_len():
+    """seq_lens[b] above seq_cap[b]: the sequence is skipped, the status word says so."""
+    P = _parity()
+    w = _small(B=2, seq=(500, 800))
+    q, wq, wk = P.layer_inputs(w, 0, DEV)
+    lay = P.make_layer(w, 0, DEV, seq_lens=[500, 800], caps=[500, 800])
+    P.fill_layer(w, 0, lay, wk, [500, 800], device=DEV)
+    out, cnt, _ = P.decode(lay, q, wq, [501, 800], 0.9, DEV, with_sel=False)
+    assert lay.status() == -6
+    assert np.all(cnt[0].cpu().numpy() == 0)
+    assert np.all(cnt[1].cpu().numpy() > 0)
+    assert lay.status() == 0                                        # read clears it
+
+
+def test_qwen_layer_32k_parity():
+    """One full Qwen3-8B-shaped layer at N = 32768 (every head), caches from the GPU fill."""
+    w = workloads.workload(2)
+    layer = int(np.nonzero(w.ret_mask.sum(1) >= 2)[0][0])
+    rep = _parity().run_layer_parity(w=w, layer=layer, source="gpu")
+    conc = [e["n_gpu"] for e in rep["heads"] if e["retrieval"] and e["h"] % 2 == 0]
+    diff = [e["n_gpu"] for e in rep["heads"] if e["retrieval"] and e["h"] % 2 == 1]
+    assert conc and diff and np.mean(diff) > 3 * np.mean(conc)
