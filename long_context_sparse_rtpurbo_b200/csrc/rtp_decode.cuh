@@ -571,7 +571,7 @@ __global__ void __launch_bounds__(kThreads) emit_sel_kernel(DecodeParams P, int3
   if (slot < 0) {
     const int s1 = min(N, P.L.sinks);
     const int w0 = max(P.L.sinks, N - P.L.window);
-    const int cnt = s1 + (N - w0);
+    const int cnt = s1 + max(0, N - w0);
     for (int k = threadIdx.x; k < cnt; k += kThreads) dst[k] = k < s1 ? k : w0 + (k - s1);
     return;
   }

@@ -63,10 +63,16 @@ def stream_bits(key: int, counters) -> np.ndarray:
 
 def normal_f32(key: int, counters) -> np.ndarray:
     """Near-normal float32 values (mean 0, variance 1, bounded at about 3.46)."""
-    h = stream_bits(key, counters)
-    s = ((h & U64(0xFFFF)) + ((h >> U64(16)) & U64(0xFFFF)) + ((h >> U64(32)) & U64(0xFFFF))
-         + (h >> U64(48))).astype(np.int64) - IH_CENTRE
-    return s.astype(np.float32) * INV_STD
+    h = np.ascontiguousarray(stream_bits(key, counters))
+    shape = h.shape
+    # the four 16-bit fields of each word (little-endian view), summed exactly in int32
+    f = h.reshape(-1).view(np.uint16).reshape(-1, 4)
+    s = f[:, 0].astype(np.int32)
+    s += f[:, 1]
+    s += f[:, 2]
+    s += f[:, 3]
+    s -= IH_CENTRE
+    return (s.astype(np.float32) * INV_STD).reshape(shape)
 
 
 def f32_to_bf16_bits(x) -> np.ndarray:
@@ -86,8 +92,7 @@ def token_rows_bits(key: int, t0: int, t1: int, dim: int, shifts=None) -> np.nda
     ``shifts`` is an optional list of (start, length, delta float32[dim]): rows inside
     [start, start + length) get ``delta`` added (one float32 addition) before rounding.
     """
-    t = np.arange(t0, t1, dtype=np.int64)
-    c = (t[:, None] * dim + np.arange(dim, dtype=np.int64)[None, :]).astype(np.uint64)
+    c = np.arange(t0 * dim, t1 * dim, dtype=np.uint64).reshape(t1 - t0, dim)
     x = normal_f32(key, c)
     if shifts:
         for (start, length, delta) in shifts:
