@@ -484,10 +484,13 @@ def main(argv=None):
     ap.add_argument("--cpu-budget", type=float, default=12.0)
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--layers", type=int, default=0, help="run only the first N layers")
     ap.add_argument("--preroll", type=float, default=0.6, help="untimed seconds before timing")
     args = ap.parse_args(argv)
     from synth import workloads
     w = workloads.workload(args.workload, args.p)
+    if args.layers:
+        w.layers = min(w.layers, args.layers)
     if args.impl == "reference":
         return run_reference(args, w)
     return run_ours(args, w)

@@ -3,6 +3,7 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <cmath>
 #include <cstring>
 
 #include "../../include/rtp.h"
@@ -14,23 +15,25 @@ namespace {
 
 thread_local int32_t g_launches = 0;
 
-constexpr int kPlanSMs = 148;       // B200 SM count used to size the score chunks
+constexpr int kPlanCTAs = 160;      // upper bound on decode CTAs (one per SM; B200 has 148)
 constexpr int kLocRows = 128;       // ring rows per local attention item
-constexpr int kMaxChunks = 1024;
+constexpr long long kSpinLimit = 2000000000LL;   // ~1 s of SM clock per device-side wait
 
 inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+inline int align16(int x) { return (x + 15) & ~15; }
 
 struct Plan {
   LayerShape L;
-  int C, MC, S, PL, n_groups, n_ret_items, n_loc_items;
+  int C_min, max_nch, NC_max, n_groups, n_lgroups, PL, n_loc_items;
+  int64_t maxN_pad;
   size_t off_ctrl, ctrl_bytes;
-  size_t off_lohi, off_hcnt, off_arr_ret, off_arr_loc, off_hist;
-  size_t off_scores, off_ent, off_ccnt, off_part_ret, off_part_loc, total;
+  size_t off_lohi, off_hcnt, off_bar, off_team, off_locarr, off_misc, off_hist;
+  size_t off_scores, off_ent, off_ccnt, off_part, off_tpart, off_lpart, total;
 };
 
 int check_desc(const rtp_layer_desc* d, LayerShape& L) {
   if (!d || !d->slot_of_kv) return RTP_EINVAL;
-  if (d->B < 1 || d->Hkv < 1 || d->Hkv > kMaxHkv || d->Hq < 1) return RTP_ESHAPE;
+  if (d->B < 1 || d->B > 4096 || d->Hkv < 1 || d->Hkv > kMaxHkv || d->Hq < 1) return RTP_ESHAPE;
   if (d->Hq % d->Hkv != 0) return RTP_ESHAPE;
   const int G = d->Hq / d->Hkv;
   if (G != 1 && G != 2 && G != 4 && G != 8) return RTP_ESHAPE;
@@ -42,6 +45,7 @@ int check_desc(const rtp_layer_desc* d, LayerShape& L) {
   L.B = d->B; L.Hq = d->Hq; L.Hkv = d->Hkv; L.G = G;
   L.sinks = d->sinks; L.window = d->window; L.ring = d->sinks + d->window;
   L.maxN = d->max_seq_len; L.rope_base = d->rope_base;
+  for (int i = 0; i < kD / 2; ++i) L.theta[i] = std::pow(d->rope_base, -2.0 * i / (double)kD);
   bool seen_r[kMaxHkv] = {false}, seen_l[kMaxHkv] = {false};
   int nr = 0, nl = 0;
   for (int g = 0; g < d->Hkv; ++g) {
@@ -69,34 +73,37 @@ int make_plan(const rtp_layer_desc* d, Plan& pl) {
   const int G = L.G;
   const int64_t maxN = L.maxN;
   pl.n_groups = L.B * L.n_ret;
-  // score chunks: about two per SM over all groups, 1K..64K tokens, <= kMaxChunks per group
-  int64_t C = (int64_t(pl.n_groups) * maxN + 2 * kPlanSMs - 1) / (2 * kPlanSMs);
-  C = std::max<int64_t>(C, 1024);
-  C = std::max<int64_t>(C, (maxN + kMaxChunks - 1) / kMaxChunks);
-  C = std::min<int64_t>(C, 65536);
-  C = (C + 255) / 256 * 256;
-  pl.C = (int)C;
-  pl.MC = (int)((maxN + C - 1) / C);
-  if (pl.MC > kMaxChunks) return RTP_ESHAPE;
-  pl.S = (int)std::min<int64_t>(32, std::max<int64_t>(1, maxN / 2048));
+  pl.n_lgroups = L.B * L.n_loc;
+  if (pl.n_groups > 8 * kFThreads) return RTP_ESHAPE;
+  // chunks: at least C_min tokens, so a launch never has more than 8 per CTA plus one per group
+  int64_t cmin = (int64_t(pl.n_groups) * maxN + 8 * kPlanCTAs - 1) / (8 * kPlanCTAs);
+  cmin = std::max<int64_t>(cmin, 256);
+  cmin = (cmin + 255) / 256 * 256;
+  pl.C_min = (int)cmin;
+  pl.max_nch = (int)((maxN + cmin - 1) / cmin);
+  if (pl.max_nch > 8 * kFThreads) return RTP_ESHAPE;
+  pl.NC_max = 8 * kPlanCTAs + pl.n_groups + 16;
+  pl.maxN_pad = (maxN + 63) / 64 * 64;
   const int64_t loc_rows = std::min<int64_t>(maxN, L.ring);
   pl.PL = (int)((loc_rows + kLocRows - 1) / kLocRows);
-  pl.n_ret_items = pl.n_groups * pl.S;
-  pl.n_loc_items = L.B * L.n_loc * pl.PL;
+  pl.n_loc_items = pl.n_lgroups * pl.PL;
+  const size_t part_bytes = sizeof(float) * G * (kD + 2);
   size_t o = 256;                                   // [0, 256): status word
   pl.off_ctrl = o;
-  pl.off_lohi = o; o = align256(o + sizeof(uint32_t) * pl.n_groups * 2 * G);
-  pl.off_hcnt = o; o = align256(o + sizeof(int32_t) * pl.n_groups * G);
-  pl.off_arr_ret = o; o = align256(o + sizeof(uint32_t) * pl.n_groups);
-  pl.off_arr_loc = o; o = align256(o + sizeof(uint32_t) * L.B * L.n_loc);
-  pl.off_hist = o; o = align256(o + sizeof(unsigned long long) * pl.n_groups * G * kBins);
+  pl.off_lohi = o;   o = align256(o + sizeof(uint32_t) * pl.n_groups * 2 * G);
+  pl.off_hcnt = o;   o = align256(o + sizeof(int32_t) * pl.n_groups * G);
+  pl.off_bar = o;    o = align256(o + sizeof(uint32_t) * pl.n_groups * 4);
+  pl.off_team = o;   o = align256(o + sizeof(uint32_t) * pl.NC_max);
+  pl.off_locarr = o; o = align256(o + sizeof(uint32_t) * std::max(pl.n_lgroups, 1));
+  pl.off_misc = o;   o = align256(o + sizeof(uint32_t) * 16);
+  pl.off_hist = o;   o = align256(o + sizeof(unsigned long long) * pl.n_groups * G * kBins);
   pl.ctrl_bytes = o - pl.off_ctrl;
-  const int64_t stride = int64_t(pl.MC) * pl.C;
-  pl.off_scores = o; o = align256(o + sizeof(float) * pl.n_groups * G * stride);
-  pl.off_ent = o; o = align256(o + sizeof(uint32_t) * pl.n_groups * stride);
-  pl.off_ccnt = o; o = align256(o + sizeof(uint32_t) * pl.n_groups * pl.MC);
-  pl.off_part_ret = o; o = align256(o + sizeof(float) * pl.n_ret_items * G * (kD + 2));
-  pl.off_part_loc = o; o = align256(o + sizeof(float) * pl.n_loc_items * G * (kD + 2));
+  pl.off_scores = o; o = align256(o + sizeof(float) * pl.n_groups * G * pl.maxN_pad);
+  pl.off_ent = o;    o = align256(o + sizeof(uint32_t) * pl.n_groups * pl.maxN_pad);
+  pl.off_ccnt = o;   o = align256(o + sizeof(uint32_t) * pl.n_groups * pl.max_nch);
+  pl.off_part = o;   o = align256(o + part_bytes * pl.NC_max);
+  pl.off_tpart = o;  o = align256(o + part_bytes * pl.NC_max);
+  pl.off_lpart = o;  o = align256(o + part_bytes * std::max(pl.n_loc_items, 1));
   pl.total = o;
   return RTP_OK;
 }
@@ -104,30 +111,83 @@ int make_plan(const rtp_layer_desc* d, Plan& pl) {
 template <class T>
 T* at(void* ws, size_t off) { return reinterpret_cast<T*>(static_cast<char*>(ws) + off); }
 
+struct DevInfo {
+  int sms = 0, smem_optin = 0;
+};
+
+int dev_info(DevInfo& di) {
+  static thread_local int cached_dev = -1;
+  static thread_local DevInfo cached;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return RTP_ECUDA;
+  if (dev != cached_dev) {
+    DevInfo x;
+    if (cudaDeviceGetAttribute(&x.sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&x.smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) !=
+            cudaSuccess)
+      return RTP_ECUDA;
+    cached = x;
+    cached_dev = dev;
+  }
+  di = cached;
+  return RTP_OK;
+}
+
+// Shared-memory layout of the decode kernel; returns the bytes, sets C_cap.
+int smem_layout(DecodeParams& P, const Plan& pl, int smem_optin) {
+  const int G = P.L.G;
+  int o = 0;
+  P.sm_attn = o;  o = align16(o + 4 * (16 * G * kD + 2 * 16 * G));
+  P.sm_res = o;   o = align16(o + 4 * G * (kD + 2));
+  P.sm_qret = o;  o = align16(o + 4 * G * kD);
+  P.sm_qloc = o;  o = align16(o + 4 * G * kD);
+  P.sm_qidx = o;  o = align16(o + 4 * G * kR);
+  P.sm_tmp = o;   o = align16(o + 4 * kFThreads);
+  P.sm_hist = o;  o = align16(o + 8 * G * kBins);
+  P.sm_N = o;     o = align16(o + 4 * P.L.B);
+  P.sm_cbase = o; o = align16(o + 4 * (pl.n_groups + 1));
+  P.sm_pref = o;  o = align16(o + 4 * (pl.max_nch + 1));
+  P.sm_int = o;   o = align16(o + 4 * 64);
+  P.sm_scores = o;
+  const int budget = smem_optin - 1024;
+  int cap = (budget - o) / (4 * G);
+  cap = std::min(cap, 16384) / 256 * 256;
+  if (cap < 256) cap = 0;
+  P.C_cap = cap;
+  return o + 4 * G * cap;
+}
+
 template <int G>
-int launch_decode(DecodeParams& P, const Plan& pl, cudaStream_t st, int32_t* sel_idx,
-                  int64_t sel_stride) {
-  int n = 0;
-  if (pl.n_groups > 0) {
-    const dim3 grid(pl.MC, pl.n_groups);
-    score_kernel<G><<<grid, kThreads, 0, st>>>(P); ++n;
-    if (!P.select_all) { hist_kernel<G><<<grid, kThreads, 0, st>>>(P); ++n; }
-    select_kernel<G><<<grid, kThreads, 0, st>>>(P); ++n;
+int launch_decode(DecodeParams& P, const Plan& pl, const DevInfo& di, cudaStream_t st,
+                  int32_t* sel_idx, int64_t sel_stride) {
+  const int smem = smem_layout(P, pl, di.smem_optin);
+  static int attr_smem = -1;              // per template instance
+  if (attr_smem < smem) {
+    if (cudaFuncSetAttribute(decode_kernel<G>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             smem) != cudaSuccess)
+      return RTP_ECUDA;
+    attr_smem = smem;
   }
-  const int items = pl.n_ret_items + pl.n_loc_items;
-  if (items > 0) {
-    const size_t dyn = sizeof(float) * (16 * G * kD + G * (kD + 2));
-    static bool attr_set = false;     // per template instance
-    if (!attr_set) {
-      if (cudaFuncSetAttribute(attend_kernel<G>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               (int)dyn) != cudaSuccess)
-        return RTP_ECUDA;
-      attr_set = true;
-    }
-    attend_kernel<G><<<items, kThreads, dyn, st>>>(P); ++n;
-  }
+  int per_sm = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, decode_kernel<G>, kFThreads, smem) !=
+          cudaSuccess || per_sm < 1)
+    return RTP_ECUDA;
+  P.P = std::min(di.sms, kPlanCTAs);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(P.P);
+  cfg.blockDim = dim3(kFThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeCooperative;
+  attr[0].val.cooperative = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, decode_kernel<G>, P) != cudaSuccess) return RTP_ECUDA;
+  int n = 1;
   if (sel_idx) {
-    emit_sel_kernel<G><<<P.L.B * P.L.Hq, kThreads, 0, st>>>(P, sel_idx, sel_stride); ++n;
+    emit_sel_kernel<G><<<P.L.B * P.L.Hq, kThreads, 0, st>>>(P, sel_idx, sel_stride);
+    ++n;
   }
   g_launches += n;
   return cudaGetLastError() == cudaSuccess ? RTP_OK : RTP_ECUDA;
@@ -189,7 +249,7 @@ int rtp_append_kv(const rtp_layer_desc* desc, const rtp_cache* cache, const uint
   L.T_total = cache->T_total;
   CachePtrs C{cache->k_ret, cache->v_ret, cache->idx, cache->k_loc, cache->v_loc, cache->seq_off,
               cache->seq_cap};
-  const dim3 grid((n_new + kAppendTok - 1) / kAppendTok, L.B);
+  const dim3 grid((n_new + kAppendTok - 1) / kAppendTok, L.B, L.Hkv);
   if (grid.x > 0x7fffffffu || L.B > 65535) return RTP_ESHAPE;
   append_kernel<<<grid, 128, 0, (cudaStream_t)stream>>>(
       L, C, k_pre, v, w_kidx, start_pos, n_new_b, n_new, ws ? static_cast<int*>(ws) : nullptr);
@@ -216,14 +276,19 @@ int rtp_decode_step(const rtp_layer_desc* desc, const rtp_cache* cache, const ui
   if (!ws || ws_bytes < pl.total) return RTP_EWORKSPACE;
   if ((reinterpret_cast<uintptr_t>(ws) & 255) != 0) return RTP_EWORKSPACE;
   cudaStream_t st = (cudaStream_t)stream;
+  DevInfo di;
+  if (dev_info(di) != RTP_OK) return RTP_ECUDA;
   DecodeParams P;
   memset(&P, 0, sizeof(P));
   P.L = L;
   P.L.T_total = cache->T_total;
-  P.C = pl.C; P.MC = pl.MC; P.S = pl.S; P.RL = kLocRows; P.PL = pl.PL;
-  P.n_groups = pl.n_groups; P.n_ret_items = pl.n_ret_items; P.n_loc_items = pl.n_loc_items;
+  P.C_min = pl.C_min; P.max_nch = pl.max_nch; P.NC_max = pl.NC_max;
+  P.n_groups = pl.n_groups; P.n_lgroups = pl.n_lgroups; P.PL = pl.PL; P.RL = kLocRows;
+  P.n_loc_items = pl.n_loc_items;
   P.select_all = p >= 1.0 ? 1 : 0;
   P.p = p;
+  P.spin_limit = kSpinLimit;
+  P.maxN_pad = pl.maxN_pad;
   P.q_pre = q_pre; P.w_qidx = w_qidx; P.seq_lens = seq_lens;
   P.cache = CachePtrs{cache->k_ret, cache->v_ret, cache->idx, cache->k_loc, cache->v_loc,
                       cache->seq_off, cache->seq_cap};
@@ -231,22 +296,25 @@ int rtp_decode_step(const rtp_layer_desc* desc, const rtp_cache* cache, const ui
   P.status = at<int>(ws, 0);
   P.lohi = at<uint32_t>(ws, pl.off_lohi);
   P.hcnt = at<int32_t>(ws, pl.off_hcnt);
-  P.arrive_ret = at<uint32_t>(ws, pl.off_arr_ret);
-  P.arrive_loc = at<uint32_t>(ws, pl.off_arr_loc);
+  P.bar = at<uint32_t>(ws, pl.off_bar);
+  P.team_arr = at<uint32_t>(ws, pl.off_team);
+  P.loc_arr = at<uint32_t>(ws, pl.off_locarr);
+  P.misc = at<uint32_t>(ws, pl.off_misc);
   P.hist = at<unsigned long long>(ws, pl.off_hist);
   P.scores = at<float>(ws, pl.off_scores);
   P.ent = at<uint32_t>(ws, pl.off_ent);
-  P.chunk_cnt = at<uint32_t>(ws, pl.off_ccnt);
-  P.part_ret = at<float>(ws, pl.off_part_ret);
-  P.part_loc = at<float>(ws, pl.off_part_loc);
+  P.ccnt = at<uint32_t>(ws, pl.off_ccnt);
+  P.part = at<float>(ws, pl.off_part);
+  P.tpart = at<float>(ws, pl.off_tpart);
+  P.lpart = at<float>(ws, pl.off_lpart);
   if (cudaMemsetAsync(at<char>(ws, pl.off_ctrl), 0, pl.ctrl_bytes, st) != cudaSuccess)
     return RTP_ECUDA;
   int r;
   switch (L.G) {
-    case 1: r = launch_decode<1>(P, pl, st, sel_idx, sel_stride); break;
-    case 2: r = launch_decode<2>(P, pl, st, sel_idx, sel_stride); break;
-    case 4: r = launch_decode<4>(P, pl, st, sel_idx, sel_stride); break;
-    default: r = launch_decode<8>(P, pl, st, sel_idx, sel_stride); break;
+    case 1: r = launch_decode<1>(P, pl, di, st, sel_idx, sel_stride); break;
+    case 2: r = launch_decode<2>(P, pl, di, st, sel_idx, sel_stride); break;
+    case 4: r = launch_decode<4>(P, pl, di, st, sel_idx, sel_stride); break;
+    default: r = launch_decode<8>(P, pl, di, st, sel_idx, sel_stride); break;
   }
   return r;
 }

@@ -1,42 +1,57 @@
-// Decode step of one layer: index scoring, 256-bin top-p threshold, selection, and exact
-// softmax attention over the selected rows (retrieval heads) or the sinks + window (local
-// heads).
+// Decode step of one layer in one persistent kernel: index scoring, the 256-bin top-p
+// threshold, selection, and exact softmax attention over the selected rows (retrieval heads)
+// or over the sinks + window (local heads).
 //
 // "Full Attention Strikes Back" (paper text) §3.2: eq. (4) s(m,n) = (W^Q q^pre)^T (W^K k^pre),
 // eq. (5) O = sum over S of softmax(q^T k / sqrt(d)) v with S = Top-P(s, p); local heads use
 // attention sinks plus a sliding window. MCISLAB DeepRead notes on RTPurbo, "Method": top-p
 // is found sort-free with a 256-bin histogram per head, fused with the scoring.
 //
-// Phases (one kernel each in this file, all on the caller's stream):
-//   score  : per chunk of C tokens of a (sequence, retrieval KV head) group, the G query
-//            heads' index scores -> workspace; group min / max through integer atomics.
-//   hist   : per chunk, the 256-bin mass histogram exp(s - max) of each head -> group
-//            histogram (exact 2^-40 fixed point, order independent).
-//   select : per chunk, b* of each head from the group histogram; tokens whose bin >= b* for
-//            any head of the group are compacted, in ascending order, into entries
-//            (n << 8 | head mask); per-chunk entry counts.
-//   attend : split-KV attention. Retrieval items take an equal share of the group's entries
-//            (each K/V row is read once for all G heads of the group, heads that did not
-//            select the row skip it); local items take a slice of the ring. Each item writes
-//            (max, sum, acc[128]) per head; the last item of a group merges them.
+// Work split. A retrieval group is one (sequence, retrieval KV head) with its G query heads;
+// its N tokens are cut into chunks of C tokens; chunk k of the launch runs on CTA k mod P.
+// Per group the chunks pass four phases, separated by arrival counters in global memory:
+//   S  scores of the G heads for the chunk's tokens (kept in shared memory when every CTA
+//      owns at most one chunk, else in the workspace); group min / max by integer atomics.
+//   H  the chunk's 256-bin mass histogram exp(s - max) per head, added to the group's
+//      histogram in 2^-40 fixed point (exact and order independent).
+//   T  b* per head from the group histogram; tokens whose bin >= b* for any head are
+//      compacted in ascending order into entries (n << 8 | head mask); counts.
+//   W  the group's entries are split evenly over its chunks' CTAs; each gathers its rows
+//      once for all G heads (a head that did not select a row skips it) and writes a
+//      partial softmax state; partials merge in teams of 16, the last team writes out.
+// Local items (a slice of one local head's ring) come from a global queue; a CTA takes one
+// whenever it would otherwise wait for a counter, and drains the queue at the end.
+// Every wait is bounded (clock64 limit): on expiry the kernel records RTP_ETIMEOUT, raises
+// an abort flag that ends every other wait, and returns.
 #pragma once
 
 #include "rtp_append.cuh"
+#include "rtp_attend.cuh"
 
 namespace rtp {
 
+constexpr int kFThreads = 512;          // threads of the decode kernel
+constexpr int kTeam = 16;               // partials merged per team
+
 struct DecodeParams {
   LayerShape L;
-  int C;           // tokens per score chunk
-  int MC;          // chunks per group (upper bound)
-  int S;           // attention splits per retrieval group
-  int RL;          // ring rows per local item
-  int PL;          // local items per (sequence, local head)
-  int n_groups;    // B * n_ret
-  int n_ret_items; // n_groups * S
-  int n_loc_items; // B * n_loc * PL
-  int select_all;  // p >= 1
+  int P;             // CTAs of the launch
+  int C_min;         // smallest chunk (tokens), bounds the chunk count
+  int C_cap;         // chunk tokens whose scores fit the shared-memory score buffer
+  int max_nch;       // chunks per group upper bound (shared array size)
+  int NC_max;        // chunks per launch upper bound (workspace arrays)
+  int n_groups;      // B * n_ret
+  int n_lgroups;     // B * n_loc
+  int PL;            // local items per local group
+  int RL;            // ring rows per local item
+  int n_loc_items;
+  int select_all;    // p >= 1
   double p;
+  long long spin_limit;
+  int64_t maxN_pad;
+  // shared-memory layout (byte offsets into the dynamic buffer)
+  int sm_scores, sm_attn, sm_res, sm_qret, sm_qloc, sm_qidx, sm_tmp, sm_hist, sm_N, sm_cbase,
+      sm_pref, sm_int;
   // inputs / outputs
   const uint16_t* q_pre;
   const float* w_qidx;
@@ -46,18 +61,22 @@ struct DecodeParams {
   int32_t* sel_counts;
   // workspace
   int* status;
-  uint32_t* lohi;              // [n_groups][2][G]   (~ord(min), ord(max)), zeroed per call
-  int32_t* hcnt;               // [n_groups][G]      selected tokens per head, zeroed
-  uint32_t* arrive_ret;        // [n_groups]         zeroed
-  uint32_t* arrive_loc;        // [B * n_loc]        zeroed
-  unsigned long long* hist;    // [n_groups][G][256] zeroed
-  float* scores;               // [n_groups][G][MC * C]
-  uint32_t* ent;               // [n_groups][MC * C]
-  uint32_t* chunk_cnt;         // [n_groups][MC]
-  float* part_ret;             // [n_ret_items][G][2 + 128]
-  float* part_loc;             // [n_loc_items][G][2 + 128]
+  uint32_t* lohi;              // [n_groups][2][G]   ~ord(min), ord(max)        (zeroed)
+  int32_t* hcnt;               // [n_groups][G]      selected tokens per head    (zeroed)
+  uint32_t* bar;               // [n_groups][4]      phase arrivals, teams done  (zeroed)
+  uint32_t* team_arr;          // [NC_max]           team arrivals              (zeroed)
+  uint32_t* loc_arr;           // [n_lgroups]        local item arrivals        (zeroed)
+  uint32_t* misc;              // [0] local queue head, [1] abort, [2] chunk size (zeroed)
+  unsigned long long* hist;    // [n_groups][G][256]                            (zeroed)
+  float* scores;               // [n_groups][G][maxN_pad] (when chunks do not fit on chip)
+  uint32_t* ent;               // [n_groups][maxN_pad]
+  uint32_t* ccnt;              // [n_groups][max_nch]
+  float* part;                 // [NC_max][G][130]
+  float* tpart;                // [NC_max][G][130]
+  float* lpart;                // [n_loc_items][G][130]
 };
 
+// ------------------------------------------------------------------------------ helpers
 __device__ __forceinline__ int seq_len_checked(const DecodeParams& P, int b) {
   const int N = P.seq_lens[b];
   if (N < 1 || N > P.cache.seq_cap[b] || (int64_t)N > P.L.maxN) return 0;
@@ -65,101 +84,139 @@ __device__ __forceinline__ int seq_len_checked(const DecodeParams& P, int b) {
   return N;
 }
 
-// Index score of one token: fixed order of fused multiply-adds (identical in every phase).
-template <int G>
-__device__ __forceinline__ void score_row(const float (&qi)[G][kR], const uint4& a,
-                                          const uint4& c, float (&s)[G]) {
-  float x[16];
-  unpack8(a, x);
-  unpack8(c, x + 8);
-#pragma unroll
-  for (int h = 0; h < G; ++h) {
-    float acc = 0.f;
-#pragma unroll
-    for (int j = 0; j < kR; ++j) acc = fmaf(qi[h][j], x[j], acc);
-    s[h] = acc;
-  }
+__device__ __forceinline__ uint32_t ld_acquire(const uint32_t* p) {
+  uint32_t v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
 }
 
-// q_idx = W_qidx[h]^T q_pre[b][h] for the G query heads of KV head kvh, into smem.
-template <int G>
-__device__ __forceinline__ void index_query(const DecodeParams& P, int b, int kvh,
-                                            float (*qi)[kR]) {
-  const int t = threadIdx.x;
-  if (t < G * kR) {
-    const int h = kvh * G + t / kR, j = t % kR;
-    const uint16_t* q = P.q_pre + ((int64_t)b * P.L.Hq + h) * kD;
-    const float* w = P.w_qidx + (int64_t)h * kD * kR + j;
-    float acc = 0.f;
-    for (int i = 0; i < kD; ++i) acc = fmaf(bf1(q[i]), __ldg(w + i * kR), acc);
-    qi[t / kR][j] = acc;
-  }
-}
-
-// ------------------------------------------------------------------------------ score
-template <int G>
-__global__ void __launch_bounds__(kThreads) score_kernel(DecodeParams P) {
-  const int c = blockIdx.x, gr = blockIdx.y;
-  const int b = gr / P.L.n_ret, r = gr % P.L.n_ret;
-  const int N = seq_len_checked(P, b);
-  const int n0 = c * P.C;
-  if (n0 >= N) return;
-  const int n1 = min(N, n0 + P.C);
-  const int kvh = P.L.ret_kv[r];
-  __shared__ float qs[G][kR];
-  __shared__ float red[2][G][kThreads / 32];
-  index_query<G>(P, b, kvh, qs);
-  __syncthreads();
-  float qi[G][kR];
-#pragma unroll
-  for (int h = 0; h < G; ++h)
-#pragma unroll
-    for (int j = 0; j < kR; ++j) qi[h][j] = qs[h][j];
-  float mn[G], mx[G];
-#pragma unroll
-  for (int h = 0; h < G; ++h) { mn[h] = INFINITY; mx[h] = -INFINITY; }
-  const uint16_t* idx = P.cache.idx + ((int64_t)r * P.L.T_total + P.cache.seq_off[b]) * kR;
-  const int64_t stride = (int64_t)P.MC * P.C;
-  float* sc = P.scores + (int64_t)gr * G * stride;
-  for (int n = n0 + threadIdx.x; n < n1; n += kThreads) {
-    const uint4 a = ld_stream(idx + (int64_t)n * kR);
-    const uint4 d = ld_stream(idx + (int64_t)n * kR + 8);
-    float s[G];
-    score_row<G>(qi, a, d, s);
-#pragma unroll
-    for (int h = 0; h < G; ++h) {
-      sc[h * stride + n] = s[h];
-      mn[h] = fminf(mn[h], s[h]);
-      mx[h] = fmaxf(mx[h], s[h]);
-    }
-  }
+__device__ __forceinline__ int block_sum_int(int v, int* scratch /*>= 32 ints*/) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
 #pragma unroll
-  for (int h = 0; h < G; ++h) {
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  __syncthreads();
+  if (lane == 0) scratch[warp] = v;
+  __syncthreads();
+  int s = 0;
+  for (int w = 0; w < kFThreads / 32; ++w) s += scratch[w];
+  __syncthreads();
+  return s;
+}
+
+// Exclusive scan of n ints in smem (in place), n <= kFThreads * 8; returns the total.
+__device__ __forceinline__ int block_scan_excl(int* a, int n, int* scratch /*>= 32*/) {
+  const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
+  constexpr int PER = 8;
+  int v[PER], local = 0;
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-      mn[h] = fminf(mn[h], __shfl_xor_sync(0xffffffffu, mn[h], o));
-      mx[h] = fmaxf(mx[h], __shfl_xor_sync(0xffffffffu, mx[h], o));
-    }
-    if (lane == 0) { red[0][h][warp] = mn[h]; red[1][h][warp] = mx[h]; }
+  for (int i = 0; i < PER; ++i) {
+    const int idx = t * PER + i;
+    v[i] = idx < n ? a[idx] : 0;
+    local += v[i];
+  }
+  int incl = local;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += y;
   }
   __syncthreads();
-  if (threadIdx.x < G) {
-    const int h = threadIdx.x;
-    float a = red[0][h][0], z = red[1][h][0];
-    for (int w = 1; w < kThreads / 32; ++w) { a = fminf(a, red[0][h][w]); z = fmaxf(z, red[1][h][w]); }
-    atomicMax(P.lohi + ((int64_t)gr * 2 + 0) * G + h, ~f2ord(a));
-    atomicMax(P.lohi + ((int64_t)gr * 2 + 1) * G + h, f2ord(z));
+  if (lane == 31) scratch[warp] = incl;
+  __syncthreads();
+  int wbase = 0, total = 0;
+  for (int w = 0; w < kFThreads / 32; ++w) {
+    const int x = scratch[w];
+    wbase += (w < warp) ? x : 0;
+    total += x;
+  }
+  int run = wbase + incl - local;
+#pragma unroll
+  for (int i = 0; i < PER; ++i) {
+    const int idx = t * PER + i;
+    if (idx < n) a[idx] = run;
+    run += v[i];
+  }
+  __syncthreads();
+  return total;
+}
+
+// Last index i in [0, n) with a[i] <= key (a non-decreasing, a[0] <= key).
+__device__ __forceinline__ int upper_index(const int* a, int n, int key) {
+  int lo = 0, hi = n - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (a[mid] <= key) lo = mid; else hi = mid - 1;
+  }
+  return lo;
+}
+
+template <int G> struct Smem {
+  float* scores; float* attn; float* res; float* qret; float* qloc; float* qidx; float* tmp;
+  unsigned long long* hist; int* N; int* cbase; int* pref; int* ints;
+  __device__ Smem(unsigned char* base, const DecodeParams& P)
+      : scores((float*)(base + P.sm_scores)), attn((float*)(base + P.sm_attn)),
+        res((float*)(base + P.sm_res)), qret((float*)(base + P.sm_qret)),
+        qloc((float*)(base + P.sm_qloc)), qidx((float*)(base + P.sm_qidx)),
+        tmp((float*)(base + P.sm_tmp)), hist((unsigned long long*)(base + P.sm_hist)),
+        N((int*)(base + P.sm_N)), cbase((int*)(base + P.sm_cbase)), pref((int*)(base + P.sm_pref)),
+        ints((int*)(base + P.sm_int)) {}
+};
+// ints[]: [0..31] reduction scratch, [32] wait flag, [33] local item, [34] local queue empty,
+//         [40..47] b*, [48..50] last-arrival flags
+
+// RoPE'd, pre-scaled query of the G heads of KV head kvh at position N - 1 -> q_s[G][128].
+template <int G>
+__device__ __forceinline__ void rope_query(const DecodeParams& P, int b, int kvh, int N,
+                                           float* q_s) {
+  const int t = threadIdx.x;
+  if (t < kD) {
+    const int i = t & 63;
+    double sn, cs;
+    rope_sincos((double)(N - 1), P.L.theta[i], &sn, &cs);
+    const float scale = kLog2e * 0.08838834764831845f;   // log2(e) / sqrt(128)
+#pragma unroll
+    for (int h = 0; h < G; ++h) {
+      const uint16_t* q = P.q_pre + ((int64_t)b * P.L.Hq + kvh * G + h) * kD;
+      const double qa = bf1(q[i]), qb = bf1(q[i + 64]);
+      const double r = (t < 64) ? (qa * cs - qb * sn) : (qa * sn + qb * cs);
+      q_s[h * kD + t] = (float)r * scale;
+    }
   }
 }
 
+// q_idx[h][j] = W_qidx[h]^T q_pre[b][h] for the G heads of kvh; fixed summation order.
 template <int G>
-__device__ __forceinline__ void load_range(const DecodeParams& P, int gr, float* lo, float* hi,
+__device__ __forceinline__ void index_query(const DecodeParams& P, int b, int kvh, float* qidx,
+                                            float* tmp) {
+  constexpr int NO = G * kR;
+  constexpr int NPART = kFThreads / NO;
+  constexpr int DPP = kD / NPART;
+  const int t = threadIdx.x;
+  const int o = t % NO, part = t / NO;
+  const int h = kvh * G + o / kR, j = o % kR;
+  const uint16_t* q = P.q_pre + ((int64_t)b * P.L.Hq + h) * kD + part * DPP;
+  const float* w = P.w_qidx + ((int64_t)h * kD + part * DPP) * kR + j;
+  float acc = 0.f;
+#pragma unroll
+  for (int i = 0; i < DPP; ++i) acc = fmaf(bf1(q[i]), __ldg(w + i * kR), acc);
+  __syncthreads();
+  tmp[part * NO + o] = acc;
+  __syncthreads();
+  if (t < NO) {
+    float s = tmp[t];
+    for (int pp = 1; pp < NPART; ++pp) s += tmp[pp * NO + t];
+    qidx[t] = s;
+  }
+  __syncthreads();
+}
+
+template <int G>
+__device__ __forceinline__ void load_range(const DecodeParams& P, int g, float* lo, float* hi,
                                            float* inv) {
 #pragma unroll
   for (int h = 0; h < G; ++h) {
-    lo[h] = ord2f(~P.lohi[((int64_t)gr * 2 + 0) * G + h]);
-    hi[h] = ord2f(P.lohi[((int64_t)gr * 2 + 1) * G + h]);
+    lo[h] = ord2f(~__ldcg(P.lohi + ((int64_t)g * 2 + 0) * G + h));
+    hi[h] = ord2f(__ldcg(P.lohi + ((int64_t)g * 2 + 1) * G + h));
     inv[h] = (hi[h] > lo[h] && !P.select_all) ? (float)kBins / (hi[h] - lo[h]) : 0.f;
   }
 }
@@ -168,391 +225,472 @@ __device__ __forceinline__ int bin_of(float s, float lo, float inv) {
   return min(kBins - 1, (int)((s - lo) * inv));
 }
 
-// ------------------------------------------------------------------------------ hist
+// ------------------------------------------------------------------------------ kernel
 template <int G>
-__global__ void __launch_bounds__(kThreads) hist_kernel(DecodeParams P) {
-  const int c = blockIdx.x, gr = blockIdx.y;
-  const int b = gr / P.L.n_ret;
-  const int N = seq_len_checked(P, b);
-  const int n0 = c * P.C;
-  if (n0 >= N || P.select_all) return;
-  const int n1 = min(N, n0 + P.C);
-  __shared__ unsigned long long hs[G][kBins];
-  for (int i = threadIdx.x; i < G * kBins; i += kThreads) (&hs[0][0])[i] = 0ull;
-  float lo[G], hi[G], inv[G];
-  load_range<G>(P, gr, lo, hi, inv);
-  __syncthreads();
-  const int64_t stride = (int64_t)P.MC * P.C;
-  const float* sc = P.scores + (int64_t)gr * G * stride;
-  for (int n = n0 + threadIdx.x; n < n1; n += kThreads) {
-#pragma unroll
-    for (int h = 0; h < G; ++h) {
-      const float s = sc[h * stride + n];
-      const float m = exp2f((s - hi[h]) * kLog2e);
-      const unsigned long long q = __float2ull_rn(m * kMassScale);
-      if (q) atomicAdd(&hs[h][bin_of(s, lo[h], inv[h])], q);
-    }
-  }
-  __syncthreads();
-  unsigned long long* gh = P.hist + (int64_t)gr * G * kBins;
-  for (int i = threadIdx.x; i < G * kBins; i += kThreads) {
-    const unsigned long long v = (&hs[0][0])[i];
-    if (v) atomicAdd(gh + i, v);
-  }
-}
+struct DecodeCta {
+  const DecodeParams& P;
+  Smem<G> sm;
+  int C, NC, smem_mode;
 
-// b* of the G heads of a group from its histogram; warp h < G handles head h.
-template <int G>
-__device__ __forceinline__ void find_bstar(const DecodeParams& P, int gr, int* bstar) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  if (warp < G) {
-    const int h = warp;
-    if (P.select_all) {
-      if (lane == 0) bstar[h] = 0;
-      return;
-    }
-    const unsigned long long* gh = P.hist + ((int64_t)gr * G + h) * kBins;
-    unsigned long long v[8], tot = 0;
-#pragma unroll
-    for (int e = 0; e < 8; ++e) { v[e] = gh[lane * 8 + e]; tot += v[e]; }
-    // x = inclusive suffix sum of the lane totals (this lane and every higher lane)
-    unsigned long long x = tot;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const unsigned long long y = __shfl_down_sync(0xffffffffu, x, o);
-      if (lane + o < 32) x += y;
-    }
-    const unsigned long long above = x - tot;
-    const unsigned long long T = __shfl_sync(0xffffffffu, x, 0);
-    const double thr = P.p * (double)T;
-    int best = -1;
-    unsigned long long cum = above;
-#pragma unroll
-    for (int e = 7; e >= 0; --e) {
-      cum += v[e];
-      if (best < 0 && (double)cum >= thr) best = lane * 8 + e;
-    }
-    // b* = largest bin b with C_b >= p T: the largest candidate over lanes
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) best = max(best, __shfl_xor_sync(0xffffffffu, best, o));
-    if (lane == 0) bstar[h] = best < 0 ? 0 : best;
-  }
-}
+  __device__ DecodeCta(const DecodeParams& p, unsigned char* base) : P(p), sm(base, p) {}
 
-// ------------------------------------------------------------------------------ select
-template <int G>
-__global__ void __launch_bounds__(kThreads) select_kernel(DecodeParams P) {
-  const int c = blockIdx.x, gr = blockIdx.y;
-  const int b = gr / P.L.n_ret;
-  const int N = seq_len_checked(P, b);
-  const int n0 = c * P.C;
-  if (n0 >= N) return;
-  const int n1 = min(N, n0 + P.C);
-  __shared__ int bstar[G];
-  __shared__ int wsum[kThreads / 32];
-  __shared__ int hsum[G];
-  __shared__ int base;
-  float lo[G], hi[G], inv[G];
-  load_range<G>(P, gr, lo, hi, inv);
-  find_bstar<G>(P, gr, bstar);
-  if (threadIdx.x < G) hsum[threadIdx.x] = 0;
-  if (threadIdx.x == 0) base = 0;
-  __syncthreads();
-  int bs[G];
-#pragma unroll
-  for (int h = 0; h < G; ++h) bs[h] = bstar[h];
-  const int64_t stride = (int64_t)P.MC * P.C;
-  const float* sc = P.scores + (int64_t)gr * G * stride;
-  uint32_t* ent = P.ent + (int64_t)gr * stride + n0;
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  int hc[G];
-#pragma unroll
-  for (int h = 0; h < G; ++h) hc[h] = 0;
-  for (int nb = n0; nb < n1; nb += kThreads) {
-    const int n = nb + threadIdx.x;
-    uint32_t mask = 0;
-    if (n < n1) {
-#pragma unroll
-      for (int h = 0; h < G; ++h) {
-        const float s = sc[h * stride + n];
-        if (bin_of(s, lo[h], inv[h]) >= bs[h]) { mask |= 1u << h; hc[h]++; }
+  __device__ __forceinline__ int group_of(int k) const { return upper_index(sm.cbase, P.n_groups, k); }
+  __device__ __forceinline__ int nch(int g) const { return sm.cbase[g + 1] - sm.cbase[g]; }
+  __device__ __forceinline__ int gN(int g) const { return sm.N[g / P.L.n_ret]; }
+
+  __device__ __forceinline__ float* score_ptr(int g, int j) const {
+    return smem_mode ? sm.scores : P.scores + (int64_t)g * G * P.maxN_pad + (int64_t)j * C;
+  }
+  __device__ __forceinline__ int64_t score_hstride() const {
+    return smem_mode ? (int64_t)P.C_cap : P.maxN_pad;
+  }
+
+  // arrival on a counter after this CTA's writes
+  __device__ __forceinline__ void arrive(uint32_t* ctr) {
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      __threadfence();
+      atomicAdd(ctr, 1u);
+    }
+  }
+
+  // Waits until *ctr >= target, running local items meanwhile. false on timeout / abort.
+  __device__ bool wait_for(const uint32_t* ctr, uint32_t target) {
+    const long long t0 = clock64();
+    volatile uint32_t* abort_flag = P.misc + 1;
+    while (true) {
+      if (threadIdx.x == 0) {
+        int f = 0;
+        if (ld_acquire(ctr) >= target) {
+          f = 1;
+        } else if (*abort_flag) {
+          f = 2;
+        } else if (clock64() - t0 > P.spin_limit) {
+          set_status(P.status, -5);
+          *abort_flag = 1u;
+          __threadfence();
+          f = 2;
+        }
+        if (f == 1) __threadfence();
+        sm.ints[32] = f;
+      }
+      __syncthreads();
+      const int f = sm.ints[32];
+      __syncthreads();
+      if (f == 1) return true;
+      if (f == 2) return false;
+      if (!local_item()) {
+        if (threadIdx.x == 0) __nanosleep(200);
       }
     }
-    const uint32_t bal = __ballot_sync(0xffffffffu, mask != 0);
-    if (lane == 0) wsum[warp] = __popc(bal);
-    __syncthreads();
-    int before = 0, total = 0;
-    for (int w = 0; w < kThreads / 32; ++w) {
-      const int x = wsum[w];
-      before += (w < warp) ? x : 0;
-      total += x;
-    }
-    if (mask) ent[base + before + __popc(bal & ((1u << lane) - 1u))] = ((uint32_t)n << 8) | mask;
-    __syncthreads();
-    if (threadIdx.x == 0) base += total;
-    __syncthreads();
   }
-#pragma unroll
-  for (int h = 0; h < G; ++h) {
-    int v = hc[h];
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-    if (lane == 0 && v) atomicAdd(&hsum[h], v);
-  }
-  __syncthreads();
-  if (threadIdx.x == 0) P.chunk_cnt[(int64_t)gr * P.MC + c] = (uint32_t)base;
-  if (threadIdx.x < G && hsum[threadIdx.x])
-    atomicAdd(P.hcnt + (int64_t)gr * G + threadIdx.x, hsum[threadIdx.x]);
-}
 
-// ------------------------------------------------------------------------------ attend
-// RoPE'd, pre-scaled query of the G heads of KV head kvh at position m = N - 1, into smem.
-template <int G>
-__device__ __forceinline__ void rope_query(const DecodeParams& P, int b, int kvh, int N,
-                                           float (*qs)[kD]) {
-  const int t = threadIdx.x;
-  if (t < kD) {
-    const int i = t & 63;
-    const double th = pow(P.L.rope_base, -2.0 * (double)i / (double)kD);
-    double sn, cs;
-    sincos((double)(N - 1) * th, &sn, &cs);
-    const float scale = kLog2e * 0.08838834764831845f;   // log2(e) / sqrt(128)
-#pragma unroll
-    for (int h = 0; h < G; ++h) {
-      const uint16_t* q = P.q_pre + ((int64_t)b * P.L.Hq + kvh * G + h) * kD;
-      const double qa = bf1(q[i]), qb = bf1(q[i + 64]);
-      const double r = (t < 64) ? (qa * cs - qb * sn) : (qa * sn + qb * cs);
-      qs[h][t] = (float)r * scale;
+  // ------------------------------------------------------------ plan (every CTA identical)
+  __device__ void plan() {
+    const int t = threadIdx.x;
+    for (int b = t; b < P.L.B; b += kFThreads) sm.N[b] = seq_len_checked(P, b);
+    __syncthreads();
+    int part = 0;
+    for (int b = t; b < P.L.B; b += kFThreads) part += sm.N[b];
+    const long long Tr = (long long)block_sum_int(part, sm.ints) * P.L.n_ret;
+    long long c = 256;
+    smem_mode = 0;
+    if (P.P > P.n_groups && Tr > 0) {
+      c = (Tr + (P.P - P.n_groups) - 1) / (P.P - P.n_groups);
+      c = max(c, (long long)P.C_min);
+      c = (c + 255) / 256 * 256;
+      if (c <= P.C_cap) smem_mode = 1;
     }
+    if (!smem_mode) {
+      c = (Tr + 2LL * P.P - 1) / (2LL * P.P);
+      c = max(c, (long long)max(P.C_min, 256));
+      c = (c + 255) / 256 * 256;
+    }
+    C = (int)c;
+    for (int g = t; g < P.n_groups; g += kFThreads) sm.cbase[g] = (gN(g) + C - 1) / C;
+    __syncthreads();
+    NC = block_scan_excl(sm.cbase, P.n_groups, sm.ints);
+    if (t == 0) sm.cbase[P.n_groups] = NC;
+    if (blockIdx.x == 0 && t == 0) P.misc[2] = (uint32_t)C;
+    // invalid sequences: zero their outputs once (CTA 0) and record the status
+    if (blockIdx.x == 0) {
+      for (int b = 0; b < P.L.B; ++b) {
+        if (sm.N[b] != 0) continue;
+        for (int o = t; o < P.L.Hq * kD; o += kFThreads) P.out[(int64_t)b * P.L.Hq * kD + o] = 0;
+        for (int o = t; o < P.L.Hq; o += kFThreads) P.sel_counts[(int64_t)b * P.L.Hq + o] = 0;
+        if (t == 0) set_status(P.status, -6);
+      }
+    }
+    __syncthreads();
   }
-}
 
-struct AttnSmem {
-  float m[16][8];
-  float l[16][8];
-};
-
-// Online-softmax attention of G heads over rows given by `row(i, &kp, &vp, &mask)`, i < nrows.
-// Half-warp per row, lane owns 8 channels. Result: per-head (M, L, A[128]) in `res`
-// ([G][2 + 128], shared memory). Log2 domain: logits carry log2(e) / sqrt(d).
-template <int G, class RowFn>
-__device__ __forceinline__ void attend_rows(const float (*qs)[kD], int nrows, RowFn row,
-                                            float* acc_smem /*[16][G][128]*/, AttnSmem& sm,
-                                            float* res /*[G][130]*/) {
-  const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
-  const int hl = lane & 15, hw = t >> 4;
-  float q[G][8];
-#pragma unroll
-  for (int h = 0; h < G; ++h)
-#pragma unroll
-    for (int e = 0; e < 8; ++e) q[h][e] = qs[h][hl * 8 + e];
-  float m[G], l[G], acc[G][8];
-#pragma unroll
-  for (int h = 0; h < G; ++h) {
-    m[h] = -INFINITY;
-    l[h] = 0.f;
-#pragma unroll
-    for (int e = 0; e < 8; ++e) acc[h][e] = 0.f;
-  }
-  for (int base = warp * 2; base < nrows; base += kThreads / 16) {
-    const int i = base + (lane >> 4);
-    const bool valid = i < nrows;
-    const uint16_t *kp = nullptr, *vp = nullptr;
-    uint32_t mask = 0;
-    if (valid) row(i, kp, vp, mask);
-    uint4 kw = make_uint4(0, 0, 0, 0), vw = make_uint4(0, 0, 0, 0);
-    if (valid) {
-      kw = ld_stream(kp + hl * 8);
-      vw = ld_stream(vp + hl * 8);
-    }
-    float k[8], v[8];
-    unpack8(kw, k);
-    unpack8(vw, v);
-    float d[G];
-#pragma unroll
-    for (int h = 0; h < G; ++h) {
-      float a = 0.f;
-#pragma unroll
-      for (int e = 0; e < 8; ++e) a = fmaf(q[h][e], k[e], a);
-      d[h] = a;
-    }
+  // ------------------------------------------------------------ phase S
+  __device__ void phase_score(int k) {
+    const int g = group_of(k), j = k - sm.cbase[g];
+    const int b = g / P.L.n_ret, r = g % P.L.n_ret, kvh = P.L.ret_kv[r];
+    const int N = gN(g);
+    const int n0 = j * C, n1 = min(N, n0 + C);
+    index_query<G>(P, b, kvh, sm.qidx, sm.tmp);
+    float qi[G][kR];
 #pragma unroll
     for (int h = 0; h < G; ++h)
 #pragma unroll
-      for (int o = 8; o > 0; o >>= 1) d[h] += __shfl_xor_sync(0xffffffffu, d[h], o);
+      for (int jj = 0; jj < kR; ++jj) qi[h][jj] = sm.qidx[h * kR + jj];
+    float mn[G], mx[G];
+#pragma unroll
+    for (int h = 0; h < G; ++h) { mn[h] = INFINITY; mx[h] = -INFINITY; }
+    const uint16_t* idx = P.cache.idx + ((int64_t)r * P.L.T_total + P.cache.seq_off[b]) * kR;
+    float* sc = score_ptr(g, j);
+    const int64_t hs = score_hstride();
+    constexpr int U = 4;
+    for (int nb = n0 + threadIdx.x; nb < n1; nb += U * kFThreads) {
+      uint4 a[U], c2[U];
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const int n = nb + u * kFThreads;
+        if (n < n1) {
+          a[u] = ld_stream(idx + (int64_t)n * kR);
+          c2[u] = ld_stream(idx + (int64_t)n * kR + 8);
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const int n = nb + u * kFThreads;
+        if (n < n1) {
+          float x[16];
+          unpack8(a[u], x);
+          unpack8(c2[u], x + 8);
+#pragma unroll
+          for (int h = 0; h < G; ++h) {
+            float acc = 0.f;
+#pragma unroll
+            for (int jj = 0; jj < kR; ++jj) acc = fmaf(qi[h][jj], x[jj], acc);
+            sc[h * hs + (n - n0)] = acc;
+            mn[h] = fminf(mn[h], acc);
+            mx[h] = fmaxf(mx[h], acc);
+          }
+        }
+      }
+    }
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    float* red = sm.tmp;                    // [2][G][16]
+    __syncthreads();
 #pragma unroll
     for (int h = 0; h < G; ++h) {
-      if (valid && (mask >> h) & 1u) {
-        const float mn = fmaxf(m[h], d[h]);
-        const float cf = exp2f(m[h] - mn);
-        const float pr = exp2f(d[h] - mn);
-        l[h] = l[h] * cf + pr;
 #pragma unroll
-        for (int e = 0; e < 8; ++e) acc[h][e] = fmaf(pr, v[e], acc[h][e] * cf);
-        m[h] = mn;
+      for (int o = 16; o > 0; o >>= 1) {
+        mn[h] = fminf(mn[h], __shfl_xor_sync(0xffffffffu, mn[h], o));
+        mx[h] = fmaxf(mx[h], __shfl_xor_sync(0xffffffffu, mx[h], o));
       }
+      if (lane == 0) { red[(0 * G + h) * 16 + warp] = mn[h]; red[(1 * G + h) * 16 + warp] = mx[h]; }
     }
-  }
-  // merge the 16 half-warps
-  if (hl == 0) {
-#pragma unroll
-    for (int h = 0; h < G; ++h) { sm.m[hw][h] = m[h]; sm.l[hw][h] = l[h]; }
-  }
-#pragma unroll
-  for (int h = 0; h < G; ++h)
-#pragma unroll
-    for (int e = 0; e < 8; ++e) acc_smem[(hw * G + h) * kD + hl * 8 + e] = acc[h][e];
-  __syncthreads();
-  for (int o = t; o < G * kD; o += kThreads) {
-    const int h = o / kD, dch = o % kD;
-    float M = -INFINITY;
-    for (int w = 0; w < 16; ++w) M = fmaxf(M, sm.m[w][h]);
-    float Ls = 0.f, A = 0.f;
-    if (M != -INFINITY) {
-      for (int w = 0; w < 16; ++w) {
-        const float f = exp2f(sm.m[w][h] - M);
-        Ls += sm.l[w][h] * f;
-        A += acc_smem[(w * G + h) * kD + dch] * f;
-      }
-    }
-    res[h * (kD + 2) + 2 + dch] = A;
-    if (dch == 0) { res[h * (kD + 2)] = M; res[h * (kD + 2) + 1] = Ls; }
-  }
-  __syncthreads();
-}
-
-// Merge n partial states (M, L, A) per head and write bf16 output rows of the G heads.
-template <int G>
-__device__ __forceinline__ void combine_partials(const float* parts, int n, uint16_t* out_rows) {
-  for (int o = threadIdx.x; o < G * kD; o += kThreads) {
-    const int h = o / kD, dch = o % kD;
-    float M = -INFINITY;
-    for (int i = 0; i < n; ++i) M = fmaxf(M, __ldcg(parts + ((int64_t)i * G + h) * (kD + 2)));
-    float Ls = 0.f, A = 0.f;
-    if (M != -INFINITY) {
-      for (int i = 0; i < n; ++i) {
-        const float* pp = parts + ((int64_t)i * G + h) * (kD + 2);
-        const float mi = __ldcg(pp);
-        if (mi == -INFINITY) continue;
-        const float f = exp2f(mi - M);
-        Ls += __ldcg(pp + 1) * f;
-        A += __ldcg(pp + 2 + dch) * f;
-      }
-    }
-    out_rows[(int64_t)h * kD + dch] = f2bf_rn(Ls > 0.f ? A / Ls : 0.f);
-  }
-}
-
-template <int G>
-__global__ void __launch_bounds__(kThreads) attend_kernel(DecodeParams P) {
-  extern __shared__ __align__(16) float dyn[];
-  float* acc_smem = dyn;                                  // [16][G][128]
-  float* res = dyn + 16 * G * kD;                         // [G][130]
-  __shared__ float qs[G][kD];
-  __shared__ AttnSmem sm;
-  __shared__ uint32_t pref[1025];
-  __shared__ int is_last;
-  const int item = blockIdx.x;
-  const int t = threadIdx.x;
-  if (item < P.n_ret_items) {
-    const int gr = item / P.S, s = item % P.S;
-    const int b = gr / P.L.n_ret, r = gr % P.L.n_ret;
-    const int kvh = P.L.ret_kv[r];
-    const int N = seq_len_checked(P, b);
-    if (N == 0) {
-      if (s == 0) {
-        if (t == 0) set_status(P.status, -6);
-        for (int o = t; o < G * kD; o += kThreads)
-          P.out[((int64_t)b * P.L.Hq + kvh * G) * kD + o] = 0;
-        if (t < G) P.sel_counts[(int64_t)b * P.L.Hq + kvh * G + t] = 0;
-      }
-      return;
-    }
-    const int nch = (N + P.C - 1) / P.C;
-    // prefix of entry counts over chunks (nch <= 1024)
-    if (t == 0) {
-      uint32_t acc = 0;
-      for (int c = 0; c < nch; ++c) { pref[c] = acc; acc += __ldcg(P.chunk_cnt + (int64_t)gr * P.MC + c); }
-      pref[nch] = acc;
-    }
-    rope_query<G>(P, b, kvh, N, qs);
     __syncthreads();
-    const uint32_t U = pref[nch];
-    const uint32_t e0 = (uint32_t)(((uint64_t)U * s) / P.S);
-    const uint32_t e1 = (uint32_t)(((uint64_t)U * (s + 1)) / P.S);
-    const int64_t stride = (int64_t)P.MC * P.C;
-    const uint32_t* ent = P.ent + (int64_t)gr * stride;
+    if (threadIdx.x < G) {
+      const int h = threadIdx.x;
+      float a = red[(0 * G + h) * 16], z = red[(1 * G + h) * 16];
+      for (int w = 1; w < kFThreads / 32; ++w) {
+        a = fminf(a, red[(0 * G + h) * 16 + w]);
+        z = fmaxf(z, red[(1 * G + h) * 16 + w]);
+      }
+      atomicMax(P.lohi + ((int64_t)g * 2 + 0) * G + h, ~f2ord(a));
+      atomicMax(P.lohi + ((int64_t)g * 2 + 1) * G + h, f2ord(z));
+    }
+    arrive(P.bar + (int64_t)g * 4 + 0);
+  }
+
+  // ------------------------------------------------------------ phase H
+  __device__ void phase_hist(int k) {
+    const int g = group_of(k), j = k - sm.cbase[g];
+    const int N = gN(g);
+    const int n0 = j * C, n1 = min(N, n0 + C);
+    for (int i = threadIdx.x; i < G * kBins; i += kFThreads) sm.hist[i] = 0ull;
+    float lo[G], hi[G], inv[G];
+    load_range<G>(P, g, lo, hi, inv);
+    __syncthreads();
+    const float* sc = score_ptr(g, j);
+    const int64_t hs = score_hstride();
+    for (int n = n0 + threadIdx.x; n < n1; n += kFThreads) {
+#pragma unroll
+      for (int h = 0; h < G; ++h) {
+        const float s = sc[h * hs + (n - n0)];
+        const float e = (s - hi[h]) * kLog2e;
+        if (e > -42.f) {                      // below 2^-41 the fixed-point mass rounds to 0
+          const unsigned long long q = __float2ull_rn(exp2f(e) * kMassScale);
+          if (q) atomicAdd(&sm.hist[h * kBins + bin_of(s, lo[h], inv[h])], q);
+        }
+      }
+    }
+    __syncthreads();
+    unsigned long long* gh = P.hist + (int64_t)g * G * kBins;
+    for (int i = threadIdx.x; i < G * kBins; i += kFThreads) {
+      const unsigned long long v = sm.hist[i];
+      if (v) atomicAdd(gh + i, v);
+    }
+    arrive(P.bar + (int64_t)g * 4 + 1);
+  }
+
+  // b* of the G heads of group g into sm.ints[40 + h]; warp h handles head h.
+  __device__ void find_bstar(int g) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    if (warp < G) {
+      const int h = warp;
+      if (P.select_all) {
+        if (lane == 0) sm.ints[40 + h] = 0;
+      } else {
+        const unsigned long long* gh = P.hist + ((int64_t)g * G + h) * kBins;
+        unsigned long long v[8], tot = 0;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) { v[e] = __ldcg(gh + lane * 8 + e); tot += v[e]; }
+        unsigned long long x = tot;           // inclusive suffix sum over lanes
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const unsigned long long y = __shfl_down_sync(0xffffffffu, x, o);
+          if (lane + o < 32) x += y;
+        }
+        const unsigned long long T = __shfl_sync(0xffffffffu, x, 0);
+        const double thr = P.p * (double)T;
+        int best = -1;
+        unsigned long long cum = x - tot;
+#pragma unroll
+        for (int e = 7; e >= 0; --e) {
+          cum += v[e];
+          if (best < 0 && (double)cum >= thr) best = lane * 8 + e;
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) best = max(best, __shfl_xor_sync(0xffffffffu, best, o));
+        if (lane == 0) sm.ints[40 + h] = best < 0 ? 0 : best;
+      }
+    }
+    __syncthreads();
+  }
+
+  // ------------------------------------------------------------ phase T
+  __device__ void phase_select(int k) {
+    const int g = group_of(k), j = k - sm.cbase[g];
+    const int N = gN(g);
+    const int n0 = j * C, n1 = min(N, n0 + C);
+    float lo[G], hi[G], inv[G];
+    load_range<G>(P, g, lo, hi, inv);
+    find_bstar(g);
+    int bs[G];
+#pragma unroll
+    for (int h = 0; h < G; ++h) bs[h] = sm.ints[40 + h];
+    const float* sc = score_ptr(g, j);
+    const int64_t hs = score_hstride();
+    uint32_t* ent = P.ent + (int64_t)g * P.maxN_pad + n0;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    int hc[G];
+#pragma unroll
+    for (int h = 0; h < G; ++h) hc[h] = 0;
+    int base = 0;
+    for (int nb = n0; nb < n1; nb += kFThreads) {
+      const int n = nb + threadIdx.x;
+      uint32_t mask = 0;
+      if (n < n1) {
+#pragma unroll
+        for (int h = 0; h < G; ++h) {
+          const float s = sc[h * hs + (n - n0)];
+          if (bin_of(s, lo[h], inv[h]) >= bs[h]) { mask |= 1u << h; hc[h]++; }
+        }
+      }
+      const uint32_t bal = __ballot_sync(0xffffffffu, mask != 0);
+      __syncthreads();
+      if (lane == 0) sm.ints[warp] = __popc(bal);
+      __syncthreads();
+      int before = 0, total = 0;
+      for (int w = 0; w < kFThreads / 32; ++w) {
+        const int x = sm.ints[w];
+        before += (w < warp) ? x : 0;
+        total += x;
+      }
+      if (mask) ent[base + before + __popc(bal & ((1u << lane) - 1u))] = ((uint32_t)n << 8) | mask;
+      base += total;
+    }
+#pragma unroll
+    for (int h = 0; h < G; ++h) {
+      const int v = block_sum_int(hc[h], sm.ints);
+      if (threadIdx.x == 0 && v) atomicAdd(P.hcnt + (int64_t)g * G + h, v);
+    }
+    if (threadIdx.x == 0) P.ccnt[(int64_t)g * P.max_nch + j] = (uint32_t)base;
+    arrive(P.bar + (int64_t)g * 4 + 2);
+  }
+
+  // attention over rows [0, cnt) given by rowfn(i, kp, vp, mask); result in sm.res
+  template <class RowFn>
+  __device__ void attend_list(const float* q_s, int cnt, RowFn rowfn) {
+    constexpr int R = AttnCfg<G>::kRows;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, hl = lane & 15;
+    float q[G][8];
+#pragma unroll
+    for (int h = 0; h < G; ++h)
+#pragma unroll
+      for (int e = 0; e < 8; ++e) q[h][e] = q_s[h * kD + hl * 8 + e];
+    AttnState<G> st;
+    st.init();
+    for (int wb = warp * 2 * R; wb < cnt; wb += (kFThreads / 32) * 2 * R) {
+      const uint16_t* kp[R];
+      const uint16_t* vp[R];
+      uint32_t mask[R];
+#pragma unroll
+      for (int r = 0; r < R; ++r) {
+        const int i = wb + (lane >> 4) * R + r;
+        kp[r] = nullptr; vp[r] = nullptr; mask[r] = 0;
+        if (i < cnt) rowfn(i, kp[r], vp[r], mask[r]);
+      }
+      attend_step<G>(st, q, kp, vp, mask, hl);
+    }
+    attend_merge<G>(st, sm.attn, sm.res, kFThreads);
+  }
+
+  // ------------------------------------------------------------ phase W
+  __device__ void phase_attend(int k) {
+    const int g = group_of(k), j = k - sm.cbase[g];
+    const int b = g / P.L.n_ret, r = g % P.L.n_ret, kvh = P.L.ret_kv[r];
+    const int N = gN(g);
+    const int S = nch(g);
+    for (int c = threadIdx.x; c < S; c += kFThreads)
+      sm.pref[c] = (int)__ldcg(P.ccnt + (int64_t)g * P.max_nch + c);
+    __syncthreads();
+    const int U = block_scan_excl(sm.pref, S, sm.ints);
+    if (threadIdx.x == 0) sm.pref[S] = U;
+    rope_query<G>(P, b, kvh, N, sm.qret);
+    __syncthreads();
+    const int e0 = (int)(((long long)U * j) / S), e1 = (int)(((long long)U * (j + 1)) / S);
+    const uint32_t* ent = P.ent + (int64_t)g * P.maxN_pad;
     const int64_t rowbase = (int64_t)r * P.L.T_total + P.cache.seq_off[b];
     const uint16_t* kb = P.cache.k_ret;
     const uint16_t* vb = P.cache.v_ret;
-    auto rowfn = [&](int i, const uint16_t*& kp, const uint16_t*& vp, uint32_t& mask) {
-      const uint32_t e = e0 + (uint32_t)i;
-      int lo = 0, hi = nch - 1;                 // last chunk with pref[c] <= e
-      while (lo < hi) {
-        const int mid = (lo + hi + 1) >> 1;
-        if (pref[mid] <= e) lo = mid; else hi = mid - 1;
-      }
-      const uint32_t w = __ldcg(ent + (int64_t)lo * P.C + (e - pref[lo]));
+    const int* pref = sm.pref;
+    const int Cc = C;
+    attend_list(sm.qret, e1 - e0, [&](int i, const uint16_t*& kp, const uint16_t*& vp,
+                                      uint32_t& mask) {
+      const int e = e0 + i;
+      const int c = upper_index(pref, S, e);
+      const uint32_t w = __ldcg(ent + (int64_t)c * Cc + (e - pref[c]));
       const int64_t n = w >> 8;
       mask = w & 0xffu;
       kp = kb + (rowbase + n) * kD;
       vp = vb + (rowbase + n) * kD;
-    };
-    attend_rows<G>(qs, (int)(e1 - e0), rowfn, acc_smem, sm, res);
-    float* part = P.part_ret + (int64_t)item * G * (kD + 2);
-    for (int o = t; o < G * (kD + 2); o += kThreads) part[o] = res[o];
-    __threadfence();
+    });
+    // partial -> workspace; team / group merge by the last arrivals
+    const int stride = G * (kD + 2);
+    float* mine = P.part + (int64_t)k * stride;
+    for (int o = threadIdx.x; o < stride; o += kFThreads) mine[o] = sm.res[o];
+    const int team = j / kTeam, nteams = (S + kTeam - 1) / kTeam;
+    const int tcount = min(kTeam, S - team * kTeam);
     __syncthreads();
-    if (t == 0) is_last = (atomicAdd(P.arrive_ret + gr, 1u) == (uint32_t)(P.S - 1));
-    __syncthreads();
-    if (is_last) {
+    if (threadIdx.x == 0) {
       __threadfence();
-      combine_partials<G>(P.part_ret + (int64_t)gr * P.S * G * (kD + 2), P.S,
-                          P.out + ((int64_t)b * P.L.Hq + kvh * G) * kD);
-      if (t < G)
-        P.sel_counts[(int64_t)b * P.L.Hq + kvh * G + t] = __ldcg(P.hcnt + (int64_t)gr * G + t);
+      sm.ints[48] = atomicAdd(P.team_arr + sm.cbase[g] + team, 1u) == (uint32_t)(tcount - 1);
     }
-  } else {
-    const int li = item - P.n_ret_items;
-    const int lg = li / P.PL, piece = li % P.PL;   // lg = b * n_loc + x
-    const int b = lg / P.L.n_loc, x = lg % P.L.n_loc;
-    const int kvh = P.L.loc_kv[x];
-    const int N = seq_len_checked(P, b);
-    if (N == 0) {
-      if (piece == 0) {
-        if (t == 0) set_status(P.status, -6);
-        for (int o = t; o < G * kD; o += kThreads)
-          P.out[((int64_t)b * P.L.Hq + kvh * G) * kD + o] = 0;
-        if (t < G) P.sel_counts[(int64_t)b * P.L.Hq + kvh * G + t] = 0;
+    __syncthreads();
+    if (!sm.ints[48]) return;
+    __threadfence();
+    uint16_t* orow = P.out + ((int64_t)b * P.L.Hq + kvh * G) * kD;
+    const float* tparts = P.part + (int64_t)(sm.cbase[g] + team * kTeam) * stride;
+    if (nteams == 1) {
+      merge_partials<G>(tparts, tcount, nullptr, orow, kFThreads);
+    } else {
+      merge_partials<G>(tparts, tcount, P.tpart + (int64_t)(sm.cbase[g] + team) * stride,
+                        nullptr, kFThreads);
+      __syncthreads();
+      if (threadIdx.x == 0) {
+        __threadfence();
+        sm.ints[49] = atomicAdd(P.bar + (int64_t)g * 4 + 3, 1u) == (uint32_t)(nteams - 1);
       }
-      return;
+      __syncthreads();
+      if (!sm.ints[49]) return;
+      __threadfence();
+      merge_partials<G>(P.tpart + (int64_t)sm.cbase[g] * stride, nteams, nullptr, orow, kFThreads);
     }
+    if (threadIdx.x < G)
+      P.sel_counts[(int64_t)b * P.L.Hq + kvh * G + threadIdx.x] =
+          __ldcg(P.hcnt + (int64_t)g * G + threadIdx.x);
+    __syncthreads();
+  }
+
+  // ------------------------------------------------------------ local items
+  // Takes and runs one local item; false when the queue is empty.
+  __device__ bool local_item() {
+    __syncthreads();
+    if (sm.ints[34]) return false;
+    if (threadIdx.x == 0) {
+      const uint32_t it = atomicAdd(P.misc + 0, 1u);
+      sm.ints[33] = (int)it;
+      if ((int)it >= P.n_loc_items) sm.ints[34] = 1;
+    }
+    __syncthreads();
+    const int li = sm.ints[33];
+    if (li >= P.n_loc_items) return false;
+    const int lg = li / P.PL, piece = li % P.PL;
+    const int b = lg / P.L.n_loc, x = lg % P.L.n_loc, kvh = P.L.loc_kv[x];
+    const int N = sm.N[b];
+    if (N == 0) return true;                        // invalid sequence: outputs zeroed in plan
     const int nrows_all = min(N, P.L.ring);
     const int r0 = piece * P.RL;
     const int nrows = max(0, min(nrows_all - r0, P.RL));
-    rope_query<G>(P, b, kvh, N, qs);
+    rope_query<G>(P, b, kvh, N, sm.qloc);
     __syncthreads();
     const uint16_t* kb = P.cache.k_loc + ((int64_t)x * P.L.B + b) * P.L.ring * kD;
     const uint16_t* vb = P.cache.v_loc + ((int64_t)x * P.L.B + b) * P.L.ring * kD;
-    auto rowfn = [&](int i, const uint16_t*& kp, const uint16_t*& vp, uint32_t& mask) {
+    attend_list(sm.qloc, nrows, [&](int i, const uint16_t*& kp, const uint16_t*& vp,
+                                    uint32_t& mask) {
       kp = kb + (int64_t)(r0 + i) * kD;
       vp = vb + (int64_t)(r0 + i) * kD;
       mask = 0xffu;
-    };
-    attend_rows<G>(qs, nrows, rowfn, acc_smem, sm, res);
-    float* part = P.part_loc + (int64_t)li * G * (kD + 2);
-    for (int o = t; o < G * (kD + 2); o += kThreads) part[o] = res[o];
-    __threadfence();
+    });
+    const int stride = G * (kD + 2);
+    float* mine = P.lpart + (int64_t)li * stride;
+    for (int o = threadIdx.x; o < stride; o += kFThreads) mine[o] = sm.res[o];
     __syncthreads();
-    if (t == 0) is_last = (atomicAdd(P.arrive_loc + lg, 1u) == (uint32_t)(P.PL - 1));
-    __syncthreads();
-    if (is_last) {
+    if (threadIdx.x == 0) {
       __threadfence();
-      combine_partials<G>(P.part_loc + (int64_t)lg * P.PL * G * (kD + 2), P.PL,
-                          P.out + ((int64_t)b * P.L.Hq + kvh * G) * kD);
-      if (t < G) P.sel_counts[(int64_t)b * P.L.Hq + kvh * G + t] = nrows_all;
+      sm.ints[50] = atomicAdd(P.loc_arr + lg, 1u) == (uint32_t)(P.PL - 1);
+    }
+    __syncthreads();
+    if (sm.ints[50]) {
+      __threadfence();
+      merge_partials<G>(P.lpart + (int64_t)lg * P.PL * stride, P.PL, nullptr,
+                        P.out + ((int64_t)b * P.L.Hq + kvh * G) * kD, kFThreads);
+      if (threadIdx.x < G) P.sel_counts[(int64_t)b * P.L.Hq + kvh * G + threadIdx.x] = nrows_all;
+    }
+    __syncthreads();
+    return true;
+  }
+
+  __device__ void run() {
+    if (threadIdx.x == 0) sm.ints[34] = 0;
+    __syncthreads();
+    plan();
+    bool ok = true;
+    // phase-major over this CTA's chunks: no wait ever depends on a later phase
+    for (int k = blockIdx.x; k < NC; k += P.P) phase_score(k);
+    for (int k = blockIdx.x; ok && k < NC; k += P.P) {
+      const int g = group_of(k);
+      ok = wait_for(P.bar + (int64_t)g * 4 + 0, (uint32_t)nch(g));
+      if (ok) phase_hist(k);
+    }
+    for (int k = blockIdx.x; ok && k < NC; k += P.P) {
+      const int g = group_of(k);
+      ok = wait_for(P.bar + (int64_t)g * 4 + 1, (uint32_t)nch(g));
+      if (ok) phase_select(k);
+    }
+    for (int k = blockIdx.x; ok && k < NC; k += P.P) {
+      const int g = group_of(k);
+      ok = wait_for(P.bar + (int64_t)g * 4 + 2, (uint32_t)nch(g));
+      if (ok) phase_attend(k);
+    }
+    if (!ok) return;
+    while (local_item()) {
     }
   }
+};
+
+template <int G>
+__global__ void __launch_bounds__(kFThreads, 1) decode_kernel(const __grid_constant__ DecodeParams P) {
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  DecodeCta<G> cta(P, smem_raw);
+  cta.run();
 }
 
 // ------------------------------------------------------------------------------ sel_idx
@@ -561,7 +699,7 @@ template <int G>
 __global__ void __launch_bounds__(kThreads) emit_sel_kernel(DecodeParams P, int32_t* sel_idx,
                                                             int64_t sel_stride) {
   const int b = blockIdx.x / P.L.Hq, h = blockIdx.x % P.L.Hq;
-  const int kvh = h / G, j = h % G;
+  const int kvh = h / G, jh = h % G;
   const int N = seq_len_checked(P, b);
   int32_t* dst = sel_idx + ((int64_t)b * P.L.Hq + h) * sel_stride;
   if (N == 0) return;
@@ -575,18 +713,18 @@ __global__ void __launch_bounds__(kThreads) emit_sel_kernel(DecodeParams P, int3
     for (int k = threadIdx.x; k < cnt; k += kThreads) dst[k] = k < s1 ? k : w0 + (k - s1);
     return;
   }
-  const int gr = b * P.L.n_ret + slot;
-  const int nch = (N + P.C - 1) / P.C;
-  const int64_t stride = (int64_t)P.MC * P.C;
-  const uint32_t* ent = P.ent + (int64_t)gr * stride;
+  const int g = b * P.L.n_ret + slot;
+  const int C = (int)__ldcg(P.misc + 2);
+  const int nchg = (N + C - 1) / C;
+  const uint32_t* ent = P.ent + (int64_t)g * P.maxN_pad;
   int base = 0;
-  for (int c = 0; c < nch; ++c) {
-    const int cnt = (int)__ldcg(P.chunk_cnt + (int64_t)gr * P.MC + c);
+  for (int c = 0; c < nchg; ++c) {
+    const int cnt = (int)__ldcg(P.ccnt + (int64_t)g * P.max_nch + c);
     for (int k0 = 0; k0 < cnt; k0 += kThreads) {
       const int k = k0 + threadIdx.x;
       uint32_t w = 0;
       bool keep = false;
-      if (k < cnt) { w = __ldcg(ent + (int64_t)c * P.C + k); keep = (w >> j) & 1u; }
+      if (k < cnt) { w = __ldcg(ent + (int64_t)c * C + k); keep = (w >> jh) & 1u; }
       const uint32_t bal = __ballot_sync(0xffffffffu, keep);
       if (lane == 0) wsum[warp] = __popc(bal);
       __syncthreads();

@@ -13,8 +13,10 @@ decides *what* the inputs are:
   key is shifted by the minimum-norm vector ``delta = W_k (W_k^T W_k)^{-1} (alpha u)``, which
   moves the 16-dim projection ``W_k^T k_pre`` by ``alpha u`` (u a unit 16-vector); ``alpha`` is
   set from a strength in background standard deviations, ``alpha / sqrt(u^T W_k^T W_k u)``;
-* queries: for a retrieval query head the target projection is ``lam * u_hat`` (``u_hat`` the
-  head's cluster direction, or the normalised weighted sum of several for a diffuse head);
+* queries: for a retrieval query head the target projection is ``lam * u_hat / sigma`` (``u_hat``
+  the head's cluster direction, or the normalised weighted sum of several for a diffuse head;
+  ``sigma = sqrt(u_hat^T W_k^T W_k u_hat)`` the background standard deviation of the index
+  key along it, so lam is a temperature in background units for every head);
   ``q_pre = z + W_q (W_q^T W_q)^{-1} (target - W_q^T z)`` with ``z`` from the counter stream, so the
   projected query equals the target before bf16 storage rounding. ``lam`` is the one
   temperature knob, fixed per workload so that concentrated heads keep a few hundred tokens
@@ -120,7 +122,9 @@ class Workload:
             d += w * lay.clusters[i].u
         d /= np.linalg.norm(d)
         lam = self.lam_conc if kind == "conc" else self.lam_diff
-        return lam * d
+        # in units of the background score standard deviation along d: sqrt(d^T W_k^T W_k d)
+        W = self.w_kidx(layer)[kvh].astype(np.float64)
+        return lam / np.sqrt(d @ (W.T @ W) @ d) * d
 
     def q_pre_bits(self, layer: int) -> np.ndarray:
         """bf16 bits [B][Hq][128] of the pre-RoPE queries of one layer."""
@@ -245,14 +249,14 @@ def _ret_mask_qwen(seed: int, layers: int = 36, hkv: int = 8, n_ret: int = 43) -
 
 
 # Query temperatures (lam) per workload; see the module docstring.
-# (concentrated, diffuse): at 32K with 4-sigma clusters these keep about 400 and 2500 tokens
-# per head at p = 0.9 (about 250 in the 4K single-needle case).
+# (concentrated, diffuse): at 32K with 4-sigma clusters these keep about 420 and 2500 tokens
+# per head on average at p = 0.9.
 LAM = {
-    1: (1.65, 2.05),
-    2: (1.65, 2.05),
-    3: (1.65, 2.05),
-    4: (1.65, 2.05),
-    5: (1.65, 2.05),
+    1: (1.67, 1.97),
+    2: (1.67, 1.97),
+    3: (1.67, 1.97),
+    4: (1.67, 1.97),
+    5: (1.67, 1.97),
 }
 
 
