@@ -16,8 +16,10 @@ def nvcc() -> str:
     return "nvcc"
 
 
-def build(verbose: bool = False, extra_flags=()) -> str:
-    out = os.path.join(HERE, "librtp.so")
+def build(verbose: bool = False, extra_flags=(), out_name: str = "librtp.so") -> str:
+    """Compiles csrc/rtp_api.cu into ``out_name`` (librtp_trace.so with -DRTP_TRACE records
+    per-CTA phase timestamps of the decode kernel in the workspace)."""
+    out = os.path.join(HERE, out_name)
     src = os.path.join(HERE, "csrc", "rtp_api.cu")
     cmd = [nvcc(), *NVCC_FLAGS, *extra_flags, "-o", out, src]
     if verbose:

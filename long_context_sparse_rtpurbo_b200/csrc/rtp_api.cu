@@ -16,7 +16,7 @@ namespace {
 thread_local int32_t g_launches = 0;
 
 constexpr int kPlanCTAs = 160;      // upper bound on decode CTAs (one per SM; B200 has 148)
-constexpr int kLocRows = 128;       // ring rows per local attention item
+constexpr int kLocRows = 256;       // ring rows per local attention item
 constexpr long long kSpinLimit = 2000000000LL;   // ~1 s of SM clock per device-side wait
 
 inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
@@ -24,11 +24,11 @@ inline int align16(int x) { return (x + 15) & ~15; }
 
 struct Plan {
   LayerShape L;
-  int C_min, max_nch, NC_max, n_groups, n_lgroups, PL, n_loc_items;
+  int C_min, max_nch, NC_max, n_groups, n_lgroups, RL, PL, n_loc_items;
   int64_t maxN_pad;
   size_t off_ctrl, ctrl_bytes;
   size_t off_lohi, off_hcnt, off_bar, off_team, off_locarr, off_misc, off_hist;
-  size_t off_scores, off_ent, off_ccnt, off_part, off_tpart, off_lpart, total;
+  size_t off_scores, off_ent, off_ccnt, off_part, off_tpart, off_lpart, off_trace, total;
 };
 
 int check_desc(const rtp_layer_desc* d, LayerShape& L) {
@@ -77,15 +77,18 @@ int make_plan(const rtp_layer_desc* d, Plan& pl) {
   if (pl.n_groups > 8 * kFThreads) return RTP_ESHAPE;
   // chunks: at least C_min tokens, so a launch never has more than 8 per CTA plus one per group
   int64_t cmin = (int64_t(pl.n_groups) * maxN + 8 * kPlanCTAs - 1) / (8 * kPlanCTAs);
-  cmin = std::max<int64_t>(cmin, 256);
+  cmin = std::max<int64_t>(cmin, 1024);
+  cmin = std::max<int64_t>(cmin, (maxN + kTeam * kMaxMerge - 1) / (kTeam * kMaxMerge));
   cmin = (cmin + 255) / 256 * 256;
   pl.C_min = (int)cmin;
   pl.max_nch = (int)((maxN + cmin - 1) / cmin);
-  if (pl.max_nch > 8 * kFThreads) return RTP_ESHAPE;
+  if (pl.max_nch > kTeam * kMaxMerge) return RTP_ESHAPE;
   pl.NC_max = 8 * kPlanCTAs + pl.n_groups + 16;
   pl.maxN_pad = (maxN + 63) / 64 * 64;
   const int64_t loc_rows = std::min<int64_t>(maxN, L.ring);
-  pl.PL = (int)((loc_rows + kLocRows - 1) / kLocRows);
+  const int64_t rl = std::max<int64_t>(kLocRows, (loc_rows + kMaxMerge - 1) / kMaxMerge);
+  pl.RL = (int)rl;
+  pl.PL = (int)((loc_rows + rl - 1) / rl);
   pl.n_loc_items = pl.n_lgroups * pl.PL;
   const size_t part_bytes = sizeof(float) * G * (kD + 2);
   size_t o = 256;                                   // [0, 256): status word
@@ -104,6 +107,11 @@ int make_plan(const rtp_layer_desc* d, Plan& pl) {
   pl.off_part = o;   o = align256(o + part_bytes * pl.NC_max);
   pl.off_tpart = o;  o = align256(o + part_bytes * pl.NC_max);
   pl.off_lpart = o;  o = align256(o + part_bytes * std::max(pl.n_loc_items, 1));
+#ifdef RTP_TRACE
+  pl.off_trace = o;  o = align256(o + sizeof(unsigned long long) * kPlanCTAs * kTraceEvents);
+#else
+  pl.off_trace = 0;
+#endif
   pl.total = o;
   return RTP_OK;
 }
@@ -137,7 +145,10 @@ int dev_info(DevInfo& di) {
 int smem_layout(DecodeParams& P, const Plan& pl, int smem_optin) {
   const int G = P.L.G;
   int o = 0;
-  P.sm_attn = o;  o = align16(o + 4 * (16 * G * kD + 2 * 16 * G));
+  const int merge_scratch = 4 * std::max((kFThreads / 32) * G * kD + 2 * (kFThreads / 32) * G,
+                                         2 * kMaxMerge * G + 2 * G);
+  const int stage = std::max({AttnCfg<8>::stage_bytes(kFThreads), 4 * 512 * 32, merge_scratch});
+  P.sm_stage = o; o = align16(o + stage);
   P.sm_res = o;   o = align16(o + 4 * G * (kD + 2));
   P.sm_qret = o;  o = align16(o + 4 * G * kD);
   P.sm_qloc = o;  o = align16(o + 4 * G * kD);
@@ -283,7 +294,7 @@ int rtp_decode_step(const rtp_layer_desc* desc, const rtp_cache* cache, const ui
   P.L = L;
   P.L.T_total = cache->T_total;
   P.C_min = pl.C_min; P.max_nch = pl.max_nch; P.NC_max = pl.NC_max;
-  P.n_groups = pl.n_groups; P.n_lgroups = pl.n_lgroups; P.PL = pl.PL; P.RL = kLocRows;
+  P.n_groups = pl.n_groups; P.n_lgroups = pl.n_lgroups; P.PL = pl.PL; P.RL = pl.RL;
   P.n_loc_items = pl.n_loc_items;
   P.select_all = p >= 1.0 ? 1 : 0;
   P.p = p;
@@ -307,6 +318,7 @@ int rtp_decode_step(const rtp_layer_desc* desc, const rtp_cache* cache, const ui
   P.part = at<float>(ws, pl.off_part);
   P.tpart = at<float>(ws, pl.off_tpart);
   P.lpart = at<float>(ws, pl.off_lpart);
+  P.trace = pl.off_trace ? at<unsigned long long>(ws, pl.off_trace) : nullptr;
   if (cudaMemsetAsync(at<char>(ws, pl.off_ctrl), 0, pl.ctrl_bytes, st) != cudaSuccess)
     return RTP_ECUDA;
   int r;

@@ -1,12 +1,15 @@
 // Exact softmax attention of the G query heads of one KV head over a list of K/V rows
 // ("Full Attention Strikes Back" (paper text) §3.2 eq. (5): O = sum_n softmax(q^T k_n / sqrt(d)) v_n).
 //
-// Layout on the SM: a half-warp (16 lanes) owns one row per step, each lane 8 of the 128
-// channels (one 16-byte load of K and one of V). A half-warp keeps kRows rows in flight. The
-// kRows x G partial dot products of a lane are reduced over the 16 lanes by recursive halving
-// (each step exchanges half of the remaining values), so every lane ends with one complete
-// logit; the probabilities are then broadcast for the V update. Softmax state (running max,
-// sum, 8-channel accumulator per head) is kept per half-warp in the log2 domain (q carries
+// Layout on the SM: a half-warp (16 lanes) owns kRows rows per step, each lane 8 of the 128
+// channels (16 bytes of K and of V per row). Rows are staged in shared memory with cp.async
+// (16 bytes per lane, L2-only), two steps deep, so the loads of step i+1 are in flight while
+// step i is computed and no registers are held by loads in flight. A lane only ever reads the
+// bytes it copied itself, so no barrier is needed between copy and use. The kRows x G partial
+// dot products of a lane are reduced over the 16 lanes by recursive halving (each step
+// exchanges half of the remaining values), so every lane ends with one complete logit; the
+// probabilities are then broadcast for the V update. Softmax state (running max, sum,
+// 8-channel accumulator per head) is kept per half-warp in the log2 domain (q carries
 // log2(e)/sqrt(d)) and merged across half-warps at the end.
 #pragma once
 
@@ -15,9 +18,20 @@
 namespace rtp {
 
 template <int G> struct AttnCfg {
-  static constexpr int kRows = (G >= 8) ? 2 : 4;          // rows in flight per half-warp
+  static constexpr int kRows = 2;                         // rows per half-warp per step
   static constexpr int kVals = kRows * G;                 // partial dots per lane
+  static constexpr int kStages = 2;
+  // staging bytes for a CTA of nthreads threads
+  static constexpr int stage_bytes(int nthreads) { return kStages * (nthreads / 16) * kRows * 512; }
 };
+
+__device__ __forceinline__ void cp_async16(void* smem, const void* gmem) {
+  const unsigned s = (unsigned)__cvta_generic_to_shared(smem);
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(s), "l"(gmem) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
 
 // Recursive-halving reduction of n values over the 16 lanes of a half-warp. On exit v[0] of
 // lane hl holds the full sum of value index (hl >> (4 - log2 n)) (n <= 16).
@@ -58,21 +72,15 @@ template <int G> struct AttnState {
   }
 };
 
-// One step of kRows rows for a half-warp. kp/vp: row pointers (lane-independent within the
-// half-warp), mask: heads that attend each row (0 for an invalid row).
+// One step of kRows staged rows for a half-warp; kw/vw: this lane's 16 bytes of each row
+// (zero for rows no head attends), mask: heads that attend each row.
 template <int G>
 __device__ __forceinline__ void attend_step(AttnState<G>& st, const float (&q)[G][8],
-                                            const uint16_t* const (&kp)[AttnCfg<G>::kRows],
-                                            const uint16_t* const (&vp)[AttnCfg<G>::kRows],
+                                            const uint4 (&kw)[AttnCfg<G>::kRows],
+                                            const uint4 (&vw)[AttnCfg<G>::kRows],
                                             const uint32_t (&mask)[AttnCfg<G>::kRows], int hl) {
   constexpr int R = AttnCfg<G>::kRows;
   constexpr int V = AttnCfg<G>::kVals;
-  uint4 kw[R], vw[R];
-#pragma unroll
-  for (int r = 0; r < R; ++r) {
-    kw[r] = mask[r] ? ld_stream(kp[r] + hl * 8) : make_uint4(0, 0, 0, 0);
-    vw[r] = mask[r] ? ld_stream(vp[r] + hl * 8) : make_uint4(0, 0, 0, 0);
-  }
   float d[V];
 #pragma unroll
   for (int r = 0; r < R; ++r) {
@@ -94,7 +102,7 @@ __device__ __forceinline__ void attend_step(AttnState<G>& st, const float (&q)[G
   uint32_t my_mask = 0;
 #pragma unroll
   for (int r = 0; r < R; ++r) my_mask = (r == my_r) ? mask[r] : my_mask;
-  float logit = ((my_mask >> my_h) & 1u) ? d[0] : -INFINITY;
+  const float logit = ((my_mask >> my_h) & 1u) ? d[0] : -INFINITY;
   // block max per head over the R rows: lanes holding the same head differ in the row bits
   float bm = logit;
 #pragma unroll
@@ -102,23 +110,22 @@ __device__ __forceinline__ void attend_step(AttnState<G>& st, const float (&q)[G
     const int lanebit = (o * G) << kShift;
     bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, lanebit));
   }
-  // new running max and p for my value
   float mnew_my = -INFINITY;
 #pragma unroll
   for (int h = 0; h < G; ++h) mnew_my = (h == my_h) ? fmaxf(st.m[h], bm) : mnew_my;
   const float p_my = (logit == -INFINITY) ? 0.f : exp2f(logit - mnew_my);
   // broadcast: every lane gets p of each (r, h) and the block max of each head
   const int base = (threadIdx.x & 31) & 16;
-  float scale[G];
 #pragma unroll
   for (int h = 0; h < G; ++h) {
-    const float bmh = __shfl_sync(0xffffffffu, bm, base + ((h) << kShift));
-    const float mn = fmaxf(st.m[h], bmh);
-    scale[h] = (mn == -INFINITY) ? 1.f : exp2f(st.m[h] - mn);
-    st.m[h] = mn;
-    st.l[h] *= scale[h];
+    const float bmh = __shfl_sync(0xffffffffu, bm, base + (h << kShift));
+    if (bmh > st.m[h]) {                       // the running max moved: rescale the state
+      const float scale = exp2f(st.m[h] - bmh);  // 0 when the state was empty (m = -inf)
+      st.m[h] = bmh;
+      st.l[h] *= scale;
 #pragma unroll
-    for (int e = 0; e < 8; ++e) st.acc[h][e] *= scale[h];
+      for (int e = 0; e < 8; ++e) st.acc[h][e] *= scale;
+    }
   }
 #pragma unroll
   for (int r = 0; r < R; ++r) {
@@ -134,8 +141,63 @@ __device__ __forceinline__ void attend_step(AttnState<G>& st, const float (&q)[G
   }
 }
 
+// Attention of the G heads over rows [0, cnt), row i given by rowfn(i, kp, vp, mask).
+// stage: AttnCfg<G>::stage_bytes(nthreads) bytes of shared memory. Leaves the half-warp
+// states in st (merge with attend_merge).
+template <int G, class RowFn>
+__device__ __forceinline__ void attend_rows(AttnState<G>& st, const float (&q)[G][8], int cnt,
+                                            RowFn rowfn, unsigned char* stage, int nthreads) {
+  constexpr int R = AttnCfg<G>::kRows;
+  const int t = threadIdx.x, lane = t & 31, warp = t >> 5, hl = lane & 15, hw = t >> 4;
+  const int nhw = nthreads >> 4;
+  const int step = (nthreads >> 5) * 2 * R;                  // rows per CTA step
+  // this half-warp's slot: stage s, row r -> stage + ((s * nhw + hw) * R + r) * 512
+  auto slot = [&](int s, int r) -> unsigned char* {
+    return stage + ((size_t)(s * nhw + hw) * R + r) * 512;
+  };
+  uint32_t mask_cur[R], mask_nxt[R];
+  auto issue = [&](int wb, int s, uint32_t (&mk)[R]) {
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+      const int i = wb + (lane >> 4) * R + r;
+      const uint16_t* kp = nullptr;
+      const uint16_t* vp = nullptr;
+      mk[r] = 0;
+      if (i < cnt) rowfn(i, kp, vp, mk[r]);
+      if (mk[r]) {
+        cp_async16(slot(s, r) + hl * 16, kp + hl * 8);
+        cp_async16(slot(s, r) + 256 + hl * 16, vp + hl * 8);
+      }
+    }
+    cp_async_commit();
+  };
+  int wb = warp * 2 * R;
+  int s = 0;
+  if (wb < cnt) issue(wb, 0, mask_cur);
+  for (; wb < cnt; wb += step, s ^= 1) {
+    if (wb + step < cnt) issue(wb + step, s ^ 1, mask_nxt);
+    else cp_async_commit();                                   // keep one group per step
+    cp_async_wait<1>();
+    uint4 kw[R], vw[R];
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+      if (mask_cur[r]) {
+        kw[r] = *reinterpret_cast<const uint4*>(slot(s, r) + hl * 16);
+        vw[r] = *reinterpret_cast<const uint4*>(slot(s, r) + 256 + hl * 16);
+      } else {
+        kw[r] = make_uint4(0, 0, 0, 0);
+        vw[r] = make_uint4(0, 0, 0, 0);
+      }
+    }
+    attend_step<G>(st, q, kw, vw, mask_cur, hl);
+#pragma unroll
+    for (int r = 0; r < R; ++r) mask_cur[r] = mask_nxt[r];
+  }
+  cp_async_wait<0>();
+}
+
 // Merges the per-half-warp states of a CTA of nthreads threads into res[G][2 + 128]
-// (M, L, A). scratch: >= (nthreads / 32) * G * 128 floats plus 2 * (nthreads / 32) * G.
+// (M, L, A). scratch: >= (nthreads / 32) * G * 128 + 2 * (nthreads / 32) * G floats.
 template <int G>
 __device__ __forceinline__ void attend_merge(AttnState<G>& st, float* scratch, float* res,
                                              int nthreads) {
@@ -157,6 +219,7 @@ __device__ __forceinline__ void attend_merge(AttnState<G>& st, float* scratch, f
     }
     st.m[h] = mn;
   }
+  __syncthreads();                                // scratch may alias the staging buffer
   float* sm_m = scratch + nw * G * kD;
   float* sm_l = sm_m + nw * G;
   if (lane < 16) {
@@ -188,34 +251,58 @@ __device__ __forceinline__ void attend_merge(AttnState<G>& st, float* scratch, f
   __syncthreads();
 }
 
-// Merges n partial states (stride G*(2+128) floats, in global memory written by other CTAs)
-// into one; result into `dst` (global, same format) or, when out_rows is given, the bf16
-// output rows of the G heads.
+// Merges n <= kMaxMerge partial states (stride G*(2+128) floats, global memory written by
+// other CTAs) into `dst` (same format) or, when out_rows is given, into the bf16 output rows
+// of the G heads. scratch: >= 2 * kMaxMerge * G + G floats of shared memory.
+constexpr int kMaxMerge = 64;
 template <int G>
 __device__ __forceinline__ void merge_partials(const float* parts, int n, float* dst,
-                                               uint16_t* out_rows, int nthreads) {
-  for (int o = threadIdx.x; o < G * kD; o += nthreads) {
-    const int h = o / kD, dch = o % kD;
+                                               uint16_t* out_rows, float* scratch, int nthreads) {
+  float* fM = scratch;                 // [n][G]: max, then the weight 2^(M_i - M)
+  float* fL = scratch + kMaxMerge * G; // [n][G]
+  float* tot = fL + kMaxMerge * G;     // [G]: M, then L
+  const int t = threadIdx.x;
+  for (int o = t; o < n * G; o += nthreads) {
+    const int i = o / G, h = o % G;
+    const float* pp = parts + ((int64_t)i * G + h) * (kD + 2);
+    fM[o] = __ldcg(pp);
+    fL[o] = __ldcg(pp + 1);
+  }
+  __syncthreads();
+  if (t < G) {
     float M = -INFINITY;
-    for (int i = 0; i < n; ++i) M = fmaxf(M, __ldcg(parts + ((int64_t)i * G + h) * (kD + 2)));
-    float Ls = 0.f, A = 0.f;
-    if (M != -INFINITY) {
-      for (int i = 0; i < n; ++i) {
-        const float* pp = parts + ((int64_t)i * G + h) * (kD + 2);
-        const float mi = __ldcg(pp);
-        if (mi == -INFINITY) continue;
-        const float f = exp2f(mi - M);
-        Ls += __ldcg(pp + 1) * f;
-        A += __ldcg(pp + 2 + dch) * f;
-      }
+    for (int i = 0; i < n; ++i) M = fmaxf(M, fM[i * G + t]);
+    float Ls = 0.f;
+    for (int i = 0; i < n; ++i) {
+      const float f = (M == -INFINITY || fM[i * G + t] == -INFINITY) ? 0.f : exp2f(fM[i * G + t] - M);
+      fM[i * G + t] = f;
+      Ls += fL[i * G + t] * f;
     }
+    tot[t] = M;
+    tot[G + t] = Ls;
+  }
+  __syncthreads();
+  for (int o = t; o < G * kD; o += nthreads) {
+    const int h = o / kD, dch = o % kD;
+    float A = 0.f;
+    int i = 0;
+    for (; i + 8 <= n; i += 8) {
+      float a[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) a[u] = __ldcg(parts + ((int64_t)(i + u) * G + h) * (kD + 2) + 2 + dch);
+#pragma unroll
+      for (int u = 0; u < 8; ++u) A = fmaf(a[u], fM[(i + u) * G + h], A);
+    }
+    for (; i < n; ++i) A = fmaf(__ldcg(parts + ((int64_t)i * G + h) * (kD + 2) + 2 + dch), fM[i * G + h], A);
+    const float Ls = tot[G + h];
     if (out_rows) {
       out_rows[(int64_t)h * kD + dch] = f2bf_rn(Ls > 0.f ? A / Ls : 0.f);
     } else {
       dst[h * (kD + 2) + 2 + dch] = A;
-      if (dch == 0) { dst[h * (kD + 2)] = M; dst[h * (kD + 2) + 1] = Ls; }
+      if (dch == 0) { dst[h * (kD + 2)] = tot[h]; dst[h * (kD + 2) + 1] = Ls; }
     }
   }
+  __syncthreads();
 }
 
 }  // namespace rtp

@@ -18,9 +18,10 @@
 //      compacted in ascending order into entries (n << 8 | head mask); counts.
 //   W  the group's entries are split evenly over its chunks' CTAs; each gathers its rows
 //      once for all G heads (a head that did not select a row skips it) and writes a
-//      partial softmax state; partials merge in teams of 16, the last team writes out.
-// Local items (a slice of one local head's ring) come from a global queue; a CTA takes one
-// whenever it would otherwise wait for a counter, and drains the queue at the end.
+//      partial softmax state; partials merge in teams of 32, the last team writes out.
+// Local items (a slice of one local head's ring) come from a global queue. CTAs without a
+// retrieval chunk start on them at once; the others join when their chunks are done, so a
+// local item never delays a phase of the retrieval chain.
 // Every wait is bounded (clock64 limit): on expiry the kernel records RTP_ETIMEOUT, raises
 // an abort flag that ends every other wait, and returns.
 #pragma once
@@ -31,7 +32,7 @@
 namespace rtp {
 
 constexpr int kFThreads = 512;          // threads of the decode kernel
-constexpr int kTeam = 16;               // partials merged per team
+constexpr int kTeam = 32;               // partials merged per team
 
 struct DecodeParams {
   LayerShape L;
@@ -50,7 +51,7 @@ struct DecodeParams {
   long long spin_limit;
   int64_t maxN_pad;
   // shared-memory layout (byte offsets into the dynamic buffer)
-  int sm_scores, sm_attn, sm_res, sm_qret, sm_qloc, sm_qidx, sm_tmp, sm_hist, sm_N, sm_cbase,
+  int sm_scores, sm_stage, sm_res, sm_qret, sm_qloc, sm_qidx, sm_tmp, sm_hist, sm_N, sm_cbase,
       sm_pref, sm_int;
   // inputs / outputs
   const uint16_t* q_pre;
@@ -74,7 +75,12 @@ struct DecodeParams {
   float* part;                 // [NC_max][G][130]
   float* tpart;                // [NC_max][G][130]
   float* lpart;                // [n_loc_items][G][130]
+  unsigned long long* trace;   // [P][kTraceEvents] %globaltimer stamps (tracing builds only)
 };
+
+// Phase-boundary timestamps, recorded only when built with -DRTP_TRACE.
+enum TraceEvent { kEvStart, kEvPlan, kEvScore, kEvWait1, kEvHist, kEvWait2, kEvSelect, kEvWait3,
+                  kEvAttend, kEvLocal, kEvEnd, kTraceEvents = 16 };
 
 // ------------------------------------------------------------------------------ helpers
 __device__ __forceinline__ int seq_len_checked(const DecodeParams& P, int b) {
@@ -150,19 +156,20 @@ __device__ __forceinline__ int upper_index(const int* a, int n, int key) {
   return lo;
 }
 
+// stage: index-row staging (phase S), K/V row staging and merge scratch (attention).
 template <int G> struct Smem {
-  float* scores; float* attn; float* res; float* qret; float* qloc; float* qidx; float* tmp;
-  unsigned long long* hist; int* N; int* cbase; int* pref; int* ints;
+  float* scores; unsigned char* stage; float* res; float* qret; float* qloc; float* qidx;
+  float* tmp; unsigned long long* hist; int* N; int* cbase; int* pref; int* ints;
   __device__ Smem(unsigned char* base, const DecodeParams& P)
-      : scores((float*)(base + P.sm_scores)), attn((float*)(base + P.sm_attn)),
+      : scores((float*)(base + P.sm_scores)), stage(base + P.sm_stage),
         res((float*)(base + P.sm_res)), qret((float*)(base + P.sm_qret)),
         qloc((float*)(base + P.sm_qloc)), qidx((float*)(base + P.sm_qidx)),
         tmp((float*)(base + P.sm_tmp)), hist((unsigned long long*)(base + P.sm_hist)),
         N((int*)(base + P.sm_N)), cbase((int*)(base + P.sm_cbase)), pref((int*)(base + P.sm_pref)),
         ints((int*)(base + P.sm_int)) {}
 };
-// ints[]: [0..31] reduction scratch, [32] wait flag, [33] local item, [34] local queue empty,
-//         [40..47] b*, [48..50] last-arrival flags
+// ints[]: [0..31] reduction scratch, [32] wait flag, [33] next local item, [40..47] b*,
+//         [48..50] last-arrival flags
 
 // RoPE'd, pre-scaled query of the G heads of KV head kvh at position N - 1 -> q_s[G][128].
 template <int G>
@@ -245,6 +252,18 @@ struct DecodeCta {
     return smem_mode ? (int64_t)P.C_cap : P.maxN_pad;
   }
 
+  __device__ __forceinline__ void trace(int ev) {
+#ifdef RTP_TRACE
+    if (threadIdx.x == 0 && P.trace) {
+      unsigned long long t;
+      asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+      P.trace[(int64_t)blockIdx.x * kTraceEvents + ev] = t;
+    }
+#else
+    (void)ev;
+#endif
+  }
+
   // arrival on a counter after this CTA's writes
   __device__ __forceinline__ void arrive(uint32_t* ctr) {
     __syncthreads();
@@ -279,9 +298,7 @@ struct DecodeCta {
       __syncthreads();
       if (f == 1) return true;
       if (f == 2) return false;
-      if (!local_item()) {
-        if (threadIdx.x == 0) __nanosleep(200);
-      }
+      if (threadIdx.x == 0) __nanosleep(100);
     }
   }
 
@@ -325,11 +342,30 @@ struct DecodeCta {
   }
 
   // ------------------------------------------------------------ phase S
+  // The chunk's index rows (32 B each, contiguous) stream through a ring of kSStages stages
+  // of kSRows rows in shared memory with cp.async; the projected query is formed while the
+  // first stages are in flight.
+  static constexpr int kSRows = 512, kSStages = 4;
   __device__ void phase_score(int k) {
     const int g = group_of(k), j = k - sm.cbase[g];
     const int b = g / P.L.n_ret, r = g % P.L.n_ret, kvh = P.L.ret_kv[r];
     const int N = gN(g);
     const int n0 = j * C, n1 = min(N, n0 + C);
+    const unsigned char* src =
+        (const unsigned char*)(P.cache.idx + ((int64_t)r * P.L.T_total + P.cache.seq_off[b] + n0) * kR);
+    const int nst = (n1 - n0 + kSRows - 1) / kSRows;
+    auto issue = [&](int st) {
+      if (st < nst) {
+        unsigned char* dst = sm.stage + (st % kSStages) * (kSRows * 32);
+        const int rows = min(kSRows, n1 - n0 - st * kSRows);
+        for (int piece = threadIdx.x; piece < rows * 2; piece += kFThreads)
+          cp_async16(dst + piece * 16, src + ((int64_t)st * kSRows * 32) + piece * 16);
+      }
+      cp_async_commit();
+    };
+    __syncthreads();                       // the stage buffer may still be read by a merge
+#pragma unroll
+    for (int st = 0; st < kSStages - 1; ++st) issue(st);
     index_query<G>(P, b, kvh, sm.qidx, sm.tmp);
     float qi[G][kR];
 #pragma unroll
@@ -339,39 +375,34 @@ struct DecodeCta {
     float mn[G], mx[G];
 #pragma unroll
     for (int h = 0; h < G; ++h) { mn[h] = INFINITY; mx[h] = -INFINITY; }
-    const uint16_t* idx = P.cache.idx + ((int64_t)r * P.L.T_total + P.cache.seq_off[b]) * kR;
     float* sc = score_ptr(g, j);
     const int64_t hs = score_hstride();
-    constexpr int U = 4;
-    for (int nb = n0 + threadIdx.x; nb < n1; nb += U * kFThreads) {
-      uint4 a[U], c2[U];
+    for (int st = 0; st < nst; ++st) {
+      issue(st + kSStages - 1);
+      cp_async_wait<kSStages - 1>();
+      __syncthreads();
+      const int rows = min(kSRows, n1 - n0 - st * kSRows);
+      const unsigned char* buf = sm.stage + (st % kSStages) * (kSRows * 32);
+      for (int i = threadIdx.x; i < rows; i += kFThreads) {
+        const uint4 a = *reinterpret_cast<const uint4*>(buf + i * 32);
+        const uint4 c2 = *reinterpret_cast<const uint4*>(buf + i * 32 + 16);
+        float x[16];
+        unpack8(a, x);
+        unpack8(c2, x + 8);
+        const int nl = st * kSRows + i;
 #pragma unroll
-      for (int u = 0; u < U; ++u) {
-        const int n = nb + u * kFThreads;
-        if (n < n1) {
-          a[u] = ld_stream(idx + (int64_t)n * kR);
-          c2[u] = ld_stream(idx + (int64_t)n * kR + 8);
+        for (int h = 0; h < G; ++h) {
+          float acc = 0.f;
+#pragma unroll
+          for (int jj = 0; jj < kR; ++jj) acc = fmaf(qi[h][jj], x[jj], acc);
+          sc[h * hs + nl] = acc;
+          mn[h] = fminf(mn[h], acc);
+          mx[h] = fmaxf(mx[h], acc);
         }
       }
-#pragma unroll
-      for (int u = 0; u < U; ++u) {
-        const int n = nb + u * kFThreads;
-        if (n < n1) {
-          float x[16];
-          unpack8(a[u], x);
-          unpack8(c2[u], x + 8);
-#pragma unroll
-          for (int h = 0; h < G; ++h) {
-            float acc = 0.f;
-#pragma unroll
-            for (int jj = 0; jj < kR; ++jj) acc = fmaf(qi[h][jj], x[jj], acc);
-            sc[h * hs + (n - n0)] = acc;
-            mn[h] = fminf(mn[h], acc);
-            mx[h] = fmaxf(mx[h], acc);
-          }
-        }
-      }
+      __syncthreads();                     // before the slot is refilled
     }
+    cp_async_wait<0>();
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     float* red = sm.tmp;                    // [2][G][16]
     __syncthreads();
@@ -403,7 +434,11 @@ struct DecodeCta {
     const int g = group_of(k), j = k - sm.cbase[g];
     const int N = gN(g);
     const int n0 = j * C, n1 = min(N, n0 + C);
-    for (int i = threadIdx.x; i < G * kBins; i += kFThreads) sm.hist[i] = 0ull;
+    // 64-bit fixed-point bins as (low word, high word) pairs of 32-bit shared atomics: the
+    // low-word add returns the old value, its carry goes to the high word (exact)
+    uint32_t* hlo = reinterpret_cast<uint32_t*>(sm.hist);
+    uint32_t* hhi = hlo + G * kBins;
+    for (int i = threadIdx.x; i < 2 * G * kBins; i += kFThreads) hlo[i] = 0u;
     float lo[G], hi[G], inv[G];
     load_range<G>(P, g, lo, hi, inv);
     __syncthreads();
@@ -416,14 +451,18 @@ struct DecodeCta {
         const float e = (s - hi[h]) * kLog2e;
         if (e > -42.f) {                      // below 2^-41 the fixed-point mass rounds to 0
           const unsigned long long q = __float2ull_rn(exp2f(e) * kMassScale);
-          if (q) atomicAdd(&sm.hist[h * kBins + bin_of(s, lo[h], inv[h])], q);
+          const uint32_t ql = (uint32_t)q, qh = (uint32_t)(q >> 32);
+          const int bi = h * kBins + bin_of(s, lo[h], inv[h]);
+          const uint32_t old = atomicAdd(&hlo[bi], ql);
+          const uint32_t up = qh + ((old + ql < old) ? 1u : 0u);
+          if (up) atomicAdd(&hhi[bi], up);
         }
       }
     }
     __syncthreads();
     unsigned long long* gh = P.hist + (int64_t)g * G * kBins;
     for (int i = threadIdx.x; i < G * kBins; i += kFThreads) {
-      const unsigned long long v = sm.hist[i];
+      const unsigned long long v = ((unsigned long long)hhi[i] << 32) | hlo[i];
       if (v) atomicAdd(gh + i, v);
     }
     arrive(P.bar + (int64_t)g * 4 + 1);
@@ -465,6 +504,10 @@ struct DecodeCta {
   }
 
   // ------------------------------------------------------------ phase T
+  // Tiles of kFThreads * kTRun tokens; in a tile each thread owns a run of consecutive
+  // tokens: masks in registers, one block-wide scan of the per-thread counts, then each
+  // thread writes its run's entries.
+  static constexpr int kTRun = 32;
   __device__ void phase_select(int k) {
     const int g = group_of(k), j = k - sm.cbase[g];
     const int N = gN(g);
@@ -483,19 +526,36 @@ struct DecodeCta {
 #pragma unroll
     for (int h = 0; h < G; ++h) hc[h] = 0;
     int base = 0;
-    for (int nb = n0; nb < n1; nb += kFThreads) {
-      const int n = nb + threadIdx.x;
-      uint32_t mask = 0;
-      if (n < n1) {
+    for (int tb = 0; tb < n1 - n0; tb += kFThreads * kTRun) {
+      const int len = min(kFThreads * kTRun, n1 - n0 - tb);
+      const int per = (len + kFThreads - 1) / kFThreads;
+      const int t0 = tb + threadIdx.x * per, t1 = min(tb + len, t0 + per);
+      uint32_t packed[kTRun / 4];
 #pragma unroll
-        for (int h = 0; h < G; ++h) {
-          const float s = sc[h * hs + (n - n0)];
-          if (bin_of(s, lo[h], inv[h]) >= bs[h]) { mask |= 1u << h; hc[h]++; }
+      for (int w = 0; w < kTRun / 4; ++w) packed[w] = 0u;
+      int cnt = 0;
+#pragma unroll
+      for (int i = 0; i < kTRun; ++i) {
+        const int nl = t0 + i;
+        if (i < per && nl < t1) {
+          uint32_t mask = 0;
+#pragma unroll
+          for (int h = 0; h < G; ++h) {
+            const float sv = sc[h * hs + nl];
+            if (bin_of(sv, lo[h], inv[h]) >= bs[h]) { mask |= 1u << h; hc[h]++; }
+          }
+          packed[i / 4] |= mask << (8 * (i % 4));
+          cnt += mask != 0;
         }
       }
-      const uint32_t bal = __ballot_sync(0xffffffffu, mask != 0);
+      int incl = cnt;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
+      }
       __syncthreads();
-      if (lane == 0) sm.ints[warp] = __popc(bal);
+      if (lane == 31) sm.ints[warp] = incl;
       __syncthreads();
       int before = 0, total = 0;
       for (int w = 0; w < kFThreads / 32; ++w) {
@@ -503,13 +563,31 @@ struct DecodeCta {
         before += (w < warp) ? x : 0;
         total += x;
       }
-      if (mask) ent[base + before + __popc(bal & ((1u << lane) - 1u))] = ((uint32_t)n << 8) | mask;
+      int pos = base + before + incl - cnt;
+#pragma unroll
+      for (int i = 0; i < kTRun; ++i) {
+        const uint32_t mask = (packed[i / 4] >> (8 * (i % 4))) & 0xffu;
+        if (i < per && mask) ent[pos++] = ((uint32_t)(n0 + t0 + i) << 8) | mask;
+      }
       base += total;
     }
 #pragma unroll
     for (int h = 0; h < G; ++h) {
-      const int v = block_sum_int(hc[h], sm.ints);
-      if (threadIdx.x == 0 && v) atomicAdd(P.hcnt + (int64_t)g * G + h, v);
+      int v = hc[h];
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+      hc[h] = v;
+    }
+    __syncthreads();
+    if (lane == 0) {
+#pragma unroll
+      for (int h = 0; h < G; ++h) reinterpret_cast<int*>(sm.tmp)[warp * G + h] = hc[h];
+    }
+    __syncthreads();
+    if (threadIdx.x < G) {
+      int v = 0;
+      for (int w = 0; w < kFThreads / 32; ++w) v += reinterpret_cast<int*>(sm.tmp)[w * G + threadIdx.x];
+      if (v) atomicAdd(P.hcnt + (int64_t)g * G + threadIdx.x, v);
     }
     if (threadIdx.x == 0) P.ccnt[(int64_t)g * P.max_nch + j] = (uint32_t)base;
     arrive(P.bar + (int64_t)g * 4 + 2);
@@ -518,8 +596,7 @@ struct DecodeCta {
   // attention over rows [0, cnt) given by rowfn(i, kp, vp, mask); result in sm.res
   template <class RowFn>
   __device__ void attend_list(const float* q_s, int cnt, RowFn rowfn) {
-    constexpr int R = AttnCfg<G>::kRows;
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, hl = lane & 15;
+    const int hl = threadIdx.x & 15;
     float q[G][8];
 #pragma unroll
     for (int h = 0; h < G; ++h)
@@ -527,19 +604,8 @@ struct DecodeCta {
       for (int e = 0; e < 8; ++e) q[h][e] = q_s[h * kD + hl * 8 + e];
     AttnState<G> st;
     st.init();
-    for (int wb = warp * 2 * R; wb < cnt; wb += (kFThreads / 32) * 2 * R) {
-      const uint16_t* kp[R];
-      const uint16_t* vp[R];
-      uint32_t mask[R];
-#pragma unroll
-      for (int r = 0; r < R; ++r) {
-        const int i = wb + (lane >> 4) * R + r;
-        kp[r] = nullptr; vp[r] = nullptr; mask[r] = 0;
-        if (i < cnt) rowfn(i, kp[r], vp[r], mask[r]);
-      }
-      attend_step<G>(st, q, kp, vp, mask, hl);
-    }
-    attend_merge<G>(st, sm.attn, sm.res, kFThreads);
+    attend_rows<G>(st, q, cnt, rowfn, sm.stage, kFThreads);
+    attend_merge<G>(st, reinterpret_cast<float*>(sm.stage), sm.res, kFThreads);
   }
 
   // ------------------------------------------------------------ phase W
@@ -589,10 +655,10 @@ struct DecodeCta {
     uint16_t* orow = P.out + ((int64_t)b * P.L.Hq + kvh * G) * kD;
     const float* tparts = P.part + (int64_t)(sm.cbase[g] + team * kTeam) * stride;
     if (nteams == 1) {
-      merge_partials<G>(tparts, tcount, nullptr, orow, kFThreads);
+      merge_partials<G>(tparts, tcount, nullptr, orow, reinterpret_cast<float*>(sm.stage), kFThreads);
     } else {
       merge_partials<G>(tparts, tcount, P.tpart + (int64_t)(sm.cbase[g] + team) * stride,
-                        nullptr, kFThreads);
+                        nullptr, reinterpret_cast<float*>(sm.stage), kFThreads);
       __syncthreads();
       if (threadIdx.x == 0) {
         __threadfence();
@@ -601,7 +667,8 @@ struct DecodeCta {
       __syncthreads();
       if (!sm.ints[49]) return;
       __threadfence();
-      merge_partials<G>(P.tpart + (int64_t)sm.cbase[g] * stride, nteams, nullptr, orow, kFThreads);
+      merge_partials<G>(P.tpart + (int64_t)sm.cbase[g] * stride, nteams, nullptr, orow,
+                        reinterpret_cast<float*>(sm.stage), kFThreads);
     }
     if (threadIdx.x < G)
       P.sel_counts[(int64_t)b * P.L.Hq + kvh * G + threadIdx.x] =
@@ -610,22 +677,28 @@ struct DecodeCta {
   }
 
   // ------------------------------------------------------------ local items
-  // Takes and runs one local item; false when the queue is empty.
-  __device__ bool local_item() {
+  // Runs local items from the global queue until it is empty. Thread 0 takes the next index
+  // while the current item runs, so the queue costs one atomic round trip in total.
+  __device__ void local_items() {
+    if (threadIdx.x == 0) sm.ints[33] = (int)atomicAdd(P.misc + 0, 1u);
     __syncthreads();
-    if (sm.ints[34]) return false;
-    if (threadIdx.x == 0) {
-      const uint32_t it = atomicAdd(P.misc + 0, 1u);
-      sm.ints[33] = (int)it;
-      if ((int)it >= P.n_loc_items) sm.ints[34] = 1;
+    int li = sm.ints[33];
+    while (li < P.n_loc_items) {
+      __syncthreads();
+      unsigned int next = 0;
+      if (threadIdx.x == 0) next = atomicAdd(P.misc + 0, 1u);
+      local_item(li);
+      if (threadIdx.x == 0) sm.ints[33] = (int)next;
+      __syncthreads();
+      li = sm.ints[33];
     }
-    __syncthreads();
-    const int li = sm.ints[33];
-    if (li >= P.n_loc_items) return false;
+  }
+
+  __device__ void local_item(int li) {
     const int lg = li / P.PL, piece = li % P.PL;
     const int b = lg / P.L.n_loc, x = lg % P.L.n_loc, kvh = P.L.loc_kv[x];
     const int N = sm.N[b];
-    if (N == 0) return true;                        // invalid sequence: outputs zeroed in plan
+    if (N == 0) return;                             // invalid sequence: outputs zeroed in plan
     const int nrows_all = min(N, P.L.ring);
     const int r0 = piece * P.RL;
     const int nrows = max(0, min(nrows_all - r0, P.RL));
@@ -651,38 +724,46 @@ struct DecodeCta {
     if (sm.ints[50]) {
       __threadfence();
       merge_partials<G>(P.lpart + (int64_t)lg * P.PL * stride, P.PL, nullptr,
-                        P.out + ((int64_t)b * P.L.Hq + kvh * G) * kD, kFThreads);
+                        P.out + ((int64_t)b * P.L.Hq + kvh * G) * kD,
+                        reinterpret_cast<float*>(sm.stage), kFThreads);
       if (threadIdx.x < G) P.sel_counts[(int64_t)b * P.L.Hq + kvh * G + threadIdx.x] = nrows_all;
     }
     __syncthreads();
-    return true;
   }
 
   __device__ void run() {
-    if (threadIdx.x == 0) sm.ints[34] = 0;
-    __syncthreads();
+    trace(kEvStart);
     plan();
+    trace(kEvPlan);
     bool ok = true;
     // phase-major over this CTA's chunks: no wait ever depends on a later phase
     for (int k = blockIdx.x; k < NC; k += P.P) phase_score(k);
+    trace(kEvScore);
     for (int k = blockIdx.x; ok && k < NC; k += P.P) {
       const int g = group_of(k);
       ok = wait_for(P.bar + (int64_t)g * 4 + 0, (uint32_t)nch(g));
+      trace(kEvWait1);
       if (ok) phase_hist(k);
+      trace(kEvHist);
     }
     for (int k = blockIdx.x; ok && k < NC; k += P.P) {
       const int g = group_of(k);
       ok = wait_for(P.bar + (int64_t)g * 4 + 1, (uint32_t)nch(g));
+      trace(kEvWait2);
       if (ok) phase_select(k);
+      trace(kEvSelect);
     }
     for (int k = blockIdx.x; ok && k < NC; k += P.P) {
       const int g = group_of(k);
       ok = wait_for(P.bar + (int64_t)g * 4 + 2, (uint32_t)nch(g));
+      trace(kEvWait3);
       if (ok) phase_attend(k);
+      trace(kEvAttend);
     }
     if (!ok) return;
-    while (local_item()) {
-    }
+    local_items();
+    trace(kEvLocal);
+    trace(kEvEnd);
   }
 };
 

@@ -249,13 +249,16 @@ def _ret_mask_qwen(seed: int, layers: int = 36, hkv: int = 8, n_ret: int = 43) -
 
 
 # Query temperatures (lam) per workload; see the module docstring.
-# (concentrated, diffuse): at 32K with 4-sigma clusters these keep about 420 and 2500 tokens
-# per head on average at p = 0.9.
+# (concentrated, diffuse). At 32K with 4-sigma clusters (1, 2, 5) they keep about 420 and 2500
+# tokens per head on average at p = 0.9. Longer contexts need a sharper query for the same
+# sparsity: at 128K (3) about 1.5-3K tokens per head (about 95% sparse), at 1M (4) several
+# thousand per head (about 98.5% sparse), in line with the sparsity the paper's notes report
+# growing with context length (89.2% at 64K, above 97% at 512K).
 LAM = {
     1: (1.67, 1.97),
     2: (1.67, 1.97),
-    3: (1.67, 1.97),
-    4: (1.67, 1.97),
+    3: (2.45, 2.65),
+    4: (3.3, 3.3),
     5: (1.67, 1.97),
 }
 
