@@ -28,7 +28,7 @@ struct Plan {
   int64_t maxN_pad;
   size_t off_ctrl, ctrl_bytes;
   size_t off_lohi, off_hcnt, off_bar, off_team, off_locarr, off_misc, off_hist;
-  size_t off_scores, off_ent, off_ccnt, off_part, off_tpart, off_lpart, off_trace, total;
+  size_t off_scores, off_ent, off_ccnt, off_cstat, off_part, off_tpart, off_lpart, off_trace, total;
 };
 
 int check_desc(const rtp_layer_desc* d, LayerShape& L) {
@@ -104,6 +104,7 @@ int make_plan(const rtp_layer_desc* d, Plan& pl) {
   pl.off_scores = o; o = align256(o + sizeof(float) * pl.n_groups * G * pl.maxN_pad);
   pl.off_ent = o;    o = align256(o + sizeof(uint32_t) * pl.n_groups * pl.maxN_pad);
   pl.off_ccnt = o;   o = align256(o + sizeof(uint32_t) * pl.n_groups * pl.max_nch);
+  pl.off_cstat = o;  o = align256(o + sizeof(float) * 2 * pl.n_groups * pl.max_nch * G);
   pl.off_part = o;   o = align256(o + part_bytes * pl.NC_max);
   pl.off_tpart = o;  o = align256(o + part_bytes * pl.NC_max);
   pl.off_lpart = o;  o = align256(o + part_bytes * std::max(pl.n_loc_items, 1));
@@ -154,18 +155,18 @@ int smem_layout(DecodeParams& P, const Plan& pl, int smem_optin) {
   P.sm_qloc = o;  o = align16(o + 4 * G * kD);
   P.sm_qidx = o;  o = align16(o + 4 * G * kR);
   P.sm_tmp = o;   o = align16(o + 4 * kFThreads);
-  P.sm_hist = o;  o = align16(o + 8 * G * kBins);
+  P.sm_hist = o;  o = align16(o + 8 * G * kHistStride);
   P.sm_N = o;     o = align16(o + 4 * P.L.B);
   P.sm_cbase = o; o = align16(o + 4 * (pl.n_groups + 1));
   P.sm_pref = o;  o = align16(o + 4 * (pl.max_nch + 1));
   P.sm_int = o;   o = align16(o + 4 * 64);
   P.sm_scores = o;
   const int budget = smem_optin - 1024;
-  int cap = (budget - o) / (4 * G);
+  int cap = (budget - o) / (4 * G) - kHeadPad;
   cap = std::min(cap, 16384) / 256 * 256;
   if (cap < 256) cap = 0;
   P.C_cap = cap;
-  return o + 4 * G * cap;
+  return o + 4 * G * (cap + kHeadPad);
 }
 
 template <int G>
@@ -315,6 +316,7 @@ int rtp_decode_step(const rtp_layer_desc* desc, const rtp_cache* cache, const ui
   P.scores = at<float>(ws, pl.off_scores);
   P.ent = at<uint32_t>(ws, pl.off_ent);
   P.ccnt = at<uint32_t>(ws, pl.off_ccnt);
+  P.cstat = at<float2>(ws, pl.off_cstat);
   P.part = at<float>(ws, pl.off_part);
   P.tpart = at<float>(ws, pl.off_tpart);
   P.lpart = at<float>(ws, pl.off_lpart);

@@ -174,6 +174,7 @@ __device__ __forceinline__ void attend_rows(AttnState<G>& st, const float (&q)[G
   int wb = warp * 2 * R;
   int s = 0;
   if (wb < cnt) issue(wb, 0, mask_cur);
+#pragma unroll 1
   for (; wb < cnt; wb += step, s ^= 1) {
     if (wb + step < cnt) issue(wb + step, s ^ 1, mask_nxt);
     else cp_async_commit();                                   // keep one group per step
@@ -233,6 +234,7 @@ __device__ __forceinline__ void attend_merge(AttnState<G>& st, float* scratch, f
     }
   }
   __syncthreads();
+#pragma unroll 1
   for (int o = t; o < G * kD; o += nthreads) {
     const int h = o / kD, dch = o % kD;
     float M = -INFINITY;
@@ -253,14 +255,15 @@ __device__ __forceinline__ void attend_merge(AttnState<G>& st, float* scratch, f
 
 // Merges n <= kMaxMerge partial states (stride G*(2+128) floats, global memory written by
 // other CTAs) into `dst` (same format) or, when out_rows is given, into the bf16 output rows
-// of the G heads. scratch: >= 2 * kMaxMerge * G + G floats of shared memory.
+// of the G heads. Every load is issued before the first barrier (one round trip for G <= 4).
+// scratch: >= 2 * kMaxMerge * G + 2 * G floats of shared memory.
 constexpr int kMaxMerge = 64;
 template <int G>
 __device__ __forceinline__ void merge_partials(const float* parts, int n, float* dst,
                                                uint16_t* out_rows, float* scratch, int nthreads) {
   float* fM = scratch;                 // [n][G]: max, then the weight 2^(M_i - M)
   float* fL = scratch + kMaxMerge * G; // [n][G]
-  float* tot = fL + kMaxMerge * G;     // [G]: M, then L
+  float* tot = fL + kMaxMerge * G;     // [G]: M, then [G + h]: L
   const int t = threadIdx.x;
   for (int o = t; o < n * G; o += nthreads) {
     const int i = o / G, h = o % G;
@@ -268,38 +271,43 @@ __device__ __forceinline__ void merge_partials(const float* parts, int n, float*
     fM[o] = __ldcg(pp);
     fL[o] = __ldcg(pp + 1);
   }
-  __syncthreads();
-  if (t < G) {
-    float M = -INFINITY;
-    for (int i = 0; i < n; ++i) M = fmaxf(M, fM[i * G + t]);
-    float Ls = 0.f;
-    for (int i = 0; i < n; ++i) {
-      const float f = (M == -INFINITY || fM[i * G + t] == -INFINITY) ? 0.f : exp2f(fM[i * G + t] - M);
-      fM[i * G + t] = f;
-      Ls += fL[i * G + t] * f;
-    }
-    tot[t] = M;
-    tot[G + t] = Ls;
-  }
-  __syncthreads();
-  for (int o = t; o < G * kD; o += nthreads) {
+  constexpr int kBatch = 32;            // partials whose values one thread holds in registers
+#pragma unroll 1
+  for (int ob = 0; ob < G * kD; ob += nthreads) {
+    const int o = ob + t;
     const int h = o / kD, dch = o % kD;
-    float A = 0.f;
-    int i = 0;
-    for (; i + 8 <= n; i += 8) {
-      float a[8];
+    float a[kBatch];
 #pragma unroll
-      for (int u = 0; u < 8; ++u) a[u] = __ldcg(parts + ((int64_t)(i + u) * G + h) * (kD + 2) + 2 + dch);
-#pragma unroll
-      for (int u = 0; u < 8; ++u) A = fmaf(a[u], fM[(i + u) * G + h], A);
+    for (int i = 0; i < kBatch; ++i)
+      a[i] = (i < n && o < G * kD) ? __ldcg(parts + ((int64_t)i * G + h) * (kD + 2) + 2 + dch) : 0.f;
+    __syncthreads();
+    if (ob == 0 && t < G) {
+      float M = -INFINITY;
+      for (int i = 0; i < n; ++i) M = fmaxf(M, fM[i * G + t]);
+      float Ls = 0.f;
+      for (int i = 0; i < n; ++i) {
+        const float f = (M == -INFINITY || fM[i * G + t] == -INFINITY) ? 0.f : exp2f(fM[i * G + t] - M);
+        fM[i * G + t] = f;
+        Ls += fL[i * G + t] * f;
+      }
+      tot[t] = M;
+      tot[G + t] = Ls;
     }
-    for (; i < n; ++i) A = fmaf(__ldcg(parts + ((int64_t)i * G + h) * (kD + 2) + 2 + dch), fM[i * G + h], A);
-    const float Ls = tot[G + h];
-    if (out_rows) {
-      out_rows[(int64_t)h * kD + dch] = f2bf_rn(Ls > 0.f ? A / Ls : 0.f);
-    } else {
-      dst[h * (kD + 2) + 2 + dch] = A;
-      if (dch == 0) { dst[h * (kD + 2)] = tot[h]; dst[h * (kD + 2) + 1] = Ls; }
+    __syncthreads();
+    if (o < G * kD) {
+      float A = 0.f;
+#pragma unroll
+      for (int i = 0; i < kBatch; ++i)
+        if (i < n) A = fmaf(a[i], fM[i * G + h], A);
+      for (int i = kBatch; i < n; ++i)
+        A = fmaf(__ldcg(parts + ((int64_t)i * G + h) * (kD + 2) + 2 + dch), fM[i * G + h], A);
+      const float Ls = tot[G + h];
+      if (out_rows) {
+        out_rows[(int64_t)h * kD + dch] = f2bf_rn(Ls > 0.f ? A / Ls : 0.f);
+      } else {
+        dst[h * (kD + 2) + 2 + dch] = A;
+        if (dch == 0) { dst[h * (kD + 2)] = tot[h]; dst[h * (kD + 2) + 1] = Ls; }
+      }
     }
   }
   __syncthreads();

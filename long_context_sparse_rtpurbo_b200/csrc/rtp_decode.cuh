@@ -8,7 +8,9 @@
 // is found sort-free with a 256-bin histogram per head, fused with the scoring.
 //
 // Work split. A retrieval group is one (sequence, retrieval KV head) with its G query heads;
-// its N tokens are cut into chunks of C tokens; chunk k of the launch runs on CTA k mod P.
+// its N tokens are cut into chunks of C tokens. CTAs [0, P_ret) run the retrieval chunks
+// (chunk k on CTA k mod P_ret, in waves that fit the shared-memory score buffers); the other
+// CTAs start on the local heads at once, P_ret following the byte share of the two sides.
 // Per group the chunks pass four phases, separated by arrival counters in global memory:
 //   S  scores of the G heads for the chunk's tokens (kept in shared memory when every CTA
 //      owns at most one chunk, else in the workspace); group min / max by integer atomics.
@@ -19,9 +21,8 @@
 //   W  the group's entries are split evenly over its chunks' CTAs; each gathers its rows
 //      once for all G heads (a head that did not select a row skips it) and writes a
 //      partial softmax state; partials merge in teams of 32, the last team writes out.
-// Local items (a slice of one local head's ring) come from a global queue. CTAs without a
-// retrieval chunk start on them at once; the others join when their chunks are done, so a
-// local item never delays a phase of the retrieval chain.
+// Local items (a slice of one local head's ring) come from a global queue; retrieval CTAs
+// join when their chunks are done, so a local item never delays the retrieval chain.
 // Every wait is bounded (clock64 limit): on expiry the kernel records RTP_ETIMEOUT, raises
 // an abort flag that ends every other wait, and returns.
 #pragma once
@@ -33,6 +34,8 @@ namespace rtp {
 
 constexpr int kFThreads = 512;          // threads of the decode kernel
 constexpr int kTeam = 32;               // partials merged per team
+constexpr int kHeadPad = 8;             // words between the heads' rows of shared buffers
+constexpr int kHistStride = 256 + kHeadPad;
 
 struct DecodeParams {
   LayerShape L;
@@ -72,6 +75,7 @@ struct DecodeParams {
   float* scores;               // [n_groups][G][maxN_pad] (when chunks do not fit on chip)
   uint32_t* ent;               // [n_groups][maxN_pad]
   uint32_t* ccnt;              // [n_groups][max_nch]
+  float2* cstat;               // [n_groups][max_nch][G] chunk (max score, sum exp(s - max))
   float* part;                 // [NC_max][G][130]
   float* tpart;                // [NC_max][G][130]
   float* lpart;                // [n_loc_items][G][130]
@@ -80,14 +84,18 @@ struct DecodeParams {
 
 // Phase-boundary timestamps, recorded only when built with -DRTP_TRACE.
 enum TraceEvent { kEvStart, kEvPlan, kEvScore, kEvWait1, kEvHist, kEvWait2, kEvSelect, kEvWait3,
-                  kEvAttend, kEvLocal, kEvEnd, kTraceEvents = 16 };
+                  kEvAttend, kEvLocal, kEvEnd, kEvS0, kEvS1, kEvH0, kEvH1, kEvH2, kEvT0, kEvT1,
+                  kEvW0, kEvW1, kEvW2, kTraceEvents = 32 };
 
 // ------------------------------------------------------------------------------ helpers
 __device__ __forceinline__ int seq_len_checked(const DecodeParams& P, int b) {
-  const int N = P.seq_lens[b];
-  if (N < 1 || N > P.cache.seq_cap[b] || (int64_t)N > P.L.maxN) return 0;
-  if (P.L.n_ret > 0 && (P.cache.seq_off[b] < 0 || P.cache.seq_off[b] + N > P.L.T_total)) return 0;
-  return N;
+  // three independent loads, one round trip
+  const int N = __ldg(P.seq_lens + b);
+  const int cap = __ldg(P.cache.seq_cap + b);
+  const int64_t off = __ldg(P.cache.seq_off + b);
+  bool ok = N >= 1 && N <= cap && (int64_t)N <= P.L.maxN;
+  if (P.L.n_ret > 0) ok = ok && off >= 0 && off + N <= P.L.T_total;
+  return ok ? N : 0;
 }
 
 __device__ __forceinline__ uint32_t ld_acquire(const uint32_t* p) {
@@ -105,6 +113,19 @@ __device__ __forceinline__ int block_sum_int(int v, int* scratch /*>= 32 ints*/)
   __syncthreads();
   int s = 0;
   for (int w = 0; w < kFThreads / 32; ++w) s += scratch[w];
+  __syncthreads();
+  return s;
+}
+
+__device__ __forceinline__ int block_max_int(int v, int* scratch /*>= 32 ints*/) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = max(v, __shfl_xor_sync(0xffffffffu, v, o));
+  __syncthreads();
+  if (lane == 0) scratch[warp] = v;
+  __syncthreads();
+  int s = scratch[0];
+  for (int w = 1; w < kFThreads / 32; ++w) s = max(s, scratch[w]);
   __syncthreads();
   return s;
 }
@@ -173,8 +194,8 @@ template <int G> struct Smem {
 
 // RoPE'd, pre-scaled query of the G heads of KV head kvh at position N - 1 -> q_s[G][128].
 template <int G>
-__device__ __forceinline__ void rope_query(const DecodeParams& P, int b, int kvh, int N,
-                                           float* q_s) {
+__device__ __noinline__ void rope_query(const DecodeParams& P, int b, int kvh, int N,
+                                        float* q_s) {
   const int t = threadIdx.x;
   if (t < kD) {
     const int i = t & 63;
@@ -237,7 +258,7 @@ template <int G>
 struct DecodeCta {
   const DecodeParams& P;
   Smem<G> sm;
-  int C, NC, smem_mode;
+  int C, NC, smem_mode, P_ret;
 
   __device__ DecodeCta(const DecodeParams& p, unsigned char* base) : P(p), sm(base, p) {}
 
@@ -249,7 +270,7 @@ struct DecodeCta {
     return smem_mode ? sm.scores : P.scores + (int64_t)g * G * P.maxN_pad + (int64_t)j * C;
   }
   __device__ __forceinline__ int64_t score_hstride() const {
-    return smem_mode ? (int64_t)P.C_cap : P.maxN_pad;
+    return smem_mode ? (int64_t)P.C_cap + kHeadPad : P.maxN_pad;
   }
 
   __device__ __forceinline__ void trace(int ev) {
@@ -307,23 +328,44 @@ struct DecodeCta {
     const int t = threadIdx.x;
     for (int b = t; b < P.L.B; b += kFThreads) sm.N[b] = seq_len_checked(P, b);
     __syncthreads();
-    int part = 0;
-    for (int b = t; b < P.L.B; b += kFThreads) part += sm.N[b];
-    const long long Tr = (long long)block_sum_int(part, sm.ints) * P.L.n_ret;
-    long long c = 256;
-    smem_mode = 0;
-    if (P.P > P.n_groups && Tr > 0) {
-      c = (Tr + (P.P - P.n_groups) - 1) / (P.P - P.n_groups);
-      c = max(c, (long long)P.C_min);
-      c = (c + 255) / 256 * 256;
-      if (c <= P.C_cap) smem_mode = 1;
+    int sumN = 0, sumL = 0, maxN = 0;
+    for (int b = t; b < P.L.B; b += kFThreads) {
+      sumN += sm.N[b];
+      sumL += min(sm.N[b], P.L.ring);
+      maxN = max(maxN, sm.N[b]);
     }
-    if (!smem_mode) {
-      c = (Tr + 2LL * P.P - 1) / (2LL * P.P);
-      c = max(c, (long long)max(P.C_min, 256));
-      c = (c + 255) / 256 * 256;
+    const long long Tr = (long long)block_sum_int(sumN, sm.ints) * P.L.n_ret;
+    const long long loc_rows = (long long)block_sum_int(sumL, sm.ints) * P.L.n_loc;
+    maxN = block_max_int(maxN, sm.ints);
+    // CTAs [0, P_ret) run the retrieval chain, the others start on local items at once; the
+    // split follows the bytes of each side (index read twice as a proxy for index + gather).
+    P_ret = 0;
+    C = 1024;
+    smem_mode = 1;
+    if (Tr > 0) {
+      const double ret_b = 64.0 * (double)Tr, loc_b = 512.0 * (double)loc_rows;
+      int pr = (int)((double)P.P * ret_b / (ret_b + loc_b) + 0.5);
+      pr = max(1, min(P.P, pr));
+      const long long one_wave = (Tr + P.C_cap - 1) / P.C_cap + P.n_groups;   // chunks at C_cap
+      pr = max(pr, (int)min((long long)P.P, one_wave));
+      const int need = (maxN + P.C_cap - 1) / P.C_cap;          // a group within one wave
+      if (need > P.P) {
+        smem_mode = 0;                                          // scores spill to the workspace
+        pr = P.P;
+        long long c = (Tr + 2LL * P.P - 1) / (2LL * P.P);
+        c = max(c, (long long)P.C_min);
+        C = (int)((c + 255) / 256 * 256);
+      } else {
+        pr = max(pr, need);
+        long long c = (pr > P.n_groups) ? (Tr + (pr - P.n_groups) - 1) / (pr - P.n_groups)
+                                        : (Tr + pr - 1) / pr;
+        c = max(c, (long long)P.C_min);
+        c = max(c, (long long)((maxN + pr - 1) / pr));
+        c = (c + 255) / 256 * 256;
+        C = (int)min(c, (long long)P.C_cap);                   // C_cap: more than one wave
+      }
+      P_ret = pr;
     }
-    C = (int)c;
     for (int g = t; g < P.n_groups; g += kFThreads) sm.cbase[g] = (gN(g) + C - 1) / C;
     __syncthreads();
     NC = block_scan_excl(sm.cbase, P.n_groups, sm.ints);
@@ -366,7 +408,9 @@ struct DecodeCta {
     __syncthreads();                       // the stage buffer may still be read by a merge
 #pragma unroll
     for (int st = 0; st < kSStages - 1; ++st) issue(st);
+    rope_query<G>(P, b, kvh, N, sm.qret);   // for phase W; overlaps the first loads
     index_query<G>(P, b, kvh, sm.qidx, sm.tmp);
+    trace(kEvS0);
     float qi[G][kR];
 #pragma unroll
     for (int h = 0; h < G; ++h)
@@ -377,12 +421,14 @@ struct DecodeCta {
     for (int h = 0; h < G; ++h) { mn[h] = INFINITY; mx[h] = -INFINITY; }
     float* sc = score_ptr(g, j);
     const int64_t hs = score_hstride();
+#pragma unroll 1
     for (int st = 0; st < nst; ++st) {
       issue(st + kSStages - 1);
       cp_async_wait<kSStages - 1>();
       __syncthreads();
       const int rows = min(kSRows, n1 - n0 - st * kSRows);
       const unsigned char* buf = sm.stage + (st % kSStages) * (kSRows * 32);
+#pragma unroll 1
       for (int i = threadIdx.x; i < rows; i += kFThreads) {
         const uint4 a = *reinterpret_cast<const uint4*>(buf + i * 32);
         const uint4 c2 = *reinterpret_cast<const uint4*>(buf + i * 32 + 16);
@@ -403,8 +449,9 @@ struct DecodeCta {
       __syncthreads();                     // before the slot is refilled
     }
     cp_async_wait<0>();
+    trace(kEvS1);
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    float* red = sm.tmp;                    // [2][G][16]
+    float* red = sm.tmp;                    // [2][G][16], then [G][16]
     __syncthreads();
 #pragma unroll
     for (int h = 0; h < G; ++h) {
@@ -416,43 +463,115 @@ struct DecodeCta {
       if (lane == 0) { red[(0 * G + h) * 16 + warp] = mn[h]; red[(1 * G + h) * 16 + warp] = mx[h]; }
     }
     __syncthreads();
+    float cmax[G];                          // the chunk's max per head (every thread)
+#pragma unroll
+    for (int h = 0; h < G; ++h) {
+      float z = red[(1 * G + h) * 16];
+      for (int w = 1; w < kFThreads / 32; ++w) z = fmaxf(z, red[(1 * G + h) * 16 + w]);
+      cmax[h] = z;
+    }
     if (threadIdx.x < G) {
       const int h = threadIdx.x;
-      float a = red[(0 * G + h) * 16], z = red[(1 * G + h) * 16];
-      for (int w = 1; w < kFThreads / 32; ++w) {
-        a = fminf(a, red[(0 * G + h) * 16 + w]);
-        z = fmaxf(z, red[(1 * G + h) * 16 + w]);
-      }
+      float a = red[(0 * G + h) * 16];
+      for (int w = 1; w < kFThreads / 32; ++w) a = fminf(a, red[(0 * G + h) * 16 + w]);
       atomicMax(P.lohi + ((int64_t)g * 2 + 0) * G + h, ~f2ord(a));
-      atomicMax(P.lohi + ((int64_t)g * 2 + 1) * G + h, f2ord(z));
+      atomicMax(P.lohi + ((int64_t)g * 2 + 1) * G + h, f2ord(cmax[h]));
+    }
+    // the chunk's total mass relative to its max: sum exp(s - cmax) over the shared scores
+    float ls[G];
+#pragma unroll
+    for (int h = 0; h < G; ++h) ls[h] = 0.f;
+#pragma unroll 4
+    for (int i = threadIdx.x; i < n1 - n0; i += kFThreads)
+#pragma unroll
+      for (int h = 0; h < G; ++h) ls[h] += exp2f((sc[h * hs + i] - cmax[h]) * kLog2e);
+    __syncthreads();
+#pragma unroll
+    for (int h = 0; h < G; ++h) {
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) ls[h] += __shfl_xor_sync(0xffffffffu, ls[h], o);
+      if (lane == 0) red[h * 16 + warp] = ls[h];
+    }
+    __syncthreads();
+    if (threadIdx.x < G) {
+      const int h = threadIdx.x;
+      double l = 0.0;                       // fixed order
+      for (int w = 0; w < kFThreads / 32; ++w) l += (double)red[h * 16 + w];
+      P.cstat[((int64_t)g * P.max_nch + j) * G + h] = make_float2(cmax[h], (float)l);
     }
     arrive(P.bar + (int64_t)g * 4 + 0);
   }
 
+  // Total mass T_h = sum over the group's chunks of L_c exp(hi_c - hi), for the G heads,
+  // from the chunk statistics of phase S (double, fixed order: every CTA gets the same value)
+  // -> sm.tot[h] (as a double in units of the head's max-score token).
+  __device__ void group_total(int g, const float* hi, double* tot) {
+    const int n = nch(g);
+    double* part = reinterpret_cast<double*>(sm.stage);      // [kFThreads]
+    const int t = threadIdx.x;
+    const int h = t % G;
+    double acc = 0.0;
+    for (int c = t / G; c < n; c += kFThreads / G) {
+      const float2 st = __ldcg(P.cstat + ((int64_t)g * P.max_nch + c) * G + h);
+      acc += (double)st.y * (double)exp2f((st.x - hi[h]) * kLog2e);
+    }
+    __syncthreads();
+    part[t] = acc;
+    __syncthreads();
+    if (t < G) {
+      double v = 0.0;
+      for (int i = t; i < kFThreads; i += G) v += part[i];
+      tot[t] = v;
+    }
+    __syncthreads();
+  }
+
   // ------------------------------------------------------------ phase H
+  // Masses are exp(s - max) in 2^-40 fixed point. Only bins at or above a cutoff bin get
+  // per-bin sums: with T the group's total mass (from phase S), every token below bin(c),
+  // c = hi + ln((1 - p) T' / N) - 2 and T' = T (1 - 1e-3), has mass below (1 - p) T' e^-2 / N,
+  // so together they hold less than (1 - p) of the total and b* can not fall under the
+  // cutoff bin. The per-bin sums use two 32-bit shared atomics per token: the low-word add
+  // returns the old value and its carry goes to the high word (exact). Lanes take interleaved
+  // (token, head) elements and the heads' rows are padded, so a warp's atomics spread over
+  // the banks.
   __device__ void phase_hist(int k) {
     const int g = group_of(k), j = k - sm.cbase[g];
     const int N = gN(g);
     const int n0 = j * C, n1 = min(N, n0 + C);
-    // 64-bit fixed-point bins as (low word, high word) pairs of 32-bit shared atomics: the
-    // low-word add returns the old value, its carry goes to the high word (exact)
     uint32_t* hlo = reinterpret_cast<uint32_t*>(sm.hist);
-    uint32_t* hhi = hlo + G * kBins;
-    for (int i = threadIdx.x; i < 2 * G * kBins; i += kFThreads) hlo[i] = 0u;
+    uint32_t* hhi = hlo + G * kHistStride;
+    for (int i = threadIdx.x; i < 2 * G * kHistStride; i += kFThreads) hlo[i] = 0u;
     float lo[G], hi[G], inv[G];
     load_range<G>(P, g, lo, hi, inv);
-    __syncthreads();
+    double* tot = reinterpret_cast<double*>(sm.tmp);          // [G]
+    group_total(g, hi, tot);
+    trace(kEvH0);
+    const int h = threadIdx.x % G;          // G divides kFThreads: the thread's head is fixed
+    float loh = 0.f, hih = 0.f, invh = 0.f;
+#pragma unroll
+    for (int hh = 0; hh < G; ++hh)
+      if (hh == h) { loh = lo[hh]; hih = hi[hh]; invh = inv[hh]; }
+    int bch = 0;
+    if (P.p < 1.0 && invh > 0.f) {
+      const float arg = (float)((1.0 - P.p) * tot[h] * (1.0 - 1e-3) / (double)N);
+      const float c = hih + logf(arg) - 2.f;
+      bch = c > loh ? bin_of(c, loh, invh) : 0;
+    }
     const float* sc = score_ptr(g, j);
     const int64_t hs = score_hstride();
-    for (int n = n0 + threadIdx.x; n < n1; n += kFThreads) {
-#pragma unroll
-      for (int h = 0; h < G; ++h) {
-        const float s = sc[h * hs + (n - n0)];
-        const float e = (s - hi[h]) * kLog2e;
-        if (e > -42.f) {                      // below 2^-41 the fixed-point mass rounds to 0
-          const unsigned long long q = __float2ull_rn(exp2f(e) * kMassScale);
+    const int len = n1 - n0;
+#pragma unroll 4
+    for (int e = threadIdx.x; e < len * G; e += kFThreads) {
+      const int nl = e / G;
+      const float sv = sc[h * hs + nl];
+      const int b = bin_of(sv, loh, invh);
+      if (b >= bch) {
+        const float ex = (sv - hih) * kLog2e;
+        if (ex > -42.f) {                     // below 2^-41 the fixed-point mass rounds to 0
+          const unsigned long long q = __float2ull_rn(exp2f(ex) * kMassScale);
+          const int bi = h * kHistStride + b;
           const uint32_t ql = (uint32_t)q, qh = (uint32_t)(q >> 32);
-          const int bi = h * kBins + bin_of(s, lo[h], inv[h]);
           const uint32_t old = atomicAdd(&hlo[bi], ql);
           const uint32_t up = qh + ((old + ql < old) ? 1u : 0u);
           if (up) atomicAdd(&hhi[bi], up);
@@ -460,36 +579,41 @@ struct DecodeCta {
       }
     }
     __syncthreads();
+    trace(kEvH1);
     unsigned long long* gh = P.hist + (int64_t)g * G * kBins;
     for (int i = threadIdx.x; i < G * kBins; i += kFThreads) {
-      const unsigned long long v = ((unsigned long long)hhi[i] << 32) | hlo[i];
+      const int hh = i / kBins, b = i % kBins;
+      const unsigned long long v =
+          ((unsigned long long)hhi[hh * kHistStride + b] << 32) | hlo[hh * kHistStride + b];
       if (v) atomicAdd(gh + i, v);
     }
+    trace(kEvH2);
     arrive(P.bar + (int64_t)g * 4 + 1);
   }
 
   // b* of the G heads of group g into sm.ints[40 + h]; warp h handles head h.
-  __device__ void find_bstar(int g) {
+  __device__ void find_bstar(int g, const float* hi) {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    double* tot = reinterpret_cast<double*>(sm.tmp);
+    if (!P.select_all) group_total(g, hi, tot);
     if (warp < G) {
       const int h = warp;
       if (P.select_all) {
         if (lane == 0) sm.ints[40 + h] = 0;
       } else {
         const unsigned long long* gh = P.hist + ((int64_t)g * G + h) * kBins;
-        unsigned long long v[8], tot = 0;
+        unsigned long long v[8], lt = 0;
 #pragma unroll
-        for (int e = 0; e < 8; ++e) { v[e] = __ldcg(gh + lane * 8 + e); tot += v[e]; }
-        unsigned long long x = tot;           // inclusive suffix sum over lanes
+        for (int e = 0; e < 8; ++e) { v[e] = __ldcg(gh + lane * 8 + e); lt += v[e]; }
+        unsigned long long x = lt;            // inclusive suffix sum over lanes
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
           const unsigned long long y = __shfl_down_sync(0xffffffffu, x, o);
           if (lane + o < 32) x += y;
         }
-        const unsigned long long T = __shfl_sync(0xffffffffu, x, 0);
-        const double thr = P.p * (double)T;
+        const double thr = P.p * tot[h] * (double)kMassScale;
         int best = -1;
-        unsigned long long cum = x - tot;
+        unsigned long long cum = x - lt;
 #pragma unroll
         for (int e = 7; e >= 0; --e) {
           cum += v[e];
@@ -514,7 +638,8 @@ struct DecodeCta {
     const int n0 = j * C, n1 = min(N, n0 + C);
     float lo[G], hi[G], inv[G];
     load_range<G>(P, g, lo, hi, inv);
-    find_bstar(g);
+    find_bstar(g, hi);
+    trace(kEvT0);
     int bs[G];
 #pragma unroll
     for (int h = 0; h < G; ++h) bs[h] = sm.ints[40 + h];
@@ -526,27 +651,23 @@ struct DecodeCta {
 #pragma unroll
     for (int h = 0; h < G; ++h) hc[h] = 0;
     int base = 0;
+    uint8_t* mk = sm.stage;                  // per-token head masks of the current tile
+#pragma unroll 1
     for (int tb = 0; tb < n1 - n0; tb += kFThreads * kTRun) {
       const int len = min(kFThreads * kTRun, n1 - n0 - tb);
       const int per = (len + kFThreads - 1) / kFThreads;
-      const int t0 = tb + threadIdx.x * per, t1 = min(tb + len, t0 + per);
-      uint32_t packed[kTRun / 4];
-#pragma unroll
-      for (int w = 0; w < kTRun / 4; ++w) packed[w] = 0u;
+      const int t0 = threadIdx.x * per, t1 = min(len, t0 + per);
       int cnt = 0;
+#pragma unroll 1
+      for (int nl = t0; nl < t1; ++nl) {
+        uint32_t mask = 0;
 #pragma unroll
-      for (int i = 0; i < kTRun; ++i) {
-        const int nl = t0 + i;
-        if (i < per && nl < t1) {
-          uint32_t mask = 0;
-#pragma unroll
-          for (int h = 0; h < G; ++h) {
-            const float sv = sc[h * hs + nl];
-            if (bin_of(sv, lo[h], inv[h]) >= bs[h]) { mask |= 1u << h; hc[h]++; }
-          }
-          packed[i / 4] |= mask << (8 * (i % 4));
-          cnt += mask != 0;
+        for (int h = 0; h < G; ++h) {
+          const float sv = sc[h * hs + tb + nl];
+          if (bin_of(sv, lo[h], inv[h]) >= bs[h]) { mask |= 1u << h; hc[h]++; }
         }
+        mk[nl] = (uint8_t)mask;
+        cnt += mask != 0;
       }
       int incl = cnt;
 #pragma unroll
@@ -564,13 +685,15 @@ struct DecodeCta {
         total += x;
       }
       int pos = base + before + incl - cnt;
-#pragma unroll
-      for (int i = 0; i < kTRun; ++i) {
-        const uint32_t mask = (packed[i / 4] >> (8 * (i % 4))) & 0xffu;
-        if (i < per && mask) ent[pos++] = ((uint32_t)(n0 + t0 + i) << 8) | mask;
+#pragma unroll 1
+      for (int nl = t0; nl < t1; ++nl) {
+        const uint32_t mask = mk[nl];
+        if (mask) ent[pos++] = ((uint32_t)(n0 + tb + nl) << 8) | mask;
       }
       base += total;
+      __syncthreads();                       // mk is rewritten by the next tile
     }
+    trace(kEvT1);
 #pragma unroll
     for (int h = 0; h < G; ++h) {
       int v = hc[h];
@@ -593,9 +716,16 @@ struct DecodeCta {
     arrive(P.bar + (int64_t)g * 4 + 2);
   }
 
-  // attention over rows [0, cnt) given by rowfn(i, kp, vp, mask); result in sm.res
-  template <class RowFn>
-  __device__ void attend_list(const float* q_s, int cnt, RowFn rowfn) {
+  // Attention over cnt rows; result in sm.res. Gather mode (ent != nullptr): row i is entry
+  // e0 + i of the group's compacted list (chunk-local runs located through sm.pref over nch
+  // chunks of Cc tokens); contiguous mode: row i is row r0 + i of kb / vb. One instance of
+  // the attention loop serves both, which keeps the kernel's code small.
+  struct Rows {
+    const uint16_t* kb; const uint16_t* vb;   // row 0 of the sequence (gather) or of the range
+    const uint32_t* ent; const int* pref; int e0, nch, Cc;
+    const uint32_t* sent;                     // the rows' entries staged in shared memory
+  };
+  __device__ __noinline__ void attend_list(const float* q_s, int cnt, const Rows R) {
     const int hl = threadIdx.x & 15;
     float q[G][8];
 #pragma unroll
@@ -604,8 +734,28 @@ struct DecodeCta {
       for (int e = 0; e < 8; ++e) q[h][e] = q_s[h * kD + hl * 8 + e];
     AttnState<G> st;
     st.init();
-    attend_rows<G>(st, q, cnt, rowfn, sm.stage, kFThreads);
+    attend_rows<G>(st, q, cnt, [&](int i, const uint16_t*& kp, const uint16_t*& vp, uint32_t& mask) {
+      int64_t n = i;
+      mask = 0xffu;
+      if (R.sent) {
+        const uint32_t w = R.sent[i];
+        n = w >> 8;
+        mask = w & 0xffu;
+      } else if (R.ent) {
+        const int e = R.e0 + i;
+        const int c = upper_index(R.pref, R.nch, e);
+        const uint32_t w = __ldcg(R.ent + (int64_t)c * R.Cc + (e - R.pref[c]));
+        n = w >> 8;
+        mask = w & 0xffu;
+      }
+      kp = R.kb + n * kD;
+      vp = R.vb + n * kD;
+    }, sm.stage, kFThreads);
     attend_merge<G>(st, reinterpret_cast<float*>(sm.stage), sm.res, kFThreads);
+  }
+
+  __device__ __noinline__ void merge(const float* parts, int n, float* dst, uint16_t* out_rows) {
+    merge_partials<G>(parts, n, dst, out_rows, reinterpret_cast<float*>(sm.stage), kFThreads);
   }
 
   // ------------------------------------------------------------ phase W
@@ -619,25 +769,27 @@ struct DecodeCta {
     __syncthreads();
     const int U = block_scan_excl(sm.pref, S, sm.ints);
     if (threadIdx.x == 0) sm.pref[S] = U;
-    rope_query<G>(P, b, kvh, N, sm.qret);
+    if (!smem_mode) rope_query<G>(P, b, kvh, N, sm.qret);   // else formed in phase S
     __syncthreads();
     const int e0 = (int)(((long long)U * j) / S), e1 = (int)(((long long)U * (j + 1)) / S);
-    const uint32_t* ent = P.ent + (int64_t)g * P.maxN_pad;
     const int64_t rowbase = (int64_t)r * P.L.T_total + P.cache.seq_off[b];
-    const uint16_t* kb = P.cache.k_ret;
-    const uint16_t* vb = P.cache.v_ret;
-    const int* pref = sm.pref;
-    const int Cc = C;
-    attend_list(sm.qret, e1 - e0, [&](int i, const uint16_t*& kp, const uint16_t*& vp,
-                                      uint32_t& mask) {
-      const int e = e0 + i;
-      const int c = upper_index(pref, S, e);
-      const uint32_t w = __ldcg(ent + (int64_t)c * Cc + (e - pref[c]));
-      const int64_t n = w >> 8;
-      mask = w & 0xffu;
-      kp = kb + (rowbase + n) * kD;
-      vp = vb + (rowbase + n) * kD;
-    });
+    const uint32_t* gent = P.ent + (int64_t)g * P.maxN_pad;
+    Rows rows{P.cache.k_ret + rowbase * kD, P.cache.v_ret + rowbase * kD, gent, sm.pref, e0, S, C,
+              nullptr};
+    // this split's entries in one batch of loads, into the (now free) score buffer
+    uint32_t* es = reinterpret_cast<uint32_t*>(sm.scores);
+    if (e1 - e0 <= P.C_cap * G) {
+      for (int i = threadIdx.x; i < e1 - e0; i += kFThreads) {
+        const int e = e0 + i;
+        const int c = upper_index(sm.pref, S, e);
+        es[i] = __ldcg(gent + (int64_t)c * C + (e - sm.pref[c]));
+      }
+      __syncthreads();
+      rows.sent = es;
+    }
+    trace(kEvW0);
+    attend_list(sm.qret, e1 - e0, rows);
+    trace(kEvW1);
     // partial -> workspace; team / group merge by the last arrivals
     const int stride = G * (kD + 2);
     float* mine = P.part + (int64_t)k * stride;
@@ -650,15 +802,15 @@ struct DecodeCta {
       sm.ints[48] = atomicAdd(P.team_arr + sm.cbase[g] + team, 1u) == (uint32_t)(tcount - 1);
     }
     __syncthreads();
+    trace(kEvW2);
     if (!sm.ints[48]) return;
     __threadfence();
     uint16_t* orow = P.out + ((int64_t)b * P.L.Hq + kvh * G) * kD;
     const float* tparts = P.part + (int64_t)(sm.cbase[g] + team * kTeam) * stride;
     if (nteams == 1) {
-      merge_partials<G>(tparts, tcount, nullptr, orow, reinterpret_cast<float*>(sm.stage), kFThreads);
+      merge(tparts, tcount, nullptr, orow);
     } else {
-      merge_partials<G>(tparts, tcount, P.tpart + (int64_t)(sm.cbase[g] + team) * stride,
-                        nullptr, reinterpret_cast<float*>(sm.stage), kFThreads);
+      merge(tparts, tcount, P.tpart + (int64_t)(sm.cbase[g] + team) * stride, nullptr);
       __syncthreads();
       if (threadIdx.x == 0) {
         __threadfence();
@@ -667,8 +819,7 @@ struct DecodeCta {
       __syncthreads();
       if (!sm.ints[49]) return;
       __threadfence();
-      merge_partials<G>(P.tpart + (int64_t)sm.cbase[g] * stride, nteams, nullptr, orow,
-                        reinterpret_cast<float*>(sm.stage), kFThreads);
+      merge(P.tpart + (int64_t)sm.cbase[g] * stride, nteams, nullptr, orow);
     }
     if (threadIdx.x < G)
       P.sel_counts[(int64_t)b * P.L.Hq + kvh * G + threadIdx.x] =
@@ -704,14 +855,10 @@ struct DecodeCta {
     const int nrows = max(0, min(nrows_all - r0, P.RL));
     rope_query<G>(P, b, kvh, N, sm.qloc);
     __syncthreads();
-    const uint16_t* kb = P.cache.k_loc + ((int64_t)x * P.L.B + b) * P.L.ring * kD;
-    const uint16_t* vb = P.cache.v_loc + ((int64_t)x * P.L.B + b) * P.L.ring * kD;
-    attend_list(sm.qloc, nrows, [&](int i, const uint16_t*& kp, const uint16_t*& vp,
-                                    uint32_t& mask) {
-      kp = kb + (int64_t)(r0 + i) * kD;
-      vp = vb + (int64_t)(r0 + i) * kD;
-      mask = 0xffu;
-    });
+    const int64_t ring0 = ((int64_t)x * P.L.B + b) * P.L.ring + r0;
+    Rows rows{P.cache.k_loc + ring0 * kD, P.cache.v_loc + ring0 * kD, nullptr, nullptr, 0, 0, 0,
+              nullptr};
+    attend_list(sm.qloc, nrows, rows);
     const int stride = G * (kD + 2);
     float* mine = P.lpart + (int64_t)li * stride;
     for (int o = threadIdx.x; o < stride; o += kFThreads) mine[o] = sm.res[o];
@@ -723,9 +870,8 @@ struct DecodeCta {
     __syncthreads();
     if (sm.ints[50]) {
       __threadfence();
-      merge_partials<G>(P.lpart + (int64_t)lg * P.PL * stride, P.PL, nullptr,
-                        P.out + ((int64_t)b * P.L.Hq + kvh * G) * kD,
-                        reinterpret_cast<float*>(sm.stage), kFThreads);
+      merge(P.lpart + (int64_t)lg * P.PL * stride, P.PL, nullptr,
+            P.out + ((int64_t)b * P.L.Hq + kvh * G) * kD);
       if (threadIdx.x < G) P.sel_counts[(int64_t)b * P.L.Hq + kvh * G + threadIdx.x] = nrows_all;
     }
     __syncthreads();
@@ -736,29 +882,51 @@ struct DecodeCta {
     plan();
     trace(kEvPlan);
     bool ok = true;
-    // phase-major over this CTA's chunks: no wait ever depends on a later phase
-    for (int k = blockIdx.x; k < NC; k += P.P) phase_score(k);
-    trace(kEvScore);
-    for (int k = blockIdx.x; ok && k < NC; k += P.P) {
-      const int g = group_of(k);
-      ok = wait_for(P.bar + (int64_t)g * 4 + 0, (uint32_t)nch(g));
-      trace(kEvWait1);
-      if (ok) phase_hist(k);
-      trace(kEvHist);
-    }
-    for (int k = blockIdx.x; ok && k < NC; k += P.P) {
-      const int g = group_of(k);
-      ok = wait_for(P.bar + (int64_t)g * 4 + 1, (uint32_t)nch(g));
-      trace(kEvWait2);
-      if (ok) phase_select(k);
-      trace(kEvSelect);
-    }
-    for (int k = blockIdx.x; ok && k < NC; k += P.P) {
-      const int g = group_of(k);
-      ok = wait_for(P.bar + (int64_t)g * 4 + 2, (uint32_t)nch(g));
-      trace(kEvWait3);
-      if (ok) phase_attend(k);
-      trace(kEvAttend);
+    if ((int)blockIdx.x < P_ret) {
+      if (smem_mode) {
+        // waves: chunk k runs on CTA k mod P_ret in wave k / P_ret, start to finish. A group
+        // never has two chunks on one CTA, and a wait only depends on chunks of the same or
+        // the next wave held by other CTAs, which finish their current chunk first.
+        for (int k = blockIdx.x; ok && k < NC; k += P_ret) {
+          const int g = group_of(k);
+          phase_score(k);
+          trace(kEvScore);
+          ok = wait_for(P.bar + (int64_t)g * 4 + 0, (uint32_t)nch(g));
+          trace(kEvWait1);
+          if (!ok) break;
+          phase_hist(k);
+          trace(kEvHist);
+          ok = wait_for(P.bar + (int64_t)g * 4 + 1, (uint32_t)nch(g));
+          trace(kEvWait2);
+          if (!ok) break;
+          phase_select(k);
+          trace(kEvSelect);
+          ok = wait_for(P.bar + (int64_t)g * 4 + 2, (uint32_t)nch(g));
+          trace(kEvWait3);
+          if (!ok) break;
+          phase_attend(k);
+          trace(kEvAttend);
+        }
+      } else {
+        // scores in the workspace: phase-major over this CTA's chunks, so no wait ever
+        // depends on a later phase
+        for (int k = blockIdx.x; k < NC; k += P_ret) phase_score(k);
+        for (int k = blockIdx.x; ok && k < NC; k += P_ret) {
+          const int g = group_of(k);
+          ok = wait_for(P.bar + (int64_t)g * 4 + 0, (uint32_t)nch(g));
+          if (ok) phase_hist(k);
+        }
+        for (int k = blockIdx.x; ok && k < NC; k += P_ret) {
+          const int g = group_of(k);
+          ok = wait_for(P.bar + (int64_t)g * 4 + 1, (uint32_t)nch(g));
+          if (ok) phase_select(k);
+        }
+        for (int k = blockIdx.x; ok && k < NC; k += P_ret) {
+          const int g = group_of(k);
+          ok = wait_for(P.bar + (int64_t)g * 4 + 2, (uint32_t)nch(g));
+          if (ok) phase_attend(k);
+        }
+      }
     }
     if (!ok) return;
     local_items();

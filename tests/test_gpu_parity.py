@@ -67,7 +67,7 @@ def test_append_matches_oracle_rows():
     assert (got1 != k_ref1).mean() < 1e-5
 
 
-@pytest.mark.parametrize("p", [0.9, 0.5, 0.99, 1.0])
+@pytest.mark.parametrize("p", [0.9, 0.5, 0.99, 0.999, 0.999995, 1.0])
 def test_tiny_layer_parity(p):
     rep = _parity().run_layer_parity(workload_index=1, layer=0, p=p)
     assert rep["max_abs"] <= 1e-2
