@@ -137,6 +137,33 @@ int rtp_decode_step(const rtp_layer_desc* desc, const rtp_cache* cache, const ui
                     int32_t* sel_counts, int32_t* sel_idx, int64_t sel_stride, void* ws,
                     size_t ws_bytes, rtp_stream_t stream);
 
+/* Size of the library-owned scratch of rtp_decode_step_static (bytes). */
+#define RTP_STATIC_SCRATCH_BYTES (16u << 20)
+
+/*
+ * rtp_decode_step without a caller-provided workspace, for callers that cannot allocate
+ * device memory: an engine whose memory planner has already handed out the whole device
+ * pool, code running inside a CUDA-graph replay or a callback where cudaMalloc is not
+ * allowed, or a host that links the library without a device allocator of its own. The
+ * paper has no counterpart; this is a convenience of the C ABI only.
+ *   Same arguments and results as rtp_decode_step, minus sel_idx and the workspace.
+ *   Scratch: a fixed RTP_STATIC_SCRATCH_BYTES (16 MiB) buffer inside the library, one per
+ *   device, held until the process exits. A description whose rtp_workspace_bytes() exceeds
+ *   it returns RTP_EWORKSPACE and launches nothing.
+ *   Allocates nothing: no cudaMalloc, cudaFree or allocating library call.
+ *   The first call on a device looks up the buffer's device address (cudaGetSymbolAddress)
+ *   and clears its status word with synchronous runtime calls: make that first call before
+ *   any stream capture on that device.
+ *   All calls on a device share the buffer and it keeps the last call's contents; the call
+ *   clears the parts that must start at zero. Calls whose work overlaps on the GPU (different
+ *   streams, or host threads without ordering) race on it: order them on one stream.
+ *   Device-side status (RTP_EDEVICE) is not reported; an invalid sequence still yields zero
+ *   outputs and counts.
+ */
+int rtp_decode_step_static(const rtp_layer_desc* desc, const rtp_cache* cache,
+                           const uint16_t* q_pre, const float* w_qidx, const int32_t* seq_lens,
+                           double p, uint16_t* out, int32_t* sel_counts, rtp_stream_t stream);
+
 /* Synchronises `stream`, returns the workspace's sticky device status (RTP_OK, RTP_EDEVICE or
  * RTP_ETIMEOUT) and clears it. Host-blocking; not for the hot loop. */
 int rtp_read_device_status(void* ws, rtp_stream_t stream);

@@ -5,6 +5,7 @@
 #include <algorithm>
 #include <cmath>
 #include <cstring>
+#include <mutex>
 
 #include "../../include/rtp.h"
 #include "rtp_decode.cuh"
@@ -331,6 +332,49 @@ int rtp_decode_step(const rtp_layer_desc* desc, const rtp_cache* cache, const ui
     default: r = launch_decode<8>(P, pl, di, st, sel_idx, sel_stride); break;
   }
   return r;
+}
+
+// Scratch of rtp_decode_step_static: one fixed buffer per device that loads the library,
+// held until the process exits. Host code only ever uses its device address, obtained with
+// cudaGetSymbolAddress on each device (the symbol itself is a host-side stand-in).
+static __device__ __align__(256) unsigned char g_static_scratch[RTP_STATIC_SCRATCH_BYTES];
+
+namespace {
+std::mutex g_static_mu;
+void* g_static_ptr[64] = {nullptr};
+
+// Device address of g_static_scratch on the current device; the first call on a device looks
+// it up and clears the status word (not capturable: it uses synchronous runtime calls).
+int static_scratch(void** ptr) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return RTP_ECUDA;
+  std::lock_guard<std::mutex> lock(g_static_mu);
+  if (!g_static_ptr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_static_scratch) != cudaSuccess || !p) return RTP_ECUDA;
+    if (cudaMemset(p, 0, 256) != cudaSuccess) return RTP_ECUDA;
+    g_static_ptr[dev] = p;
+  }
+  *ptr = g_static_ptr[dev];
+  return RTP_OK;
+}
+}  // namespace
+
+int rtp_decode_step_static(const rtp_layer_desc* desc, const rtp_cache* cache,
+                           const uint16_t* q_pre, const float* w_qidx, const int32_t* seq_lens,
+                           double p, uint16_t* out, int32_t* sel_counts, rtp_stream_t stream) {
+  g_launches = 0;
+  const size_t need = rtp_workspace_bytes(desc);
+  if (need == 0) {
+    Plan pl;
+    return make_plan(desc, pl);              // the description's own error code
+  }
+  if (need > (size_t)RTP_STATIC_SCRATCH_BYTES) return RTP_EWORKSPACE;
+  void* ws = nullptr;
+  const int rc = static_scratch(&ws);
+  if (rc != RTP_OK) return rc;
+  return rtp_decode_step(desc, cache, q_pre, w_qidx, seq_lens, p, out, sel_counts, nullptr, 0,
+                         ws, (size_t)RTP_STATIC_SCRATCH_BYTES, stream);
 }
 
 int rtp_read_device_status(void* ws, rtp_stream_t stream) {

@@ -105,6 +105,15 @@ def rtp_decode_step(desc: LayerDesc, cache: RtpCache, q_pre, w_qidx, seq_lens, p
         _stream(stream)))
 
 
+def rtp_decode_step_static(desc: LayerDesc, cache: RtpCache, q_pre, w_qidx, seq_lens, p, out,
+                           sel_counts, stream=None):
+    """rtp_decode_step on the library's own fixed scratch (no workspace argument): for callers
+    that cannot allocate device memory. See include/rtp.h for its limits and sharing rules."""
+    return _check("rtp_decode_step_static", _lib.load().rtp_decode_step_static(
+        desc.ref, ctypes.byref(cache), _ptr(q_pre), _ptr(w_qidx), _ptr(seq_lens), float(p),
+        _ptr(out), _ptr(sel_counts), _stream(stream)))
+
+
 def rtp_read_device_status(ws, stream=None) -> int:
     return int(_lib.load().rtp_read_device_status(_ptr(ws), _stream(stream)))
 
