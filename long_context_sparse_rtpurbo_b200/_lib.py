@@ -5,7 +5,8 @@ import ctypes
 import os
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "librtp.so")
+# RTP_LIBRARY_PATH selects another build of the same library (for example a tracing build)
+LIB_PATH = os.environ.get("RTP_LIBRARY_PATH") or os.path.join(_HERE, "librtp.so")
 
 RTP_OK, RTP_EINVAL, RTP_ESHAPE, RTP_EWORKSPACE, RTP_ECUDA, RTP_ETIMEOUT, RTP_EDEVICE = \
     0, -1, -2, -3, -4, -5, -6

@@ -238,9 +238,11 @@ __device__ __forceinline__ void attend_merge(AttnState<G>& st, float* scratch, f
   for (int o = t; o < G * kD; o += nthreads) {
     const int h = o / kD, dch = o % kD;
     float M = -INFINITY;
+#pragma unroll 1
     for (int w = 0; w < nw; ++w) M = fmaxf(M, sm_m[w * G + h]);
     float Ls = 0.f, A = 0.f;
     if (M != -INFINITY) {
+#pragma unroll 1
       for (int w = 0; w < nw; ++w) {
         const float f = exp2f(sm_m[w * G + h] - M);
         Ls += sm_l[w * G + h] * f;
@@ -253,64 +255,71 @@ __device__ __forceinline__ void attend_merge(AttnState<G>& st, float* scratch, f
   __syncthreads();
 }
 
-// Merges n <= kMaxMerge partial states (stride G*(2+128) floats, global memory written by
-// other CTAs) into `dst` (same format) or, when out_rows is given, into the bf16 output rows
-// of the G heads. Every load is issued before the first barrier (one round trip for G <= 4).
-// scratch: >= 2 * kMaxMerge * G + 2 * G floats of shared memory.
+// Largest number of partial states one merge combines (the host plan sizes splits by it).
 constexpr int kMaxMerge = 64;
+
+// Merges n partial states (contiguous in global memory, stride G*(2+128) floats, written by
+// other CTAs) into `dst` (same format) or, when out_rows is given, into the bf16 output rows
+// of the G heads. The partials are first copied into shared memory (buf, buf_bytes) with
+// cp.async, as many per batch as fit, so all loads of a batch are in flight together; each
+// thread then folds its output channels over the batch with the online softmax rule. The
+// code is kept small on purpose: it runs once per group at the end of a step, when the
+// instruction cache does not hold it.
 template <int G>
 __device__ __forceinline__ void merge_partials(const float* parts, int n, float* dst,
-                                               uint16_t* out_rows, float* scratch, int nthreads) {
-  float* fM = scratch;                 // [n][G]: max, then the weight 2^(M_i - M)
-  float* fL = scratch + kMaxMerge * G; // [n][G]
-  float* tot = fL + kMaxMerge * G;     // [G]: M, then [G + h]: L
+                                               uint16_t* out_rows, float* buf, int buf_bytes,
+                                               int nthreads) {
+  constexpr int S = G * (kD + 2);                    // floats per partial
+  constexpr int kPer = (G * kD + 511) / 512;         // outputs per thread for 512 threads
+  const int per = max(1, buf_bytes / (S * 4));       // partials per batch
   const int t = threadIdx.x;
-  for (int o = t; o < n * G; o += nthreads) {
-    const int i = o / G, h = o % G;
-    const float* pp = parts + ((int64_t)i * G + h) * (kD + 2);
-    fM[o] = __ldcg(pp);
-    fL[o] = __ldcg(pp + 1);
-  }
-  constexpr int kBatch = 32;            // partials whose values one thread holds in registers
+  float M[kPer], Ls[kPer], A[kPer];
+#pragma unroll
+  for (int u = 0; u < kPer; ++u) { M[u] = -INFINITY; Ls[u] = 0.f; A[u] = 0.f; }
 #pragma unroll 1
-  for (int ob = 0; ob < G * kD; ob += nthreads) {
-    const int o = ob + t;
-    const int h = o / kD, dch = o % kD;
-    float a[kBatch];
-#pragma unroll
-    for (int i = 0; i < kBatch; ++i)
-      a[i] = (i < n && o < G * kD) ? __ldcg(parts + ((int64_t)i * G + h) * (kD + 2) + 2 + dch) : 0.f;
-    __syncthreads();
-    if (ob == 0 && t < G) {
-      float M = -INFINITY;
-      for (int i = 0; i < n; ++i) M = fmaxf(M, fM[i * G + t]);
-      float Ls = 0.f;
-      for (int i = 0; i < n; ++i) {
-        const float f = (M == -INFINITY || fM[i * G + t] == -INFINITY) ? 0.f : exp2f(fM[i * G + t] - M);
-        fM[i * G + t] = f;
-        Ls += fL[i * G + t] * f;
-      }
-      tot[t] = M;
-      tot[G + t] = Ls;
+  for (int b0 = 0; b0 < n; b0 += per) {
+    const int nb = min(per, n - b0);
+    __syncthreads();                                 // the buffer is free
+    const float* src = parts + (int64_t)b0 * S;
+    if constexpr (S % 4 == 0) {                      // 16-byte partials (G >= 2): cp.async
+      for (int i = t; i < nb * (S / 4); i += nthreads) cp_async16(buf + 4 * i, src + 4 * i);
+      cp_async_commit();
+      cp_async_wait<0>();
+    } else {                                         // G = 1: 520-byte partials, plain loads
+      for (int i = t; i < nb * S; i += nthreads) buf[i] = __ldcg(src + i);
     }
     __syncthreads();
-    if (o < G * kD) {
-      float A = 0.f;
 #pragma unroll
-      for (int i = 0; i < kBatch; ++i)
-        if (i < n) A = fmaf(a[i], fM[i * G + h], A);
-      for (int i = kBatch; i < n; ++i)
-        A = fmaf(__ldcg(parts + ((int64_t)i * G + h) * (kD + 2) + 2 + dch), fM[i * G + h], A);
-      const float Ls = tot[G + h];
-      if (out_rows) {
-        out_rows[(int64_t)h * kD + dch] = f2bf_rn(Ls > 0.f ? A / Ls : 0.f);
-      } else {
-        dst[h * (kD + 2) + 2 + dch] = A;
-        if (dch == 0) { dst[h * (kD + 2)] = tot[h]; dst[h * (kD + 2) + 1] = Ls; }
+    for (int u = 0; u < kPer; ++u) {
+      const int o = t + u * nthreads;
+      if (o >= G * kD) break;
+      const int h = o / kD, dch = o % kD;
+#pragma unroll 1
+      for (int i = 0; i < nb; ++i) {
+        const float* pp = buf + i * S + h * (kD + 2);
+        const float mi = pp[0];
+        if (mi == -INFINITY) continue;               // a split without rows
+        const float mn = fmaxf(M[u], mi);
+        const float fo = exp2f(M[u] - mn), fi = exp2f(mi - mn);   // exp2(-inf) = 0
+        A[u] = A[u] * fo + pp[2 + dch] * fi;
+        Ls[u] = Ls[u] * fo + pp[1] * fi;
+        M[u] = mn;
       }
     }
   }
-  __syncthreads();
+#pragma unroll
+  for (int u = 0; u < kPer; ++u) {
+    const int o = t + u * nthreads;
+    if (o >= G * kD) break;
+    const int h = o / kD, dch = o % kD;
+    if (out_rows) {
+      out_rows[(int64_t)h * kD + dch] = f2bf_rn(Ls[u] > 0.f ? A[u] / Ls[u] : 0.f);
+    } else {
+      dst[h * (kD + 2) + 2 + dch] = A[u];
+      if (dch == 0) { dst[h * (kD + 2)] = M[u]; dst[h * (kD + 2) + 1] = Ls[u]; }
+    }
+  }
+  __syncthreads();                                   // the caller may reuse the buffer
 }
 
 }  // namespace rtp

@@ -326,6 +326,7 @@ struct DecodeCta {
   // ------------------------------------------------------------ plan (every CTA identical)
   __device__ void plan() {
     const int t = threadIdx.x;
+    if (t == 0) sm.ints[34] = -1;           // no group total in sm.tmp yet
     for (int b = t; b < P.L.B; b += kFThreads) sm.N[b] = seq_len_checked(P, b);
     __syncthreads();
     int sumN = 0, sumL = 0, maxN = 0;
@@ -408,7 +409,6 @@ struct DecodeCta {
     __syncthreads();                       // the stage buffer may still be read by a merge
 #pragma unroll
     for (int st = 0; st < kSStages - 1; ++st) issue(st);
-    rope_query<G>(P, b, kvh, N, sm.qret);   // for phase W; overlaps the first loads
     index_query<G>(P, b, kvh, sm.qidx, sm.tmp);
     trace(kEvS0);
     float qi[G][kR];
@@ -452,6 +452,7 @@ struct DecodeCta {
     trace(kEvS1);
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     float* red = sm.tmp;                    // [2][G][16], then [G][16]
+    if (threadIdx.x == 0) sm.ints[34] = -1; // sm.tmp no longer holds a group total
     __syncthreads();
 #pragma unroll
     for (int h = 0; h < G; ++h) {
@@ -500,12 +501,16 @@ struct DecodeCta {
       P.cstat[((int64_t)g * P.max_nch + j) * G + h] = make_float2(cmax[h], (float)l);
     }
     arrive(P.bar + (int64_t)g * 4 + 0);
+    // the RoPE'd query of phase W (scores-in-shared-memory schedule), formed off the critical
+    // path: after this chunk has arrived, while the other chunks of the group finish
+    if (smem_mode) rope_query<G>(P, b, kvh, N, sm.qret);
   }
 
   // Total mass T_h = sum over the group's chunks of L_c exp(hi_c - hi), for the G heads,
   // from the chunk statistics of phase S (double, fixed order: every CTA gets the same value)
   // -> sm.tot[h] (as a double in units of the head's max-score token).
   __device__ void group_total(int g, const float* hi, double* tot) {
+    if (sm.ints[34] == g) return;          // still in sm.tmp from this group's phase H
     const int n = nch(g);
     double* part = reinterpret_cast<double*>(sm.stage);      // [kFThreads]
     const int t = threadIdx.x;
@@ -523,6 +528,7 @@ struct DecodeCta {
       for (int i = t; i < kFThreads; i += G) v += part[i];
       tot[t] = v;
     }
+    if (t == 0) sm.ints[34] = g;
     __syncthreads();
   }
 
@@ -705,6 +711,7 @@ struct DecodeCta {
     if (lane == 0) {
 #pragma unroll
       for (int h = 0; h < G; ++h) reinterpret_cast<int*>(sm.tmp)[warp * G + h] = hc[h];
+    if (threadIdx.x == 0) sm.ints[34] = -1; // sm.tmp no longer holds a group total
     }
     __syncthreads();
     if (threadIdx.x < G) {
@@ -755,7 +762,8 @@ struct DecodeCta {
   }
 
   __device__ __noinline__ void merge(const float* parts, int n, float* dst, uint16_t* out_rows) {
-    merge_partials<G>(parts, n, dst, out_rows, reinterpret_cast<float*>(sm.stage), kFThreads);
+    // the score buffer is free whenever partials are merged
+    merge_partials<G>(parts, n, dst, out_rows, sm.scores, 4 * G * P.C_cap, kFThreads);
   }
 
   // ------------------------------------------------------------ phase W

@@ -130,3 +130,13 @@ def test_qwen_layer_32k_parity():
     conc = [e["n_gpu"] for e in rep["heads"] if e["retrieval"] and kind(e["h"]) == "conc"]
     diff = [e["n_gpu"] for e in rep["heads"] if e["retrieval"] and kind(e["h"]) == "diff"]
     assert conc and diff and np.mean(diff) > 2.5 * np.mean(conc)
+
+
+def test_scores_in_workspace_schedule():
+    """Two retrieval groups of 600K tokens with G = 8: their chunks at the shared-memory score
+    capacity (at most 227 KB / 32 B = 7.1K tokens per CTA) need more than one wave of 148 CTAs,
+    so the scores go to the workspace and the phases run phase-major over each CTA's chunks."""
+    w = _small(G=8, Hkv=2, seq=(600_000,), window=2048, ret=(True, True))
+    heads = [(0, 0), (0, 5), (0, 8), (0, 15)]
+    rep = _parity().run_layer_parity(w=w, layer=0, source="gpu", heads=heads)
+    assert all(e["retrieval"] and e["count"] > 0 for e in rep["heads"])
