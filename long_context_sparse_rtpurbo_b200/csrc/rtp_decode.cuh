@@ -535,9 +535,9 @@ struct DecodeCta {
   // ------------------------------------------------------------ phase H
   // Masses are exp(s - max) in 2^-40 fixed point. Only bins at or above a cutoff bin get
   // per-bin sums: with T the group's total mass (from phase S), every token below bin(c),
-  // c = hi + ln((1 - p) T' / N) - 2 and T' = T (1 - 1e-3), has mass below (1 - p) T' e^-2 / N,
-  // so together they hold less than (1 - p) of the total and b* can not fall under the
-  // cutoff bin. The per-bin sums use two 32-bit shared atomics per token: the low-word add
+  // c = hi + ln((1 - p) T' / N) and T' = T (1 - 1e-3), has mass below (1 - p) T' / N, so
+  // together they hold less than (1 - p) of the total, C_bin(c) > p T and b* can not fall
+  // under the cutoff bin (the 1e-3 absorbs the rounding of T, the log and the bin edges). The per-bin sums use two 32-bit shared atomics per token: the low-word add
   // returns the old value and its carry goes to the high word (exact). Lanes take interleaved
   // (token, head) elements and the heads' rows are padded, so a warp's atomics spread over
   // the banks.
@@ -561,7 +561,7 @@ struct DecodeCta {
     int bch = 0;
     if (P.p < 1.0 && invh > 0.f) {
       const float arg = (float)((1.0 - P.p) * tot[h] * (1.0 - 1e-3) / (double)N);
-      const float c = hih + logf(arg) - 2.f;
+      const float c = hih + logf(arg);
       bch = c > loh ? bin_of(c, loh, invh) : 0;
     }
     const float* sc = score_ptr(g, j);
@@ -636,7 +636,8 @@ struct DecodeCta {
   // ------------------------------------------------------------ phase T
   // Tiles of kFThreads * kTRun tokens; in a tile each thread owns a run of consecutive
   // tokens: masks in registers, one block-wide scan of the per-thread counts, then each
-  // thread writes its run's entries.
+  // thread writes its run's entries. The run length is odd, so the 32 lanes of a warp, which
+  // read scores one run apart, hit 32 different banks.
   static constexpr int kTRun = 32;
   __device__ void phase_select(int k) {
     const int g = group_of(k), j = k - sm.cbase[g];
@@ -661,7 +662,7 @@ struct DecodeCta {
 #pragma unroll 1
     for (int tb = 0; tb < n1 - n0; tb += kFThreads * kTRun) {
       const int len = min(kFThreads * kTRun, n1 - n0 - tb);
-      const int per = (len + kFThreads - 1) / kFThreads;
+      const int per = ((len + kFThreads - 1) / kFThreads) | 1;
       const int t0 = threadIdx.x * per, t1 = min(len, t0 + per);
       int cnt = 0;
 #pragma unroll 1
