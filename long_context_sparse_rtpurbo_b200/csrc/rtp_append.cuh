@@ -35,6 +35,16 @@ __device__ __forceinline__ void rope_sincos(double pos, double theta, double* s,
   sincos(r, s, c);
 }
 
+// The same angle reduction in double, then single-precision sin and cos of the reduced angle
+// (|r| <= pi): for the query rotation, which is used in single precision anyway.
+__device__ __forceinline__ void rope_sincosf(double pos, double theta, float* s, float* c) {
+  const double x = pos * theta;
+  const double k = rint(x * 0.15915494309189535);
+  double r = fma(-k, 6.283185307179586, x);
+  r = fma(-k, 2.4492935982947064e-16, r);
+  sincosf((float)r, s, c);
+}
+
 // One CTA of 128 threads appends kAppendTok consecutive tokens of one (sequence, KV head).
 constexpr int kAppendTok = 4;
 

@@ -58,24 +58,35 @@ __device__ __forceinline__ void halving_reduce(float (&v)[N], int hl) {
   }
 }
 
-// Softmax state of one half-warp.
+// Softmax state of one half-warp; the accumulator holds channel pairs (2e, 2e + 1), so the
+// V update is one packed f32x2 multiply-add per pair.
 template <int G> struct AttnState {
-  float m[G], l[G], acc[G][8];
+  float m[G], l[G];
+  float2 a2[G][4];
+  __device__ __forceinline__ float& acc(int h, int e) { return (&a2[h][e >> 1].x)[e & 1]; }
   __device__ __forceinline__ void init() {
 #pragma unroll
     for (int h = 0; h < G; ++h) {
       m[h] = -INFINITY;
       l[h] = 0.f;
 #pragma unroll
-      for (int e = 0; e < 8; ++e) acc[h][e] = 0.f;
+      for (int e = 0; e < 4; ++e) a2[h][e] = make_float2(0.f, 0.f);
     }
   }
 };
 
+// 8 bf16 -> 4 packed channel pairs
+__device__ __forceinline__ void unpack_pairs(const uint4& w, float2 (&f)[4]) {
+  f[0] = make_float2(bf_lo(w.x), bf_hi(w.x));
+  f[1] = make_float2(bf_lo(w.y), bf_hi(w.y));
+  f[2] = make_float2(bf_lo(w.z), bf_hi(w.z));
+  f[3] = make_float2(bf_lo(w.w), bf_hi(w.w));
+}
+
 // One step of kRows staged rows for a half-warp; kw/vw: this lane's 16 bytes of each row
 // (zero for rows no head attends), mask: heads that attend each row.
 template <int G>
-__device__ __forceinline__ void attend_step(AttnState<G>& st, const float (&q)[G][8],
+__device__ __forceinline__ void attend_step(AttnState<G>& st, const float2 (&q)[G][4],
                                             const uint4 (&kw)[AttnCfg<G>::kRows],
                                             const uint4 (&vw)[AttnCfg<G>::kRows],
                                             const uint32_t (&mask)[AttnCfg<G>::kRows], int hl) {
@@ -84,14 +95,14 @@ __device__ __forceinline__ void attend_step(AttnState<G>& st, const float (&q)[G
   float d[V];
 #pragma unroll
   for (int r = 0; r < R; ++r) {
-    float k[8];
-    unpack8(kw[r], k);
+    float2 k[4];
+    unpack_pairs(kw[r], k);
 #pragma unroll
     for (int h = 0; h < G; ++h) {
-      float a = 0.f;
+      float2 a = __fmul2_rn(q[h][0], k[0]);
 #pragma unroll
-      for (int e = 0; e < 8; ++e) a = fmaf(q[h][e], k[e], a);
-      d[r * G + h] = a;
+      for (int e = 1; e < 4; ++e) a = __ffma2_rn(q[h][e], k[e], a);
+      d[r * G + h] = a.x + a.y;
     }
   }
   halving_reduce<V>(d, hl);
@@ -123,20 +134,22 @@ __device__ __forceinline__ void attend_step(AttnState<G>& st, const float (&q)[G
       const float scale = exp2f(st.m[h] - bmh);  // 0 when the state was empty (m = -inf)
       st.m[h] = bmh;
       st.l[h] *= scale;
+      const float2 sc2 = make_float2(scale, scale);
 #pragma unroll
-      for (int e = 0; e < 8; ++e) st.acc[h][e] *= scale;
+      for (int e = 0; e < 4; ++e) st.a2[h][e] = __fmul2_rn(st.a2[h][e], sc2);
     }
   }
 #pragma unroll
   for (int r = 0; r < R; ++r) {
-    float v[8];
-    unpack8(vw[r], v);
+    float2 v[4];
+    unpack_pairs(vw[r], v);
 #pragma unroll
     for (int h = 0; h < G; ++h) {
       const float p = __shfl_sync(0xffffffffu, p_my, base + ((r * G + h) << kShift));
       st.l[h] += p;
+      const float2 p2 = make_float2(p, p);
 #pragma unroll
-      for (int e = 0; e < 8; ++e) st.acc[h][e] = fmaf(p, v[e], st.acc[h][e]);
+      for (int e = 0; e < 4; ++e) st.a2[h][e] = __ffma2_rn(p2, v[e], st.a2[h][e]);
     }
   }
 }
@@ -145,7 +158,7 @@ __device__ __forceinline__ void attend_step(AttnState<G>& st, const float (&q)[G
 // stage: AttnCfg<G>::stage_bytes(nthreads) bytes of shared memory. Leaves the half-warp
 // states in st (merge with attend_merge).
 template <int G, class RowFn>
-__device__ __forceinline__ void attend_rows(AttnState<G>& st, const float (&q)[G][8], int cnt,
+__device__ __forceinline__ void attend_rows(AttnState<G>& st, const float2 (&q)[G][4], int cnt,
                                             RowFn rowfn, unsigned char* stage, int nthreads) {
   constexpr int R = AttnCfg<G>::kRows;
   const int t = threadIdx.x, lane = t & 31, warp = t >> 5, hl = lane & 15, hw = t >> 4;
@@ -215,8 +228,8 @@ __device__ __forceinline__ void attend_merge(AttnState<G>& st, float* scratch, f
     st.l[h] = st.l[h] * fa + lo * fb;
 #pragma unroll
     for (int e = 0; e < 8; ++e) {
-      const float ao = __shfl_xor_sync(0xffffffffu, st.acc[h][e], 16);
-      st.acc[h][e] = st.acc[h][e] * fa + ao * fb;
+      const float ao = __shfl_xor_sync(0xffffffffu, st.acc(h, e), 16);
+      st.acc(h, e) = st.acc(h, e) * fa + ao * fb;
     }
     st.m[h] = mn;
   }
@@ -227,7 +240,7 @@ __device__ __forceinline__ void attend_merge(AttnState<G>& st, float* scratch, f
 #pragma unroll
     for (int h = 0; h < G; ++h)
 #pragma unroll
-      for (int e = 0; e < 8; ++e) scratch[(warp * G + h) * kD + hl * 8 + e] = st.acc[h][e];
+      for (int e = 0; e < 8; ++e) scratch[(warp * G + h) * kD + hl * 8 + e] = st.acc(h, e);
     if (hl == 0) {
 #pragma unroll
       for (int h = 0; h < G; ++h) { sm_m[warp * G + h] = st.m[h]; sm_l[warp * G + h] = st.l[h]; }

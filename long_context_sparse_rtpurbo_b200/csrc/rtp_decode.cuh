@@ -178,16 +178,26 @@ __device__ __forceinline__ int upper_index(const int* a, int n, int key) {
 }
 
 // stage: index-row staging (phase S), K/V row staging and merge scratch (attention).
+// Dynamic shared memory of the decode kernel; its regions sit at the offsets in DecodeParams.
+extern __shared__ __align__(16) unsigned char rtp_smem[];
+
+// Region pointers, formed on each use from the kernel parameters (constant bank) rather than
+// held in registers across the phases.
 template <int G> struct Smem {
-  float* scores; unsigned char* stage; float* res; float* qret; float* qloc; float* qidx;
-  float* tmp; unsigned long long* hist; int* N; int* cbase; int* pref; int* ints;
-  __device__ Smem(unsigned char* base, const DecodeParams& P)
-      : scores((float*)(base + P.sm_scores)), stage(base + P.sm_stage),
-        res((float*)(base + P.sm_res)), qret((float*)(base + P.sm_qret)),
-        qloc((float*)(base + P.sm_qloc)), qidx((float*)(base + P.sm_qidx)),
-        tmp((float*)(base + P.sm_tmp)), hist((unsigned long long*)(base + P.sm_hist)),
-        N((int*)(base + P.sm_N)), cbase((int*)(base + P.sm_cbase)), pref((int*)(base + P.sm_pref)),
-        ints((int*)(base + P.sm_int)) {}
+  const DecodeParams& P;
+  __device__ explicit Smem(const DecodeParams& p) : P(p) {}
+  __device__ float* scores() const { return (float*)(rtp_smem + P.sm_scores); }
+  __device__ unsigned char* stage() const { return rtp_smem + P.sm_stage; }
+  __device__ float* res() const { return (float*)(rtp_smem + P.sm_res); }
+  __device__ float* qret() const { return (float*)(rtp_smem + P.sm_qret); }
+  __device__ float* qloc() const { return (float*)(rtp_smem + P.sm_qloc); }
+  __device__ float* qidx() const { return (float*)(rtp_smem + P.sm_qidx); }
+  __device__ float* tmp() const { return (float*)(rtp_smem + P.sm_tmp); }
+  __device__ unsigned long long* hist() const { return (unsigned long long*)(rtp_smem + P.sm_hist); }
+  __device__ int* N() const { return (int*)(rtp_smem + P.sm_N); }
+  __device__ int* cbase() const { return (int*)(rtp_smem + P.sm_cbase); }
+  __device__ int* pref() const { return (int*)(rtp_smem + P.sm_pref); }
+  __device__ int* ints() const { return (int*)(rtp_smem + P.sm_int); }
 };
 // ints[]: [0..31] reduction scratch, [32] wait flag, [33] next local item, [40..47] b*,
 //         [48..50] last-arrival flags
@@ -199,15 +209,15 @@ __device__ __noinline__ void rope_query(const DecodeParams& P, int b, int kvh, i
   const int t = threadIdx.x;
   if (t < kD) {
     const int i = t & 63;
-    double sn, cs;
-    rope_sincos((double)(N - 1), P.L.theta[i], &sn, &cs);
+    float sn, cs;
+    rope_sincosf((double)(N - 1), P.L.theta[i], &sn, &cs);
     const float scale = kLog2e * 0.08838834764831845f;   // log2(e) / sqrt(128)
 #pragma unroll
     for (int h = 0; h < G; ++h) {
       const uint16_t* q = P.q_pre + ((int64_t)b * P.L.Hq + kvh * G + h) * kD;
-      const double qa = bf1(q[i]), qb = bf1(q[i + 64]);
-      const double r = (t < 64) ? (qa * cs - qb * sn) : (qa * sn + qb * cs);
-      q_s[h * kD + t] = (float)r * scale;
+      const float qa = bf1(q[i]), qb = bf1(q[i + 64]);
+      const float r = (t < 64) ? (qa * cs - qb * sn) : (qa * sn + qb * cs);
+      q_s[h * kD + t] = r * scale;
     }
   }
 }
@@ -260,14 +270,14 @@ struct DecodeCta {
   Smem<G> sm;
   int C, NC, smem_mode, P_ret;
 
-  __device__ DecodeCta(const DecodeParams& p, unsigned char* base) : P(p), sm(base, p) {}
+  __device__ explicit DecodeCta(const DecodeParams& p) : P(p), sm(p) {}
 
-  __device__ __forceinline__ int group_of(int k) const { return upper_index(sm.cbase, P.n_groups, k); }
-  __device__ __forceinline__ int nch(int g) const { return sm.cbase[g + 1] - sm.cbase[g]; }
-  __device__ __forceinline__ int gN(int g) const { return sm.N[g / P.L.n_ret]; }
+  __device__ __forceinline__ int group_of(int k) const { return upper_index(sm.cbase(), P.n_groups, k); }
+  __device__ __forceinline__ int nch(int g) const { return sm.cbase()[g + 1] - sm.cbase()[g]; }
+  __device__ __forceinline__ int gN(int g) const { return sm.N()[g / P.L.n_ret]; }
 
   __device__ __forceinline__ float* score_ptr(int g, int j) const {
-    return smem_mode ? sm.scores : P.scores + (int64_t)g * G * P.maxN_pad + (int64_t)j * C;
+    return smem_mode ? sm.scores() : P.scores + (int64_t)g * G * P.maxN_pad + (int64_t)j * C;
   }
   __device__ __forceinline__ int64_t score_hstride() const {
     return smem_mode ? (int64_t)P.C_cap + kHeadPad : P.maxN_pad;
@@ -312,10 +322,10 @@ struct DecodeCta {
           f = 2;
         }
         if (f == 1) __threadfence();
-        sm.ints[32] = f;
+        sm.ints()[32] = f;
       }
       __syncthreads();
-      const int f = sm.ints[32];
+      const int f = sm.ints()[32];
       __syncthreads();
       if (f == 1) return true;
       if (f == 2) return false;
@@ -326,18 +336,18 @@ struct DecodeCta {
   // ------------------------------------------------------------ plan (every CTA identical)
   __device__ void plan() {
     const int t = threadIdx.x;
-    if (t == 0) sm.ints[34] = -1;           // no group total in sm.tmp yet
-    for (int b = t; b < P.L.B; b += kFThreads) sm.N[b] = seq_len_checked(P, b);
+    if (t == 0) sm.ints()[34] = -1;           // no group total in sm.tmp() yet
+    for (int b = t; b < P.L.B; b += kFThreads) sm.N()[b] = seq_len_checked(P, b);
     __syncthreads();
     int sumN = 0, sumL = 0, maxN = 0;
     for (int b = t; b < P.L.B; b += kFThreads) {
-      sumN += sm.N[b];
-      sumL += min(sm.N[b], P.L.ring);
-      maxN = max(maxN, sm.N[b]);
+      sumN += sm.N()[b];
+      sumL += min(sm.N()[b], P.L.ring);
+      maxN = max(maxN, sm.N()[b]);
     }
-    const long long Tr = (long long)block_sum_int(sumN, sm.ints) * P.L.n_ret;
-    const long long loc_rows = (long long)block_sum_int(sumL, sm.ints) * P.L.n_loc;
-    maxN = block_max_int(maxN, sm.ints);
+    const long long Tr = (long long)block_sum_int(sumN, sm.ints()) * P.L.n_ret;
+    const long long loc_rows = (long long)block_sum_int(sumL, sm.ints()) * P.L.n_loc;
+    maxN = block_max_int(maxN, sm.ints());
     // CTAs [0, P_ret) run the retrieval chain, the others start on local items at once; the
     // split follows the bytes of each side (index read twice as a proxy for index + gather).
     P_ret = 0;
@@ -367,15 +377,15 @@ struct DecodeCta {
       }
       P_ret = pr;
     }
-    for (int g = t; g < P.n_groups; g += kFThreads) sm.cbase[g] = (gN(g) + C - 1) / C;
+    for (int g = t; g < P.n_groups; g += kFThreads) sm.cbase()[g] = (gN(g) + C - 1) / C;
     __syncthreads();
-    NC = block_scan_excl(sm.cbase, P.n_groups, sm.ints);
-    if (t == 0) sm.cbase[P.n_groups] = NC;
+    NC = block_scan_excl(sm.cbase(), P.n_groups, sm.ints());
+    if (t == 0) sm.cbase()[P.n_groups] = NC;
     if (blockIdx.x == 0 && t == 0) P.misc[2] = (uint32_t)C;
     // invalid sequences: zero their outputs once (CTA 0) and record the status
     if (blockIdx.x == 0) {
       for (int b = 0; b < P.L.B; ++b) {
-        if (sm.N[b] != 0) continue;
+        if (sm.N()[b] != 0) continue;
         for (int o = t; o < P.L.Hq * kD; o += kFThreads) P.out[(int64_t)b * P.L.Hq * kD + o] = 0;
         for (int o = t; o < P.L.Hq; o += kFThreads) P.sel_counts[(int64_t)b * P.L.Hq + o] = 0;
         if (t == 0) set_status(P.status, -6);
@@ -390,7 +400,7 @@ struct DecodeCta {
   // first stages are in flight.
   static constexpr int kSRows = 512, kSStages = 4;
   __device__ void phase_score(int k) {
-    const int g = group_of(k), j = k - sm.cbase[g];
+    const int g = group_of(k), j = k - sm.cbase()[g];
     const int b = g / P.L.n_ret, r = g % P.L.n_ret, kvh = P.L.ret_kv[r];
     const int N = gN(g);
     const int n0 = j * C, n1 = min(N, n0 + C);
@@ -399,7 +409,7 @@ struct DecodeCta {
     const int nst = (n1 - n0 + kSRows - 1) / kSRows;
     auto issue = [&](int st) {
       if (st < nst) {
-        unsigned char* dst = sm.stage + (st % kSStages) * (kSRows * 32);
+        unsigned char* dst = sm.stage() + (st % kSStages) * (kSRows * 32);
         const int rows = min(kSRows, n1 - n0 - st * kSRows);
         for (int piece = threadIdx.x; piece < rows * 2; piece += kFThreads)
           cp_async16(dst + piece * 16, src + ((int64_t)st * kSRows * 32) + piece * 16);
@@ -409,13 +419,14 @@ struct DecodeCta {
     __syncthreads();                       // the stage buffer may still be read by a merge
 #pragma unroll
     for (int st = 0; st < kSStages - 1; ++st) issue(st);
-    index_query<G>(P, b, kvh, sm.qidx, sm.tmp);
+    index_query<G>(P, b, kvh, sm.qidx(), sm.tmp());
     trace(kEvS0);
-    float qi[G][kR];
+    float2 qi[G][kR / 2];                    // index query, channel pairs (2j, 2j + 1)
 #pragma unroll
     for (int h = 0; h < G; ++h)
 #pragma unroll
-      for (int jj = 0; jj < kR; ++jj) qi[h][jj] = sm.qidx[h * kR + jj];
+      for (int jj = 0; jj < kR / 2; ++jj)
+        qi[h][jj] = make_float2(sm.qidx()[h * kR + 2 * jj], sm.qidx()[h * kR + 2 * jj + 1]);
     float mn[G], mx[G];
 #pragma unroll
     for (int h = 0; h < G; ++h) { mn[h] = INFINITY; mx[h] = -INFINITY; }
@@ -427,20 +438,22 @@ struct DecodeCta {
       cp_async_wait<kSStages - 1>();
       __syncthreads();
       const int rows = min(kSRows, n1 - n0 - st * kSRows);
-      const unsigned char* buf = sm.stage + (st % kSStages) * (kSRows * 32);
+      const unsigned char* buf = sm.stage() + (st % kSStages) * (kSRows * 32);
 #pragma unroll 1
       for (int i = threadIdx.x; i < rows; i += kFThreads) {
         const uint4 a = *reinterpret_cast<const uint4*>(buf + i * 32);
         const uint4 c2 = *reinterpret_cast<const uint4*>(buf + i * 32 + 16);
-        float x[16];
-        unpack8(a, x);
-        unpack8(c2, x + 8);
+        const uint32_t w[8] = {a.x, a.y, a.z, a.w, c2.x, c2.y, c2.z, c2.w};
+        float2 x[kR / 2];                      // channel pairs: even and odd sums, then added
+#pragma unroll
+        for (int jj = 0; jj < kR / 2; ++jj) x[jj] = make_float2(bf_lo(w[jj]), bf_hi(w[jj]));
         const int nl = st * kSRows + i;
 #pragma unroll
         for (int h = 0; h < G; ++h) {
-          float acc = 0.f;
+          float2 a2 = __fmul2_rn(qi[h][0], x[0]);
 #pragma unroll
-          for (int jj = 0; jj < kR; ++jj) acc = fmaf(qi[h][jj], x[jj], acc);
+          for (int jj = 1; jj < kR / 2; ++jj) a2 = __ffma2_rn(qi[h][jj], x[jj], a2);
+          const float acc = a2.x + a2.y;
           sc[h * hs + nl] = acc;
           mn[h] = fminf(mn[h], acc);
           mx[h] = fmaxf(mx[h], acc);
@@ -451,8 +464,8 @@ struct DecodeCta {
     cp_async_wait<0>();
     trace(kEvS1);
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    float* red = sm.tmp;                    // [2][G][16], then [G][16]
-    if (threadIdx.x == 0) sm.ints[34] = -1; // sm.tmp no longer holds a group total
+    float* red = sm.tmp();                    // [2][G][16], then [G][16]
+    if (threadIdx.x == 0) sm.ints()[34] = -1; // sm.tmp() no longer holds a group total
     __syncthreads();
 #pragma unroll
     for (int h = 0; h < G; ++h) {
@@ -503,16 +516,16 @@ struct DecodeCta {
     arrive(P.bar + (int64_t)g * 4 + 0);
     // the RoPE'd query of phase W (scores-in-shared-memory schedule), formed off the critical
     // path: after this chunk has arrived, while the other chunks of the group finish
-    if (smem_mode) rope_query<G>(P, b, kvh, N, sm.qret);
+    if (smem_mode) rope_query<G>(P, b, kvh, N, sm.qret());
   }
 
   // Total mass T_h = sum over the group's chunks of L_c exp(hi_c - hi), for the G heads,
   // from the chunk statistics of phase S (double, fixed order: every CTA gets the same value)
   // -> sm.tot[h] (as a double in units of the head's max-score token).
   __device__ void group_total(int g, const float* hi, double* tot) {
-    if (sm.ints[34] == g) return;          // still in sm.tmp from this group's phase H
+    if (sm.ints()[34] == g) return;          // still in sm.tmp() from this group's phase H
     const int n = nch(g);
-    double* part = reinterpret_cast<double*>(sm.stage);      // [kFThreads]
+    double* part = reinterpret_cast<double*>(sm.stage());      // [kFThreads]
     const int t = threadIdx.x;
     const int h = t % G;
     double acc = 0.0;
@@ -528,7 +541,7 @@ struct DecodeCta {
       for (int i = t; i < kFThreads; i += G) v += part[i];
       tot[t] = v;
     }
-    if (t == 0) sm.ints[34] = g;
+    if (t == 0) sm.ints()[34] = g;
     __syncthreads();
   }
 
@@ -542,15 +555,15 @@ struct DecodeCta {
   // (token, head) elements and the heads' rows are padded, so a warp's atomics spread over
   // the banks.
   __device__ void phase_hist(int k) {
-    const int g = group_of(k), j = k - sm.cbase[g];
+    const int g = group_of(k), j = k - sm.cbase()[g];
     const int N = gN(g);
     const int n0 = j * C, n1 = min(N, n0 + C);
-    uint32_t* hlo = reinterpret_cast<uint32_t*>(sm.hist);
+    uint32_t* hlo = reinterpret_cast<uint32_t*>(sm.hist());
     uint32_t* hhi = hlo + G * kHistStride;
     for (int i = threadIdx.x; i < 2 * G * kHistStride; i += kFThreads) hlo[i] = 0u;
     float lo[G], hi[G], inv[G];
     load_range<G>(P, g, lo, hi, inv);
-    double* tot = reinterpret_cast<double*>(sm.tmp);          // [G]
+    double* tot = reinterpret_cast<double*>(sm.tmp());          // [G]
     group_total(g, hi, tot);
     trace(kEvH0);
     const int h = threadIdx.x % G;          // G divides kFThreads: the thread's head is fixed
@@ -597,15 +610,15 @@ struct DecodeCta {
     arrive(P.bar + (int64_t)g * 4 + 1);
   }
 
-  // b* of the G heads of group g into sm.ints[40 + h]; warp h handles head h.
+  // b* of the G heads of group g into sm.ints()[40 + h]; warp h handles head h.
   __device__ void find_bstar(int g, const float* hi) {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    double* tot = reinterpret_cast<double*>(sm.tmp);
+    double* tot = reinterpret_cast<double*>(sm.tmp());
     if (!P.select_all) group_total(g, hi, tot);
     if (warp < G) {
       const int h = warp;
       if (P.select_all) {
-        if (lane == 0) sm.ints[40 + h] = 0;
+        if (lane == 0) sm.ints()[40 + h] = 0;
       } else {
         const unsigned long long* gh = P.hist + ((int64_t)g * G + h) * kBins;
         unsigned long long v[8], lt = 0;
@@ -627,7 +640,7 @@ struct DecodeCta {
         }
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) best = max(best, __shfl_xor_sync(0xffffffffu, best, o));
-        if (lane == 0) sm.ints[40 + h] = best < 0 ? 0 : best;
+        if (lane == 0) sm.ints()[40 + h] = best < 0 ? 0 : best;
       }
     }
     __syncthreads();
@@ -640,7 +653,7 @@ struct DecodeCta {
   // read scores one run apart, hit 32 different banks.
   static constexpr int kTRun = 32;
   __device__ void phase_select(int k) {
-    const int g = group_of(k), j = k - sm.cbase[g];
+    const int g = group_of(k), j = k - sm.cbase()[g];
     const int N = gN(g);
     const int n0 = j * C, n1 = min(N, n0 + C);
     float lo[G], hi[G], inv[G];
@@ -649,7 +662,7 @@ struct DecodeCta {
     trace(kEvT0);
     int bs[G];
 #pragma unroll
-    for (int h = 0; h < G; ++h) bs[h] = sm.ints[40 + h];
+    for (int h = 0; h < G; ++h) bs[h] = sm.ints()[40 + h];
     const float* sc = score_ptr(g, j);
     const int64_t hs = score_hstride();
     uint32_t* ent = P.ent + (int64_t)g * P.maxN_pad + n0;
@@ -658,7 +671,7 @@ struct DecodeCta {
 #pragma unroll
     for (int h = 0; h < G; ++h) hc[h] = 0;
     int base = 0;
-    uint8_t* mk = sm.stage;                  // per-token head masks of the current tile
+    uint8_t* mk = sm.stage();                  // per-token head masks of the current tile
 #pragma unroll 1
     for (int tb = 0; tb < n1 - n0; tb += kFThreads * kTRun) {
       const int len = min(kFThreads * kTRun, n1 - n0 - tb);
@@ -683,11 +696,11 @@ struct DecodeCta {
         if (lane >= o) incl += y;
       }
       __syncthreads();
-      if (lane == 31) sm.ints[warp] = incl;
+      if (lane == 31) sm.ints()[warp] = incl;
       __syncthreads();
       int before = 0, total = 0;
       for (int w = 0; w < kFThreads / 32; ++w) {
-        const int x = sm.ints[w];
+        const int x = sm.ints()[w];
         before += (w < warp) ? x : 0;
         total += x;
       }
@@ -711,21 +724,21 @@ struct DecodeCta {
     __syncthreads();
     if (lane == 0) {
 #pragma unroll
-      for (int h = 0; h < G; ++h) reinterpret_cast<int*>(sm.tmp)[warp * G + h] = hc[h];
-    if (threadIdx.x == 0) sm.ints[34] = -1; // sm.tmp no longer holds a group total
+      for (int h = 0; h < G; ++h) reinterpret_cast<int*>(sm.tmp())[warp * G + h] = hc[h];
+    if (threadIdx.x == 0) sm.ints()[34] = -1; // sm.tmp() no longer holds a group total
     }
     __syncthreads();
     if (threadIdx.x < G) {
       int v = 0;
-      for (int w = 0; w < kFThreads / 32; ++w) v += reinterpret_cast<int*>(sm.tmp)[w * G + threadIdx.x];
+      for (int w = 0; w < kFThreads / 32; ++w) v += reinterpret_cast<int*>(sm.tmp())[w * G + threadIdx.x];
       if (v) atomicAdd(P.hcnt + (int64_t)g * G + threadIdx.x, v);
     }
     if (threadIdx.x == 0) P.ccnt[(int64_t)g * P.max_nch + j] = (uint32_t)base;
     arrive(P.bar + (int64_t)g * 4 + 2);
   }
 
-  // Attention over cnt rows; result in sm.res. Gather mode (ent != nullptr): row i is entry
-  // e0 + i of the group's compacted list (chunk-local runs located through sm.pref over nch
+  // Attention over cnt rows; result in sm.res(). Gather mode (ent != nullptr): row i is entry
+  // e0 + i of the group's compacted list (chunk-local runs located through sm.pref() over nch
   // chunks of Cc tokens); contiguous mode: row i is row r0 + i of kb / vb. One instance of
   // the attention loop serves both, which keeps the kernel's code small.
   struct Rows {
@@ -735,11 +748,12 @@ struct DecodeCta {
   };
   __device__ __noinline__ void attend_list(const float* q_s, int cnt, const Rows R) {
     const int hl = threadIdx.x & 15;
-    float q[G][8];
+    float2 q[G][4];
 #pragma unroll
     for (int h = 0; h < G; ++h)
 #pragma unroll
-      for (int e = 0; e < 8; ++e) q[h][e] = q_s[h * kD + hl * 8 + e];
+      for (int e = 0; e < 4; ++e)
+        q[h][e] = make_float2(q_s[h * kD + hl * 8 + 2 * e], q_s[h * kD + hl * 8 + 2 * e + 1]);
     AttnState<G> st;
     st.init();
     attend_rows<G>(st, q, cnt, [&](int i, const uint16_t*& kp, const uint16_t*& vp, uint32_t& mask) {
@@ -758,77 +772,77 @@ struct DecodeCta {
       }
       kp = R.kb + n * kD;
       vp = R.vb + n * kD;
-    }, sm.stage, kFThreads);
-    attend_merge<G>(st, reinterpret_cast<float*>(sm.stage), sm.res, kFThreads);
+    }, sm.stage(), kFThreads);
+    attend_merge<G>(st, reinterpret_cast<float*>(sm.stage()), sm.res(), kFThreads);
   }
 
   __device__ __noinline__ void merge(const float* parts, int n, float* dst, uint16_t* out_rows) {
     // the score buffer is free whenever partials are merged
-    merge_partials<G>(parts, n, dst, out_rows, sm.scores, 4 * G * P.C_cap, kFThreads);
+    merge_partials<G>(parts, n, dst, out_rows, sm.scores(), 4 * G * P.C_cap, kFThreads);
   }
 
   // ------------------------------------------------------------ phase W
   __device__ void phase_attend(int k) {
-    const int g = group_of(k), j = k - sm.cbase[g];
+    const int g = group_of(k), j = k - sm.cbase()[g];
     const int b = g / P.L.n_ret, r = g % P.L.n_ret, kvh = P.L.ret_kv[r];
     const int N = gN(g);
     const int S = nch(g);
     for (int c = threadIdx.x; c < S; c += kFThreads)
-      sm.pref[c] = (int)__ldcg(P.ccnt + (int64_t)g * P.max_nch + c);
+      sm.pref()[c] = (int)__ldcg(P.ccnt + (int64_t)g * P.max_nch + c);
     __syncthreads();
-    const int U = block_scan_excl(sm.pref, S, sm.ints);
-    if (threadIdx.x == 0) sm.pref[S] = U;
-    if (!smem_mode) rope_query<G>(P, b, kvh, N, sm.qret);   // else formed in phase S
+    const int U = block_scan_excl(sm.pref(), S, sm.ints());
+    if (threadIdx.x == 0) sm.pref()[S] = U;
+    if (!smem_mode) rope_query<G>(P, b, kvh, N, sm.qret());   // else formed in phase S
     __syncthreads();
     const int e0 = (int)(((long long)U * j) / S), e1 = (int)(((long long)U * (j + 1)) / S);
     const int64_t rowbase = (int64_t)r * P.L.T_total + P.cache.seq_off[b];
     const uint32_t* gent = P.ent + (int64_t)g * P.maxN_pad;
-    Rows rows{P.cache.k_ret + rowbase * kD, P.cache.v_ret + rowbase * kD, gent, sm.pref, e0, S, C,
+    Rows rows{P.cache.k_ret + rowbase * kD, P.cache.v_ret + rowbase * kD, gent, sm.pref(), e0, S, C,
               nullptr};
     // this split's entries in one batch of loads, into the (now free) score buffer
-    uint32_t* es = reinterpret_cast<uint32_t*>(sm.scores);
+    uint32_t* es = reinterpret_cast<uint32_t*>(sm.scores());
     if (e1 - e0 <= P.C_cap * G) {
       for (int i = threadIdx.x; i < e1 - e0; i += kFThreads) {
         const int e = e0 + i;
-        const int c = upper_index(sm.pref, S, e);
-        es[i] = __ldcg(gent + (int64_t)c * C + (e - sm.pref[c]));
+        const int c = upper_index(sm.pref(), S, e);
+        es[i] = __ldcg(gent + (int64_t)c * C + (e - sm.pref()[c]));
       }
       __syncthreads();
       rows.sent = es;
     }
     trace(kEvW0);
-    attend_list(sm.qret, e1 - e0, rows);
+    attend_list(sm.qret(), e1 - e0, rows);
     trace(kEvW1);
     // partial -> workspace; team / group merge by the last arrivals
     const int stride = G * (kD + 2);
     float* mine = P.part + (int64_t)k * stride;
-    for (int o = threadIdx.x; o < stride; o += kFThreads) mine[o] = sm.res[o];
+    for (int o = threadIdx.x; o < stride; o += kFThreads) mine[o] = sm.res()[o];
     const int team = j / kTeam, nteams = (S + kTeam - 1) / kTeam;
     const int tcount = min(kTeam, S - team * kTeam);
     __syncthreads();
     if (threadIdx.x == 0) {
       __threadfence();
-      sm.ints[48] = atomicAdd(P.team_arr + sm.cbase[g] + team, 1u) == (uint32_t)(tcount - 1);
+      sm.ints()[48] = atomicAdd(P.team_arr + sm.cbase()[g] + team, 1u) == (uint32_t)(tcount - 1);
     }
     __syncthreads();
     trace(kEvW2);
-    if (!sm.ints[48]) return;
+    if (!sm.ints()[48]) return;
     __threadfence();
     uint16_t* orow = P.out + ((int64_t)b * P.L.Hq + kvh * G) * kD;
-    const float* tparts = P.part + (int64_t)(sm.cbase[g] + team * kTeam) * stride;
+    const float* tparts = P.part + (int64_t)(sm.cbase()[g] + team * kTeam) * stride;
     if (nteams == 1) {
       merge(tparts, tcount, nullptr, orow);
     } else {
-      merge(tparts, tcount, P.tpart + (int64_t)(sm.cbase[g] + team) * stride, nullptr);
+      merge(tparts, tcount, P.tpart + (int64_t)(sm.cbase()[g] + team) * stride, nullptr);
       __syncthreads();
       if (threadIdx.x == 0) {
         __threadfence();
-        sm.ints[49] = atomicAdd(P.bar + (int64_t)g * 4 + 3, 1u) == (uint32_t)(nteams - 1);
+        sm.ints()[49] = atomicAdd(P.bar + (int64_t)g * 4 + 3, 1u) == (uint32_t)(nteams - 1);
       }
       __syncthreads();
-      if (!sm.ints[49]) return;
+      if (!sm.ints()[49]) return;
       __threadfence();
-      merge(P.tpart + (int64_t)sm.cbase[g] * stride, nteams, nullptr, orow);
+      merge(P.tpart + (int64_t)sm.cbase()[g] * stride, nteams, nullptr, orow);
     }
     if (threadIdx.x < G)
       P.sel_counts[(int64_t)b * P.L.Hq + kvh * G + threadIdx.x] =
@@ -840,44 +854,44 @@ struct DecodeCta {
   // Runs local items from the global queue until it is empty. Thread 0 takes the next index
   // while the current item runs, so the queue costs one atomic round trip in total.
   __device__ void local_items() {
-    if (threadIdx.x == 0) sm.ints[33] = (int)atomicAdd(P.misc + 0, 1u);
+    if (threadIdx.x == 0) sm.ints()[33] = (int)atomicAdd(P.misc + 0, 1u);
     __syncthreads();
-    int li = sm.ints[33];
+    int li = sm.ints()[33];
     while (li < P.n_loc_items) {
       __syncthreads();
       unsigned int next = 0;
       if (threadIdx.x == 0) next = atomicAdd(P.misc + 0, 1u);
       local_item(li);
-      if (threadIdx.x == 0) sm.ints[33] = (int)next;
+      if (threadIdx.x == 0) sm.ints()[33] = (int)next;
       __syncthreads();
-      li = sm.ints[33];
+      li = sm.ints()[33];
     }
   }
 
   __device__ void local_item(int li) {
     const int lg = li / P.PL, piece = li % P.PL;
     const int b = lg / P.L.n_loc, x = lg % P.L.n_loc, kvh = P.L.loc_kv[x];
-    const int N = sm.N[b];
+    const int N = sm.N()[b];
     if (N == 0) return;                             // invalid sequence: outputs zeroed in plan
     const int nrows_all = min(N, P.L.ring);
     const int r0 = piece * P.RL;
     const int nrows = max(0, min(nrows_all - r0, P.RL));
-    rope_query<G>(P, b, kvh, N, sm.qloc);
+    rope_query<G>(P, b, kvh, N, sm.qloc());
     __syncthreads();
     const int64_t ring0 = ((int64_t)x * P.L.B + b) * P.L.ring + r0;
     Rows rows{P.cache.k_loc + ring0 * kD, P.cache.v_loc + ring0 * kD, nullptr, nullptr, 0, 0, 0,
               nullptr};
-    attend_list(sm.qloc, nrows, rows);
+    attend_list(sm.qloc(), nrows, rows);
     const int stride = G * (kD + 2);
     float* mine = P.lpart + (int64_t)li * stride;
-    for (int o = threadIdx.x; o < stride; o += kFThreads) mine[o] = sm.res[o];
+    for (int o = threadIdx.x; o < stride; o += kFThreads) mine[o] = sm.res()[o];
     __syncthreads();
     if (threadIdx.x == 0) {
       __threadfence();
-      sm.ints[50] = atomicAdd(P.loc_arr + lg, 1u) == (uint32_t)(P.PL - 1);
+      sm.ints()[50] = atomicAdd(P.loc_arr + lg, 1u) == (uint32_t)(P.PL - 1);
     }
     __syncthreads();
-    if (sm.ints[50]) {
+    if (sm.ints()[50]) {
       __threadfence();
       merge(P.lpart + (int64_t)lg * P.PL * stride, P.PL, nullptr,
             P.out + ((int64_t)b * P.L.Hq + kvh * G) * kD);
@@ -946,8 +960,7 @@ struct DecodeCta {
 
 template <int G>
 __global__ void __launch_bounds__(kFThreads, 1) decode_kernel(const __grid_constant__ DecodeParams P) {
-  extern __shared__ __align__(16) unsigned char smem_raw[];
-  DecodeCta<G> cta(P, smem_raw);
+  DecodeCta<G> cta(P);
   cta.run();
 }
 
