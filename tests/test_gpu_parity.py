@@ -132,11 +132,12 @@ def test_qwen_layer_32k_parity():
     assert conc and diff and np.mean(diff) > 2.5 * np.mean(conc)
 
 
-def test_scores_in_workspace_schedule():
-    """Two retrieval groups of 600K tokens with G = 8: their chunks at the shared-memory score
-    capacity (at most 227 KB / 32 B = 7.1K tokens per CTA) need more than one wave of 148 CTAs,
-    so the scores go to the workspace and the phases run phase-major over each CTA's chunks."""
-    w = _small(G=8, Hkv=2, seq=(600_000,), window=2048, ret=(True, True))
-    heads = [(0, 0), (0, 5), (0, 8), (0, 15)]
+@pytest.mark.parametrize("G,N", [(8, 600_000), (4, 700_000)])
+def test_recomputed_chunk_schedule(G, N):
+    """Two retrieval groups whose chunks at the shared-memory score capacity (at most
+    227 KB / (4 G) tokens per CTA) need more than one wave of 148 CTAs: the chunks run in two
+    waves, and a group's phases wait on chunks of both waves."""
+    w = _small(G=G, Hkv=2, seq=(N,), window=2048, ret=(True, True))
+    heads = [(0, 0), (0, G - 1), (0, G), (0, 2 * G - 1)]
     rep = _parity().run_layer_parity(w=w, layer=0, source="gpu", heads=heads)
     assert all(e["retrieval"] and e["count"] > 0 for e in rep["heads"])
