@@ -133,7 +133,7 @@ def test_qwen_layer_32k_parity():
 
 
 @pytest.mark.parametrize("G,N", [(8, 600_000), (4, 700_000)])
-def test_recomputed_chunk_schedule(G, N):
+def test_two_wave_schedule(G, N):
     """Two retrieval groups whose chunks at the shared-memory score capacity (at most
     227 KB / (4 G) tokens per CTA) need more than one wave of 148 CTAs: the chunks run in two
     waves, and a group's phases wait on chunks of both waves."""
@@ -141,3 +141,47 @@ def test_recomputed_chunk_schedule(G, N):
     heads = [(0, 0), (0, G - 1), (0, G), (0, 2 * G - 1)]
     rep = _parity().run_layer_parity(w=w, layer=0, source="gpu", heads=heads)
     assert all(e["retrieval"] and e["count"] > 0 for e in rep["heads"])
+
+
+# Full benchmark sizes, in the launch configuration the bench times (one layer of the 36, all
+# caches filled on the GPU); the oracle checks sampled heads one by one.
+def _layer_with(w, n_ret):
+    return int(np.nonzero(w.ret_mask.sum(1) == n_ret)[0][0])
+
+
+def _kv(w, layer, retrieval):
+    return [int(g) for g in np.nonzero(w.ret_mask[layer] == retrieval)[0]]
+
+
+def test_full_size_128k_b4_layer():
+    """128K x 4 (Qwen3-8B shape), a layer with three retrieval KV heads: twelve groups whose
+    chunks need two waves; heads of the last and first groups and one local head."""
+    w = workloads.workload(3)
+    layer = _layer_with(w, 3)
+    ret, loc = _kv(w, layer, True), _kv(w, layer, False)
+    heads = [(3, ret[-1] * w.G), (3, ret[-1] * w.G + w.G - 1), (0, ret[0] * w.G + 1),
+             (2, loc[0] * w.G)]
+    rep = _parity().run_layer_parity(w=w, layer=layer, source="gpu", heads=heads)
+    assert all(e["count"] > 0 for e in rep["heads"])
+
+
+def test_full_size_1m_layer():
+    """1M tokens (B = 1), a layer with two retrieval KV heads (chunks in two waves): two query
+    heads of the second group."""
+    w = workloads.workload(4)
+    layer = _layer_with(w, 2)
+    g = _kv(w, layer, True)[-1]
+    heads = [(0, g * w.G), (0, g * w.G + w.G - 1)]
+    rep = _parity().run_layer_parity(w=w, layer=layer, source="gpu", heads=heads)
+    assert all(e["retrieval"] and e["count"] > 0 for e in rep["heads"])
+
+
+def test_full_size_ragged_b64_layer():
+    """Ragged batch of 64 sequences (8K-64K tokens): retrieval heads of the first and last
+    sequences and a local head of a middle one."""
+    w = workloads.workload(5)
+    layer = _layer_with(w, 1)
+    ret, loc = _kv(w, layer, True), _kv(w, layer, False)
+    heads = [(0, ret[0] * w.G), (63, ret[0] * w.G + 1), (31, loc[0] * w.G + 2)]
+    rep = _parity().run_layer_parity(w=w, layer=layer, source="gpu", heads=heads)
+    assert all(e["count"] > 0 for e in rep["heads"])
