@@ -304,7 +304,8 @@ struct DecodeCta {
     }
   }
 
-  // Waits until *ctr >= target, running local items meanwhile. false on timeout / abort.
+  // Waits until *ctr >= target: thread 0 polls with acquire loads while the CTA waits at a
+  // barrier. false on timeout / abort.
   __device__ bool wait_for(const uint32_t* ctr, uint32_t target) {
     const long long t0 = clock64();
     volatile uint32_t* abort_flag = P.misc + 1;
