@@ -1,7 +1,8 @@
 """Decode-step benchmark of the RTPurbo sparse attention path on B200.
 
-One step = one decode step of every layer of the workload: per layer, rtp_append_kv of the
-current token (n_new = 1) and rtp_decode_step, for the whole batch, replayed from a CUDA
+One step = one decode step of every layer of the workload: per layer, the append of the
+current token and the decode step, for the whole batch, in one launch (rtp_decode_step_append;
+--separate-append: rtp_append_kv with n_new = 1, then rtp_decode_step), replayed from a CUDA
 graph. Metric: decode layer-steps/s (a layer-step is one layer over the whole batch), plus the
 achieved HBM bandwidth of the algorithmic bytes the step must move.
 
@@ -308,8 +309,17 @@ def run_ours(args, w):
 
     launches = {"n": 0}
 
+    fused = not args.separate_append
+
     def step(with_append=True, count=False):
         for L in layers:
+            if with_append and fused:          # append + decode in one launch
+                L["lay"].decode_append(L["knew"].view(B, Hkv, 128), L["vnew"].view(B, Hkv, 128),
+                                       L["wk"], L["q"], L["wq"], L["seq"], w.p, L["out"],
+                                       L["cnt"])
+                if count:
+                    launches["n"] += rtp.rtp_last_launch_count()
+                continue
             if with_append:
                 L["lay"].append(L["knew"], L["vnew"], L["wk"], L["start"])
                 if count:
@@ -357,9 +367,9 @@ def run_ours(args, w):
         g_full = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g_full, stream=side):
             step()
-        g_dec = torch.cuda.CUDAGraph()
+        g_dec = torch.cuda.CUDAGraph()                      # the decode kernel alone
         with torch.cuda.graph(g_dec, stream=side):
-            step(with_append=False)
+            step(with_append=fused)
     torch.cuda.current_stream().wait_stream(side)
     torch.cuda.synchronize()
 
@@ -419,7 +429,8 @@ def run_ours(args, w):
 
     value = aggregate(Lyr, 1, world, ms_step)
     peak, peak_kind = load_peaks()
-    achieved = dec_bytes / (dec_step * 1e-3) / 1e9
+    kern_bytes = step_bytes if fused else dec_bytes       # the fused kernel also appends
+    achieved = kern_bytes / (dec_step * 1e-3) / 1e9
     tr = _traffic("rtp_decode_step")
     attended = float(sum(allc)) + sum(min(int(n), w.sinks + w.window) * w.G
                                       for l in range(Lyr) for n in N
@@ -441,7 +452,8 @@ def run_ours(args, w):
                      "peak": peak, "unit": "GB/s", "frac": achieved / peak,
                      "peak_kind": peak_kind + " hbm_gbs (copy bandwidth)",
                      "traffic": None if tr is None else tr["dram_bytes_per_launch"],
-                     "bytes_per_launch": dec_bytes / Lyr, "launch_us": dec_step * 1e3 / Lyr},
+                     "bytes_per_launch": kern_bytes / Lyr, "launch_us": dec_step * 1e3 / Lyr,
+                     "fused_append": fused},
         "e2e": {"value": aggregate(Lyr, 1, world, e2e_ms), "unit": "layer-steps/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
         "gpu_launches": per_step_launches * args.steps,
@@ -486,6 +498,9 @@ def main(argv=None):
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--layers", type=int, default=0, help="run only the first N layers")
     ap.add_argument("--preroll", type=float, default=0.6, help="untimed seconds before timing")
+    ap.add_argument("--separate-append", action="store_true",
+                    help="append with rtp_append_kv and decode with rtp_decode_step (two launches "
+                         "per layer) instead of rtp_decode_step_append")
     args = ap.parse_args(argv)
     from synth import workloads
     w = workloads.workload(args.workload, args.p)

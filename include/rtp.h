@@ -137,6 +137,25 @@ int rtp_decode_step(const rtp_layer_desc* desc, const rtp_cache* cache, const ui
                     int32_t* sel_counts, int32_t* sel_idx, int64_t sel_stride, void* ws,
                     size_t ws_bytes, rtp_stream_t stream);
 
+/*
+ * rtp_append_kv of the decode token (n_new = 1 at position seq_lens[b] - 1) and rtp_decode_step
+ * in one launch, with identical results: the caches end up holding the token exactly as
+ * rtp_append_kv writes it, and the outputs equal those of the two calls in sequence.
+ *   k_new, v_new: bf16 [B][Hkv][128], the decode token's pre-RoPE key and value.
+ *   w_kidx      : fp32 [Hkv][128][16] (may be NULL when the layer has no retrieval head).
+ * Other arguments as rtp_decode_step. Inside the launch, the CTA that scores a retrieval
+ * group's last chunk, and the local item whose ring slice holds the new row, write the token
+ * before reading those rows; every other reader comes after a device-wide arrival. The pages
+ * describe the two steps separately; one launch saves the second launch of every layer.
+ * Errors as rtp_decode_step; RTP_EINVAL when k_new or v_new is NULL, or w_kidx is NULL in a
+ * layer with retrieval heads. An invalid seq_lens[b] skips the sequence (nothing is written).
+ */
+int rtp_decode_step_append(const rtp_layer_desc* desc, const rtp_cache* cache,
+                           const uint16_t* k_new, const uint16_t* v_new, const float* w_kidx,
+                           const uint16_t* q_pre, const float* w_qidx, const int32_t* seq_lens,
+                           double p, uint16_t* out, int32_t* sel_counts, int32_t* sel_idx,
+                           int64_t sel_stride, void* ws, size_t ws_bytes, rtp_stream_t stream);
+
 /* Size of the library-owned scratch of rtp_decode_step_static (bytes). */
 #define RTP_STATIC_SCRATCH_BYTES (16u << 20)
 

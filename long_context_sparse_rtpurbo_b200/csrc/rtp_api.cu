@@ -206,6 +206,13 @@ int launch_decode(DecodeParams& P, const Plan& pl, const DevInfo& di, cudaStream
   return cudaGetLastError() == cudaSuccess ? RTP_OK : RTP_ECUDA;
 }
 
+// rtp_decode_step, optionally appending the decode token in the same launch (k_new != null)
+int decode_impl(const rtp_layer_desc* desc, const rtp_cache* cache, const uint16_t* q_pre,
+                const float* w_qidx, const int32_t* seq_lens, double p, uint16_t* out,
+                int32_t* sel_counts, int32_t* sel_idx, int64_t sel_stride, void* ws,
+                size_t ws_bytes, rtp_stream_t stream, const uint16_t* k_new,
+                const uint16_t* v_new, const float* w_kidx);
+
 }  // namespace
 
 extern "C" {
@@ -274,6 +281,32 @@ int rtp_decode_step(const rtp_layer_desc* desc, const rtp_cache* cache, const ui
                     const float* w_qidx, const int32_t* seq_lens, double p, uint16_t* out,
                     int32_t* sel_counts, int32_t* sel_idx, int64_t sel_stride, void* ws,
                     size_t ws_bytes, rtp_stream_t stream) {
+  return decode_impl(desc, cache, q_pre, w_qidx, seq_lens, p, out, sel_counts, sel_idx,
+                     sel_stride, ws, ws_bytes, stream, nullptr, nullptr, nullptr);
+}
+
+int rtp_decode_step_append(const rtp_layer_desc* desc, const rtp_cache* cache,
+                           const uint16_t* k_new, const uint16_t* v_new, const float* w_kidx,
+                           const uint16_t* q_pre, const float* w_qidx, const int32_t* seq_lens,
+                           double p, uint16_t* out, int32_t* sel_counts, int32_t* sel_idx,
+                           int64_t sel_stride, void* ws, size_t ws_bytes, rtp_stream_t stream) {
+  if (!k_new || !v_new || !desc || !desc->slot_of_kv) return RTP_EINVAL;
+  bool any_ret = false;
+  for (int g = 0; g < desc->Hkv; ++g) any_ret = any_ret || desc->slot_of_kv[g] >= 0;
+  if (any_ret && !w_kidx) return RTP_EINVAL;
+  return decode_impl(desc, cache, q_pre, w_qidx, seq_lens, p, out, sel_counts, sel_idx,
+                     sel_stride, ws, ws_bytes, stream, k_new, v_new, w_kidx);
+}
+
+}  // extern "C"
+
+namespace {
+
+int decode_impl(const rtp_layer_desc* desc, const rtp_cache* cache, const uint16_t* q_pre,
+                const float* w_qidx, const int32_t* seq_lens, double p, uint16_t* out,
+                int32_t* sel_counts, int32_t* sel_idx, int64_t sel_stride, void* ws,
+                size_t ws_bytes, rtp_stream_t stream, const uint16_t* k_new,
+                const uint16_t* v_new, const float* w_kidx) {
   g_launches = 0;
   Plan pl;
   const int rc = make_plan(desc, pl);
@@ -303,6 +336,7 @@ int rtp_decode_step(const rtp_layer_desc* desc, const rtp_cache* cache, const ui
   P.spin_limit = kSpinLimit;
   P.maxN_pad = pl.maxN_pad;
   P.q_pre = q_pre; P.w_qidx = w_qidx; P.seq_lens = seq_lens;
+  P.k_new = k_new; P.v_new = v_new; P.w_kidx = w_kidx;
   P.cache = CachePtrs{cache->k_ret, cache->v_ret, cache->idx, cache->k_loc, cache->v_loc,
                       cache->seq_off, cache->seq_cap};
   P.out = out; P.sel_counts = sel_counts;
@@ -333,6 +367,10 @@ int rtp_decode_step(const rtp_layer_desc* desc, const rtp_cache* cache, const ui
   }
   return r;
 }
+
+}  // namespace
+
+extern "C" {
 
 // Scratch of rtp_decode_step_static: one fixed buffer per device that loads the library,
 // held until the process exits. Host code only ever uses its device address, obtained with

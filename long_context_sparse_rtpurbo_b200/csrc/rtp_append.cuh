@@ -123,4 +123,58 @@ append_kernel(LayerShape L, CachePtrs C, const uint16_t* __restrict__ k_pre,
   }
 }
 
+// The decode token of one (sequence b, KV head g) at position pos, written by a whole CTA of
+// nthreads >= 128 threads inside another kernel: the arithmetic of append_kernel for one token
+// (threads 0..127 compute; every thread passes the barriers). k_row / v_row: its pre-RoPE key
+// and value; part: 8 x 16 doubles of shared memory; idx_patch (shared, nullable) also receives
+// the index row. The caller checked pos < seq_cap[b].
+__device__ __noinline__ void append_token(const LayerShape& L, const CachePtrs& C,
+                                          const uint16_t* k_row, const uint16_t* v_row,
+                                          const float* w_kidx, int b, int g, int64_t pos,
+                                          double* part, uint16_t* idx_patch) {
+  const int t = threadIdx.x;
+  const int s = L.slot[g];
+  uint16_t *kdst = nullptr, *vdst = nullptr, *idst = nullptr;
+  if (s >= 0) {
+    const int64_t row = (int64_t)s * L.T_total + C.seq_off[b] + pos;
+    kdst = C.k_ret + row * kD;
+    vdst = C.v_ret + row * kD;
+    idst = C.idx + row * kR;
+  } else {
+    const int64_t rr = pos < L.sinks ? pos : L.sinks + (pos - L.sinks) % L.window;
+    const int64_t row = ((int64_t)(-1 - s) * L.B + b) * L.ring + rr;
+    kdst = C.k_loc + row * kD;
+    vdst = C.v_loc + row * kD;
+  }
+  if (t < kD) {
+    const int i = t & 63;
+    double sn, cs;
+    rope_sincos((double)pos, L.theta[i], &sn, &cs);
+    const double xa = bf1(k_row[i]), xb = bf1(k_row[i + 64]);
+    const double r = (t < 64) ? (xa * cs - xb * sn) : (xa * sn + xb * cs);
+    kdst[t] = d2bf_rn(r);
+    vdst[t] = v_row[t];
+    if (idst) {
+      const int o = t & 15, kq = t >> 4;
+      double acc = 0.0;
+#pragma unroll
+      for (int e = 0; e < 16; ++e)
+        acc = fma((double)bf1(k_row[kq * 16 + e]),
+                  (double)__ldg(w_kidx + ((int64_t)g * kD + kq * 16 + e) * kR + o), acc);
+      part[kq * 16 + o] = acc;
+    }
+  }
+  __syncthreads();
+  if (idst && t < kR) {
+    double sum = part[t];
+#pragma unroll
+    for (int k2 = 1; k2 < 8; ++k2) sum += part[k2 * 16 + t];
+    const uint16_t bits = d2bf_rn(sum);
+    idst[t] = bits;
+    if (idx_patch) idx_patch[t] = bits;
+  }
+  __threadfence();                        // visible to this CTA's copies and, after its next
+  __syncthreads();                        // arrival, to every other CTA
+}
+
 }  // namespace rtp

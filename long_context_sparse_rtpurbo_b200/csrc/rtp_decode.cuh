@@ -60,6 +60,11 @@ struct DecodeParams {
   const uint16_t* q_pre;
   const float* w_qidx;
   const int32_t* seq_lens;
+  // decode token appended in the same launch (null: appended beforehand): pre-RoPE key and
+  // value [B][Hkv][128] bf16 of position seq_lens[b] - 1, W_kidx [Hkv][128][16]
+  const uint16_t* k_new;
+  const uint16_t* v_new;
+  const float* w_kidx;
   CachePtrs cache;
   uint16_t* out;
   int32_t* sel_counts;
@@ -199,8 +204,9 @@ template <int G> struct Smem {
   __device__ int* pref() const { return (int*)(rtp_smem + P.sm_pref); }
   __device__ int* ints() const { return (int*)(rtp_smem + P.sm_int); }
 };
-// ints[]: [0..31] reduction scratch, [32] wait flag, [33] next local item, [40..47] b*,
-//         [48..50] last-arrival flags
+// ints[]: [0..31] reduction scratch, [32] wait flag, [33] next local item, [34] group of the
+//         total in tmp, [40..47] b*, [48..50] last-arrival flags, [56..63] decode token's
+//         index row (phase S of the last chunk)
 
 // RoPE'd, pre-scaled query of the G heads of KV head kvh at position N - 1 -> q_s[G][128].
 template <int G>
@@ -293,6 +299,14 @@ struct DecodeCta {
 #else
     (void)ev;
 #endif
+  }
+
+  // the decode token (position N - 1) of sequence b, KV head kvh into the caches
+  __device__ __forceinline__ void append_new(int b, int kvh, int N, uint16_t* idx_patch) {
+    const int64_t o = ((int64_t)b * P.L.Hkv + kvh) * kD;
+    append_token(P.L, P.cache, P.k_new + o, P.v_new + o, P.w_kidx, b, kvh, (int64_t)(N - 1),
+                 reinterpret_cast<double*>(sm.tmp()), idx_patch);
+    if (threadIdx.x == 0) sm.ints()[34] = -1;  // sm.tmp() no longer holds a group total
   }
 
   // arrival on a counter after this CTA's writes
@@ -421,6 +435,11 @@ struct DecodeCta {
 #pragma unroll
     for (int st = 0; st < kSStages - 1; ++st) issue(st);
     index_query<G>(P, b, kvh, sm.qidx(), sm.tmp());
+    // The chunk holding the decode token writes it while the first stages are in flight; a
+    // copy of its index row may still be stale, so the stage holding it is patched below.
+    const bool patch = P.k_new && n1 == N;
+    uint16_t* idx_patch = reinterpret_cast<uint16_t*>(sm.ints() + 56);   // 16 bf16
+    if (patch) append_new(b, kvh, N, idx_patch);
     trace(kEvS0);
     float2 qi[G][kR / 2];                    // index query, channel pairs (2j, 2j + 1)
 #pragma unroll
@@ -440,6 +459,12 @@ struct DecodeCta {
       __syncthreads();
       const int rows = min(kSRows, n1 - n0 - st * kSRows);
       const unsigned char* buf = sm.stage() + (st % kSStages) * (kSRows * 32);
+      if (patch && st == nst - 1) {        // the last row of the chunk is the decode token
+        if (threadIdx.x < kR / 2)
+          reinterpret_cast<uint32_t*>(const_cast<unsigned char*>(buf) + (rows - 1) * 32)[threadIdx.x] =
+              reinterpret_cast<const uint32_t*>(idx_patch)[threadIdx.x];
+        __syncthreads();
+      }
 #pragma unroll 1
       for (int i = threadIdx.x; i < rows; i += kFThreads) {
         const uint4 a = *reinterpret_cast<const uint4*>(buf + i * 32);
@@ -877,6 +902,10 @@ struct DecodeCta {
     const int nrows_all = min(N, P.L.ring);
     const int r0 = piece * P.RL;
     const int nrows = max(0, min(nrows_all - r0, P.RL));
+    if (P.k_new) {
+      const int64_t rr = (N - 1) < P.L.sinks ? (N - 1) : P.L.sinks + (N - 1 - P.L.sinks) % P.L.window;
+      if (rr >= r0 && rr < r0 + nrows) append_new(b, kvh, N, nullptr);
+    }
     rope_query<G>(P, b, kvh, N, sm.qloc());
     __syncthreads();
     const int64_t ring0 = ((int64_t)x * P.L.B + b) * P.L.ring + r0;

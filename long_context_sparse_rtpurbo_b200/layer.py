@@ -50,5 +50,14 @@ class DecodeLayer:
         return rtp.rtp_decode_step(self.desc, self.cache, q_pre, w_qidx, seq_lens, p, out,
                                    sel_counts, sel_idx, stride, self.ws, self.ws_bytes, stream)
 
+    def decode_append(self, k_new, v_new, w_kidx, q_pre, w_qidx, seq_lens, p, out, sel_counts,
+                      sel_idx=None, stream=None):
+        """Append of the decode token (k_new, v_new: bf16 [B][Hkv][128] at seq_lens - 1) and
+        the decode step in one launch."""
+        stride = 0 if sel_idx is None else sel_idx.shape[-1]
+        return rtp.rtp_decode_step_append(self.desc, self.cache, k_new, v_new, w_kidx, q_pre,
+                                          w_qidx, seq_lens, p, out, sel_counts, sel_idx, stride,
+                                          self.ws, self.ws_bytes, stream)
+
     def status(self, stream=None) -> int:
         return rtp.rtp_read_device_status(self.ws, stream)

@@ -105,6 +105,18 @@ def rtp_decode_step(desc: LayerDesc, cache: RtpCache, q_pre, w_qidx, seq_lens, p
         _stream(stream)))
 
 
+def rtp_decode_step_append(desc: LayerDesc, cache: RtpCache, k_new, v_new, w_kidx, q_pre, w_qidx,
+                           seq_lens, p, out, sel_counts, sel_idx=None, sel_stride=0, ws=None,
+                           ws_bytes=None, stream=None):
+    """rtp_append_kv of the decode token and rtp_decode_step in one launch (see include/rtp.h)."""
+    if ws_bytes is None:
+        ws_bytes = 0 if ws is None else ws.numel() * ws.element_size()
+    return _check("rtp_decode_step_append", _lib.load().rtp_decode_step_append(
+        desc.ref, ctypes.byref(cache), _ptr(k_new), _ptr(v_new), _ptr(w_kidx), _ptr(q_pre),
+        _ptr(w_qidx), _ptr(seq_lens), float(p), _ptr(out), _ptr(sel_counts), _ptr(sel_idx),
+        int(sel_stride), _ptr(ws), int(ws_bytes), _stream(stream)))
+
+
 def rtp_decode_step_static(desc: LayerDesc, cache: RtpCache, q_pre, w_qidx, seq_lens, p, out,
                            sel_counts, stream=None):
     """rtp_decode_step on the library's own fixed scratch (no workspace argument): for callers

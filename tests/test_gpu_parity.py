@@ -185,3 +185,55 @@ def test_full_size_ragged_b64_layer():
     heads = [(0, ret[0] * w.G), (63, ret[0] * w.G + 1), (31, loc[0] * w.G + 2)]
     rep = _parity().run_layer_parity(w=w, layer=layer, source="gpu", heads=heads)
     assert all(e["count"] > 0 for e in rep["heads"])
+
+
+def _token_bits(w, layer, seq_lens):
+    """The decode token (position N_b - 1) of every sequence and KV head: bf16 [B][Hkv][128]."""
+    kb = np.zeros((w.B, w.Hkv, 128), np.uint16)
+    vb = np.zeros_like(kb)
+    for b in range(w.B):
+        n = int(seq_lens[b])
+        for g in range(w.Hkv):
+            kb[b, g] = w.kpre_bits(layer, b, g, n - 1, n)[0]
+            vb[b, g] = w.v_bits(layer, b, g, n - 1, n)[0]
+    return kb, vb
+
+
+@pytest.mark.parametrize("case", ["mix", "ragged", "waves"])
+def test_fused_append_equals_two_calls(case):
+    """rtp_decode_step_append equals rtp_append_kv (n_new = 1) followed by rtp_decode_step:
+    identical caches, counts and outputs, bit for bit (the same arithmetic runs in both)."""
+    P = _parity()
+    if case == "mix":
+        w = _small(G=4, Hkv=2, seq=(5000,))
+    elif case == "ragged":      # N = 1, N < sinks, N around the ring's wrap, a long one
+        w = _small(B=6, Hkv=2, seq=(1, 3, 259, 260, 261, 5000), kind="needle")
+    else:                       # two groups in two waves
+        w = _small(G=8, Hkv=2, seq=(600_000,), window=2048, ret=(True, True))
+    seq = np.asarray(w.seq_lens, np.int64)
+    q, wq, wk = P.layer_inputs(w, 0, DEV)
+    kb, vb = _token_bits(w, 0, seq)
+    k_new, v_new = P.bits_to_torch(kb, DEV), P.bits_to_torch(vb, DEV)
+    sl = torch.as_tensor(seq.astype(np.int32), device=DEV)
+    res = []
+    for fused in (False, True):
+        lay = P.make_layer(w, 0, DEV)
+        for t in (lay.k_ret, lay.v_ret, lay.idx, lay.k_loc, lay.v_loc):
+            t.zero_()                      # rows no token reaches compare equal too
+        P.fill_layer(w, 0, lay, wk, seq - 1, source="gpu", device=DEV)
+        out = torch.zeros((w.B, w.Hq, 128), dtype=torch.bfloat16, device=DEV)
+        cnt = torch.zeros((w.B, w.Hq), dtype=torch.int32, device=DEV)
+        if fused:
+            lay.decode_append(k_new, v_new, wk, q, wq, sl, w.p, out, cnt)
+        else:
+            lay.append(k_new.view(w.B, 1, w.Hkv, 128), v_new.view(w.B, 1, w.Hkv, 128), wk,
+                       torch.as_tensor((seq - 1).astype(np.int32), device=DEV))
+            lay.decode(q, wq, sl, w.p, out, cnt)
+        torch.cuda.synchronize()
+        assert lay.status() == 0
+        res.append([t.clone() for t in (out.view(torch.int16), cnt, lay.k_ret.view(torch.int16),
+                                         lay.v_ret.view(torch.int16), lay.idx.view(torch.int16),
+                                         lay.k_loc.view(torch.int16), lay.v_loc.view(torch.int16))])
+        del lay
+    for a, b in zip(*res):
+        assert torch.equal(a, b)
