@@ -102,6 +102,21 @@ def test_decode_rejects_bad_arguments_before_any_launch():
     assert rc == _lib.RTP_EINVAL
 
 
+def test_fused_decode_rejects_bad_arguments_before_any_launch():
+    d = _desc()                      # has retrieval heads
+    lib = _lib.load()
+    dummy = 0x1000
+    cache = rtp.make_cache(dummy, dummy, dummy, dummy, dummy, dummy, dummy, 65536)
+    need = rtp.rtp_workspace_bytes(d)
+    args = lambda k, v, wk, ws_bytes: (d.ref, ctypes.byref(cache), k, v, wk, dummy, dummy, dummy,
+                                       0.9, dummy, dummy, None, 0, dummy, ws_bytes, None)
+    assert lib.rtp_decode_step_append(*args(None, dummy, dummy, need)) == _lib.RTP_EINVAL
+    assert lib.rtp_decode_step_append(*args(dummy, None, dummy, need)) == _lib.RTP_EINVAL
+    assert lib.rtp_decode_step_append(*args(dummy, dummy, None, need)) == _lib.RTP_EINVAL
+    # the decode step's own checks follow
+    assert lib.rtp_decode_step_append(*args(dummy, dummy, dummy, need - 1)) == _lib.RTP_EWORKSPACE
+
+
 def test_append_rejects_bad_arguments():
     d = _desc()
     lib = _lib.load()
