@@ -453,7 +453,7 @@ def run_ours(args, w):
                      "peak_kind": peak_kind + " hbm_gbs (copy bandwidth)",
                      "traffic": None if tr is None else tr["dram_bytes_per_launch"],
                      "bytes_per_launch": kern_bytes / Lyr, "launch_us": dec_step * 1e3 / Lyr,
-                     "fused_append": fused},
+                     "fused_append": fused, "frac_of_nominal_8tbs": achieved / 8000.0},
         "e2e": {"value": aggregate(Lyr, 1, world, e2e_ms), "unit": "layer-steps/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
         "gpu_launches": per_step_launches * args.steps,
