@@ -313,3 +313,80 @@ def test_page_constants():
     assert c["n_bins"] == O.N_BINS
     assert c["hist_bytes_per_head"] == O.N_BINS * 4
     assert c["top_p"] == 0.9
+
+
+def _bf_rope(x, m, base=1e6):
+    """R(m) x with plain floats: channel pairs (i, i + 64), angle m * base^(-2i/128)."""
+    out = [0.0] * 128
+    for i in range(64):
+        ang = m * base ** (-2.0 * i / 128)
+        c, s = math.cos(ang), math.sin(ang)
+        out[i] = x[i] * c - x[i + 64] * s
+        out[i + 64] = x[i] * s + x[i + 64] * c
+    return out
+
+
+def _bf_head(q, kp, vv, wq, wk, p, retrieval, sinks, window):
+    """One query head from the definitions, with loops: scores, the 256-bin rule, softmax."""
+    N = len(kp)
+    bf = lambda vals: [float(x) for x in O.bf16_round(np.array(vals))]
+    if retrieval:
+        qi = [sum(q[d] * wq[d][j] for d in range(128)) for j in range(16)]
+        ki = [bf([sum(kp[n][d] * wk[d][j] for d in range(128)) for j in range(16)])
+              for n in range(N)]
+        s = [sum(qi[j] * ki[n][j] for j in range(16)) for n in range(N)]
+        lo, hi = min(s), max(s)
+        if p >= 1.0 or hi == lo:
+            sel = list(range(N))
+        else:
+            bins = [min(255, math.floor((x - lo) * 256 / (hi - lo))) for x in s]
+            mass = [0.0] * 256
+            for n in range(N):
+                mass[bins[n]] += math.exp(s[n] - hi)
+            suffix, acc = [0.0] * 256, 0.0
+            for b in range(255, -1, -1):
+                acc += mass[b]
+                suffix[b] = acc
+            bstar = max(b for b in range(256) if suffix[b] >= p * suffix[0])
+            sel = [n for n in range(N) if bins[n] >= bstar]
+    else:
+        sel = sorted(set(range(min(sinks, N))) | set(range(max(0, N - window), N)))
+    qr = _bf_rope(q, N - 1)
+    z = []
+    for n in sel:
+        k = bf(_bf_rope(kp[n], n))
+        z.append(sum(qr[d] * k[d] for d in range(128)) / math.sqrt(128))
+    zmax = max(z)
+    w = [math.exp(x - zmax) for x in z]
+    out = [sum(w[i] * vv[n][d] for i, n in enumerate(sel)) / sum(w) for d in range(128)]
+    return out, sel
+
+
+@pytest.mark.parametrize("seed", range(4))
+def test_decode_layer_bruteforce_tiny(seed):
+    """The whole layer (two retrieval KV heads and one local, G = 2, two sequences, N <= 64)
+    against a loop-by-loop evaluation of the definitions: query head h reads KV head h // G,
+    selected keys are rotated by their own positions, the query by N - 1."""
+    rng = np.random.default_rng(100 + seed)
+    B, Hkv, G, sinks, window = 2, 3, 2, 2, 5
+    Hq = Hkv * G
+    ret = [True, False, True]
+    lens = [int(rng.choice([1, 3, 8, 33, 64])), int(rng.choice([2, 6, 19, 64]))]
+    p = [0.5, 0.9, 0.99, 1.0][seed]
+    r16 = lambda a: O.bf16_round(a)
+    q = r16(rng.standard_normal((B, Hq, 128)) * 1.5)
+    wq = rng.standard_normal((Hq, 128, 16)) / np.sqrt(128)
+    wk = rng.standard_normal((Hkv, 128, 16)) / np.sqrt(128)
+    kp = {(b, g): r16(rng.standard_normal((lens[b], 128))) for b in range(B) for g in range(Hkv)}
+    vv = {(b, g): r16(rng.standard_normal((lens[b], 128))) for b in range(B) for g in range(Hkv)}
+    res = O.decode_layer(q, wq, wk, lambda b, g: kp[(b, g)], lambda b, g: vv[(b, g)],
+                         np.array(ret), np.array(lens), p, sinks, window)
+    for b in range(B):
+        for h in range(Hq):
+            g = h // G
+            out, sel = _bf_head(q[b, h].tolist(), kp[(b, g)].tolist(), vv[(b, g)].tolist(),
+                                wq[h].tolist(), wk[g].tolist(), p, ret[g], sinks, window)
+            r = res[(b, h)]
+            assert r.count == len(sel)
+            assert list(r.sel) == sel
+            np.testing.assert_allclose(r.out, out, rtol=0, atol=1e-12)
