@@ -33,9 +33,10 @@ Readings where the pages are silent (each is repeated where it is used):
   are positions 0..sinks-1, without duplicates.
 * R9 the attention scale is 1/sqrt(d_h).
 
-Parity of the whole-layer composition against a published number is unpinned: the pages
-print no worked example that can be reproduced without trained weights. Each part is pinned
-by the tests in ``tests/test_oracle.py``.
+The pages print no worked example of a whole layer that can be reproduced without trained
+weights, so no published number pins the composition; it is pinned instead by a brute-force
+evaluation of the definitions on tiny inputs (N <= 64), and each part by its own tests, in
+``tests/test_oracle.py``.
 """
 from __future__ import annotations
 
