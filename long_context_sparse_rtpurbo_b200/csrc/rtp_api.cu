@@ -87,7 +87,14 @@ int make_plan(const rtp_layer_desc* d, Plan& pl) {
   pl.NC_max = 8 * kPlanCTAs + pl.n_groups + 16;
   pl.maxN_pad = (maxN + 63) / 64 * 64;
   const int64_t loc_rows = std::min<int64_t>(maxN, L.ring);
-  const int64_t rl = std::max<int64_t>(kLocRows, (loc_rows + kMaxMerge - 1) / kMaxMerge);
+  // ring rows per local item: kLocRows; in a layer without retrieval heads the local items
+  // are the whole launch, so they are cut to about one per CTA (at least 64 rows)
+  int64_t rl = kLocRows;
+  if (L.n_ret == 0) {
+    const int64_t per_cta = (int64_t(pl.n_lgroups) * loc_rows + kPlanCTAs - 1) / kPlanCTAs;
+    rl = std::min<int64_t>(kLocRows, std::max<int64_t>(64, (per_cta + 63) / 64 * 64));
+  }
+  rl = std::max<int64_t>(rl, (loc_rows + kMaxMerge - 1) / kMaxMerge);
   pl.RL = (int)rl;
   pl.PL = (int)((loc_rows + rl - 1) / rl);
   pl.n_loc_items = pl.n_lgroups * pl.PL;
