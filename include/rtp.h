@@ -174,10 +174,12 @@ int rtp_decode_step_append(const rtp_layer_desc* desc, const rtp_cache* cache,
  *   and clears its status word with synchronous runtime calls: make that first call before
  *   any stream capture on that device.
  *   All calls on a device share the buffer and it keeps the last call's contents; the call
- *   clears the parts that must start at zero. Calls whose work overlaps on the GPU (different
- *   streams, or host threads without ordering) race on it: order them on one stream.
- *   Device-side status (RTP_EDEVICE) is not reported; an invalid sequence still yields zero
- *   outputs and counts.
+ *   clears the parts that must start at zero, the status word included. Calls whose work
+ *   overlaps on the GPU (different streams, or host threads without ordering) race on it:
+ *   order them on one stream.
+ *   Device-side status is not reported: neither RTP_EDEVICE (an invalid sequence still
+ *   yields zero outputs and counts) nor RTP_ETIMEOUT (a device wait that ran out leaves the
+ *   outputs of that call undefined) reaches the caller.
  */
 int rtp_decode_step_static(const rtp_layer_desc* desc, const rtp_cache* cache,
                            const uint16_t* q_pre, const float* w_qidx, const int32_t* seq_lens,
@@ -190,6 +192,22 @@ int rtp_read_device_status(void* ws, rtp_stream_t stream);
 /* Number of kernel launches the last rtp_decode_step / rtp_append_kv call on this thread
  * enqueued (for launch accounting). */
 int32_t rtp_last_launch_count(void);
+
+/*
+ * Test hooks for the failure paths. The pages describe no failure handling; these exist so
+ * the error paths can be exercised without faulting a GPU.
+ *   rtp_debug_set_wait_limit: the limit, in SM clock cycles, of every device-side wait of
+ *     later decode launches (0 restores the default of about one second; negative values are
+ *     RTP_EINVAL). A wait that runs out records RTP_ETIMEOUT in the workspace status word and
+ *     raises an abort flag that ends the launch's other waits; the outputs of that call are
+ *     undefined and its workspace must be re-initialised with rtp_workspace_init. Process-wide.
+ *   rtp_debug_fail_next_call: the next call of rtp_append_kv, rtp_decode_step,
+ *     rtp_decode_step_append or rtp_decode_step_static (on any thread) returns `status` (one
+ *     of the negative RTP_E* codes; 0 cancels) before checking its arguments, and enqueues
+ *     nothing. Process-wide, consumed by that one call.
+ */
+int rtp_debug_set_wait_limit(int64_t cycles);
+int rtp_debug_fail_next_call(int status);
 
 #ifdef __cplusplus
 }

@@ -14,7 +14,8 @@ RTP_OK, RTP_EINVAL, RTP_ESHAPE, RTP_EWORKSPACE, RTP_ECUDA, RTP_ETIMEOUT, RTP_EDE
 EXPORTS = (
     "rtp_status_str", "rtp_build_slot_map", "rtp_workspace_bytes", "rtp_workspace_init",
     "rtp_append_kv", "rtp_decode_step", "rtp_read_device_status", "rtp_last_launch_count",
-    "rtp_decode_step_static", "rtp_decode_step_append",
+    "rtp_decode_step_static", "rtp_decode_step_append", "rtp_debug_set_wait_limit",
+    "rtp_debug_fail_next_call",
 )
 RTP_STATIC_SCRATCH_BYTES = 16 << 20
 
@@ -73,5 +74,9 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.rtp_read_device_status.argtypes = [vp, vp]
     lib.rtp_last_launch_count.restype = i32
     lib.rtp_last_launch_count.argtypes = []
+    lib.rtp_debug_set_wait_limit.restype = ctypes.c_int
+    lib.rtp_debug_set_wait_limit.argtypes = [i64]
+    lib.rtp_debug_fail_next_call.restype = ctypes.c_int
+    lib.rtp_debug_fail_next_call.argtypes = [ctypes.c_int]
     _lib = lib
     return lib

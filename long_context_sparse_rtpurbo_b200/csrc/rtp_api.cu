@@ -5,6 +5,7 @@
 #include <algorithm>
 #include <cmath>
 #include <cstring>
+#include <atomic>
 #include <mutex>
 
 #include "../../include/rtp.h"
@@ -18,7 +19,14 @@ thread_local int32_t g_launches = 0;
 
 constexpr int kPlanCTAs = 160;      // upper bound on decode CTAs (one per SM; B200 has 148)
 constexpr int kLocRows = 256;       // ring rows per local attention item
-constexpr long long kSpinLimit = 2000000000LL;   // ~1 s of SM clock per device-side wait
+constexpr long long kSpinLimitDefault = 2000000000LL;   // ~1 s of SM clock per device wait
+
+// Test hooks (see include/rtp.h): the device-wait limit of later launches, and an error code
+// the next entry-point call returns before enqueueing anything.
+std::atomic<long long> g_spin_limit{kSpinLimitDefault};
+std::atomic<int> g_fail_next{0};
+
+int take_injected() { return g_fail_next.exchange(0); }
 
 inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 inline int align16(int x) { return (x + 15) & ~15; }
@@ -26,10 +34,11 @@ inline int align16(int x) { return (x + 15) & ~15; }
 struct Plan {
   LayerShape L;
   int C_min, max_nch, NC_max, n_groups, n_lgroups, RL, PL, n_loc_items;
-  int64_t maxN_pad;
+  int64_t cand_stride;
   size_t off_ctrl, ctrl_bytes;
-  size_t off_lohi, off_hcnt, off_bar, off_team, off_locarr, off_misc, off_hist;
-  size_t off_scores, off_ent, off_ccnt, off_cstat, off_part, off_tpart, off_lpart, off_trace, total;
+  size_t off_bar, off_team, off_locarr, off_misc, off_hist, off_hcnt;
+  size_t off_bstar, off_cstat, off_ccnt, off_cpos, off_cbin, off_part, off_tpart, off_lpart,
+      off_trace, total;
 };
 
 int check_desc(const rtp_layer_desc* d, LayerShape& L) {
@@ -40,7 +49,7 @@ int check_desc(const rtp_layer_desc* d, LayerShape& L) {
   if (G != 1 && G != 2 && G != 4 && G != 8) return RTP_ESHAPE;
   if (d->head_dim != kD || d->idx_dim != kR) return RTP_ESHAPE;
   if (d->sinks < 0 || d->window < 1 || d->max_seq_len < 1) return RTP_EINVAL;
-  if (d->max_seq_len > (int64_t(1) << 24)) return RTP_ESHAPE;     // entries pack n in 24 bits
+  if (d->max_seq_len > (int64_t(1) << 24)) return RTP_ESHAPE;     // gather entries pack n in 24 bits
   if (!(d->rope_base > 0.0)) return RTP_EINVAL;
   memset(&L, 0, sizeof(L));
   L.B = d->B; L.Hq = d->Hq; L.Hkv = d->Hkv; L.G = G;
@@ -76,43 +85,49 @@ int make_plan(const rtp_layer_desc* d, Plan& pl) {
   pl.n_groups = L.B * L.n_ret;
   pl.n_lgroups = L.B * L.n_loc;
   if (pl.n_groups > 8 * kFThreads) return RTP_ESHAPE;
-  // chunks: at least C_min tokens, so a launch never has more than 8 per CTA plus one per group
-  int64_t cmin = (int64_t(pl.n_groups) * maxN + 8 * kPlanCTAs - 1) / (8 * kPlanCTAs);
-  cmin = std::max<int64_t>(cmin, 1024);
-  cmin = std::max<int64_t>(cmin, (maxN + kTeam * kMaxMerge - 1) / (kTeam * kMaxMerge));
-  cmin = (cmin + 255) / 256 * 256;
+  // chunks: at least C_min tokens, so a launch has at most kMaxSteps chunks per CTA and a
+  // group at most 4096 chunks (the shared-memory prefix of phase W)
+  int64_t cmin = (int64_t(pl.n_groups) * maxN + int64_t(kMaxSteps) * kPlanCTAs - 1) /
+                 (int64_t(kMaxSteps) * kPlanCTAs);
+  cmin = std::max<int64_t>(cmin, 64);
+  cmin = std::max<int64_t>(cmin, (maxN + 4095) / 4096);
+  cmin = (cmin + 63) / 64 * 64;
   pl.C_min = (int)cmin;
   pl.max_nch = (int)((maxN + cmin - 1) / cmin);
-  if (pl.max_nch > kTeam * kMaxMerge) return RTP_ESHAPE;
-  pl.NC_max = 8 * kPlanCTAs + pl.n_groups + 16;
-  pl.maxN_pad = (maxN + 63) / 64 * 64;
+  pl.NC_max = (int)std::min<int64_t>(int64_t(pl.n_groups) * pl.max_nch,
+                                     int64_t(kMaxSteps) * kPlanCTAs + pl.n_groups);
+  pl.NC_max = std::max(pl.NC_max, 1);
+  pl.cand_stride = (maxN + 63) / 64 * 64;
   const int64_t loc_rows = std::min<int64_t>(maxN, L.ring);
-  // ring rows per local item: kLocRows; in a layer without retrieval heads the local items
-  // are the whole launch, so they are cut to about one per CTA (at least 64 rows)
-  int64_t rl = kLocRows;
+  // ring rows per local item: about kLocRows, in whole tiles; in a layer without retrieval
+  // heads the local items are the whole launch, so they are cut to about one per CTA
+  int64_t pl_n = (loc_rows + kLocRows - 1) / kLocRows;
   if (L.n_ret == 0) {
     const int64_t per_cta = (int64_t(pl.n_lgroups) * loc_rows + kPlanCTAs - 1) / kPlanCTAs;
-    rl = std::min<int64_t>(kLocRows, std::max<int64_t>(64, (per_cta + 63) / 64 * 64));
+    const int64_t rl = std::max<int64_t>(64, (per_cta + 15) / 16 * 16);
+    pl_n = std::max<int64_t>(pl_n, (loc_rows + rl - 1) / rl);
   }
-  rl = std::max<int64_t>(rl, (loc_rows + kMaxMerge - 1) / kMaxMerge);
+  pl_n = std::max<int64_t>(pl_n, 1);
+  int64_t rl = (loc_rows + pl_n - 1) / pl_n;
+  rl = (rl + 15) / 16 * 16;
   pl.RL = (int)rl;
   pl.PL = (int)((loc_rows + rl - 1) / rl);
   pl.n_loc_items = pl.n_lgroups * pl.PL;
   const size_t part_bytes = sizeof(float) * G * (kD + 2);
   size_t o = 256;                                   // [0, 256): status word
   pl.off_ctrl = o;
-  pl.off_lohi = o;   o = align256(o + sizeof(uint32_t) * pl.n_groups * 2 * G);
-  pl.off_hcnt = o;   o = align256(o + sizeof(int32_t) * pl.n_groups * G);
   pl.off_bar = o;    o = align256(o + sizeof(uint32_t) * pl.n_groups * 4);
   pl.off_team = o;   o = align256(o + sizeof(uint32_t) * pl.NC_max);
   pl.off_locarr = o; o = align256(o + sizeof(uint32_t) * std::max(pl.n_lgroups, 1));
   pl.off_misc = o;   o = align256(o + sizeof(uint32_t) * 16);
   pl.off_hist = o;   o = align256(o + sizeof(unsigned long long) * pl.n_groups * G * kBins);
+  pl.off_hcnt = o;   o = align256(o + sizeof(int32_t) * pl.n_groups * G);
   pl.ctrl_bytes = o - pl.off_ctrl;
-  pl.off_scores = o; o = align256(o + sizeof(float) * pl.n_groups * G * pl.maxN_pad);
-  pl.off_ent = o;    o = align256(o + sizeof(uint32_t) * pl.n_groups * pl.maxN_pad);
-  pl.off_ccnt = o;   o = align256(o + sizeof(uint32_t) * pl.n_groups * pl.max_nch);
-  pl.off_cstat = o;  o = align256(o + sizeof(float) * 2 * pl.n_groups * pl.max_nch * G);
+  pl.off_bstar = o;  o = align256(o + sizeof(int32_t) * pl.n_groups * G);
+  pl.off_cstat = o;  o = align256(o + 16 * size_t(pl.n_groups) * pl.max_nch * G);
+  pl.off_ccnt = o;   o = align256(o + sizeof(uint32_t) * size_t(pl.n_groups) * pl.max_nch);
+  pl.off_cpos = o;   o = align256(o + sizeof(uint32_t) * size_t(pl.n_groups) * pl.cand_stride);
+  pl.off_cbin = o;   o = align256(o + 8 * size_t(pl.n_groups) * pl.cand_stride);
   pl.off_part = o;   o = align256(o + part_bytes * pl.NC_max);
   pl.off_tpart = o;  o = align256(o + part_bytes * pl.NC_max);
   pl.off_lpart = o;  o = align256(o + part_bytes * std::max(pl.n_loc_items, 1));
@@ -129,7 +144,7 @@ template <class T>
 T* at(void* ws, size_t off) { return reinterpret_cast<T*>(static_cast<char*>(ws) + off); }
 
 struct DevInfo {
-  int sms = 0, smem_optin = 0;
+  int dev = 0, sms = 0, smem_optin = 0;
 };
 
 int dev_info(DevInfo& di) {
@@ -139,6 +154,7 @@ int dev_info(DevInfo& di) {
   if (cudaGetDevice(&dev) != cudaSuccess) return RTP_ECUDA;
   if (dev != cached_dev) {
     DevInfo x;
+    x.dev = dev;
     if (cudaDeviceGetAttribute(&x.sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
         cudaDeviceGetAttribute(&x.smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) !=
             cudaSuccess)
@@ -150,49 +166,80 @@ int dev_info(DevInfo& di) {
   return RTP_OK;
 }
 
-// Shared-memory layout of the decode kernel; returns the bytes, sets C_cap.
+// Shared-memory layout of the decode kernel: the staging region, the score slot right after
+// it (the two form the free region once the slot is dead), then the small arrays. Returns the
+// bytes, sets C_cap.
 int smem_layout(DecodeParams& P, const Plan& pl, int smem_optin) {
   const int G = P.L.G;
-  int o = 0;
-  const int merge_scratch = 4 * std::max((kFThreads / 32) * G * kD + 2 * (kFThreads / 32) * G,
-                                         2 * kMaxMerge * G + 2 * G);
-  const int stage = std::max({AttnCfg<8>::stage_bytes(kFThreads), 4 * 512 * 32, merge_scratch});
-  P.sm_stage = o; o = align16(o + stage);
-  P.sm_res = o;   o = align16(o + 4 * G * (kD + 2));
-  P.sm_qret = o;  o = align16(o + 4 * G * kD);
-  P.sm_qloc = o;  o = align16(o + 4 * G * kD);
-  P.sm_qidx = o;  o = align16(o + 4 * G * kR);
-  P.sm_tmp = o;   o = align16(o + 4 * kFThreads);
-  P.sm_hist = o;  o = align16(o + 8 * G * kHistStride);
-  P.sm_N = o;     o = align16(o + 4 * P.L.B);
-  P.sm_cbase = o; o = align16(o + 4 * (pl.n_groups + 1));
-  P.sm_pref = o;  o = align16(o + 4 * (pl.max_nch + 1));
-  P.sm_int = o;   o = align16(o + 4 * 64);
-  P.sm_scores = o;
+  int small = 0;
+  small += align16(4 * G * kD);                         // q
+  small += kQBytes;                                     // query buffer (bf16 hi / lo)
+  small += align16(4 * G * kR);                         // qidx
+  small += align16(8 * G * kHistStride);                // hist (two 32-bit words per bin)
+  small += align16(4 * G * (kD + 2));                   // res
+  small += align16(8 * kFThreads);                      // tmp
+  small += align16(4 * 64);                             // ints
+  small += align16(4 * P.L.B);                          // N
+  small += align16(4 * (pl.n_groups + 1));              // cbase
+  small += align16(8 * kMaxSteps * G);                  // tcache
   const int budget = smem_optin - 1024;
-  int cap = (budget - o) / (4 * G) - kHeadPad;
-  cap = std::min(cap, 16384) / 256 * 256;
-  if (cap < 256) cap = 0;
+  int cap = (budget - kStageBytes - small) / (4 * G) - kHeadPad;
+  cap = std::min(cap, 16384) / 64 * 64;
+  if (cap < 512) return -1;
   P.C_cap = cap;
-  return o + 4 * G * (cap + kHeadPad);
+  int o = 0;
+  P.sm_stage = o; o += kStageBytes;
+  P.sm_slot = o;  o += 4 * G * (cap + kHeadPad);
+  P.free_bytes = o;
+  P.sm_q = o;     o += align16(4 * G * kD);
+  P.sm_qbuf = o;  o += kQBytes;
+  P.sm_qidx = o;  o += align16(4 * G * kR);
+  P.sm_hist = o;  o += align16(8 * G * kHistStride);
+  P.sm_res = o;   o += align16(4 * G * (kD + 2));
+  P.sm_tmp = o;   o += align16(8 * kFThreads);
+  P.sm_int = o;   o += align16(4 * 64);
+  P.sm_N = o;     o += align16(4 * P.L.B);
+  P.sm_cbase = o; o += align16(4 * (pl.n_groups + 1));
+  P.sm_tcache = o; o += align16(8 * kMaxSteps * G);
+  return o;
+}
+
+// The shared-memory opt-in of decode_kernel<G> is a per-device function attribute: set it
+// once per (device, instance), under a lock.
+std::mutex g_attr_mu;
+int g_attr_smem[4][64];
+bool g_attr_init = false;
+
+template <int G>
+int ensure_smem_attr(int dev, int smem) {
+  constexpr int gi = G == 1 ? 0 : (G == 2 ? 1 : (G == 4 ? 2 : 3));
+  if (dev < 0 || dev >= 64) return RTP_ECUDA;
+  std::lock_guard<std::mutex> lock(g_attr_mu);
+  if (!g_attr_init) {
+    for (auto& row : g_attr_smem) for (int& v : row) v = -1;
+    g_attr_init = true;
+  }
+  if (g_attr_smem[gi][dev] < smem) {
+    if (cudaFuncSetAttribute(decode_kernel<G>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             smem) != cudaSuccess)
+      return RTP_ECUDA;
+    g_attr_smem[gi][dev] = smem;
+  }
+  return RTP_OK;
 }
 
 template <int G>
 int launch_decode(DecodeParams& P, const Plan& pl, const DevInfo& di, cudaStream_t st,
                   int32_t* sel_idx, int64_t sel_stride) {
   const int smem = smem_layout(P, pl, di.smem_optin);
-  static int attr_smem = -1;              // per template instance
-  if (attr_smem < smem) {
-    if (cudaFuncSetAttribute(decode_kernel<G>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             smem) != cudaSuccess)
-      return RTP_ECUDA;
-    attr_smem = smem;
-  }
+  if (smem < 0) return RTP_ESHAPE;
+  if (ensure_smem_attr<G>(di.dev, smem) != RTP_OK) return RTP_ECUDA;
   int per_sm = 0;
   if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, decode_kernel<G>, kFThreads, smem) !=
           cudaSuccess || per_sm < 1)
     return RTP_ECUDA;
   P.P = std::min(di.sms, kPlanCTAs);
+  if (pl.n_groups >= kMaxSteps * P.P) return RTP_ESHAPE;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(P.P);
   cfg.blockDim = dim3(kFThreads);
@@ -263,6 +310,7 @@ int rtp_append_kv(const rtp_layer_desc* desc, const rtp_cache* cache, const uint
                   const uint16_t* v, const float* w_kidx, const int32_t* start_pos,
                   const int32_t* n_new_b, int32_t n_new, void* ws, rtp_stream_t stream) {
   g_launches = 0;
+  if (const int inj = take_injected()) return inj;
   LayerShape L;
   const int rc = check_desc(desc, L);
   if (rc != RTP_OK) return rc;
@@ -315,6 +363,7 @@ int decode_impl(const rtp_layer_desc* desc, const rtp_cache* cache, const uint16
                 size_t ws_bytes, rtp_stream_t stream, const uint16_t* k_new,
                 const uint16_t* v_new, const float* w_kidx) {
   g_launches = 0;
+  if (const int inj = take_injected()) return inj;
   Plan pl;
   const int rc = make_plan(desc, pl);
   if (rc != RTP_OK) return rc;
@@ -340,25 +389,25 @@ int decode_impl(const rtp_layer_desc* desc, const rtp_cache* cache, const uint16
   P.n_loc_items = pl.n_loc_items;
   P.select_all = p >= 1.0 ? 1 : 0;
   P.p = p;
-  P.spin_limit = kSpinLimit;
-  P.maxN_pad = pl.maxN_pad;
+  P.spin_limit = g_spin_limit.load();
+  P.cand_stride = pl.cand_stride;
   P.q_pre = q_pre; P.w_qidx = w_qidx; P.seq_lens = seq_lens;
   P.k_new = k_new; P.v_new = v_new; P.w_kidx = w_kidx;
   P.cache = CachePtrs{cache->k_ret, cache->v_ret, cache->idx, cache->k_loc, cache->v_loc,
                       cache->seq_off, cache->seq_cap};
   P.out = out; P.sel_counts = sel_counts;
   P.status = at<int>(ws, 0);
-  P.lohi = at<uint32_t>(ws, pl.off_lohi);
-  P.hcnt = at<int32_t>(ws, pl.off_hcnt);
   P.bar = at<uint32_t>(ws, pl.off_bar);
   P.team_arr = at<uint32_t>(ws, pl.off_team);
   P.loc_arr = at<uint32_t>(ws, pl.off_locarr);
   P.misc = at<uint32_t>(ws, pl.off_misc);
   P.hist = at<unsigned long long>(ws, pl.off_hist);
-  P.scores = at<float>(ws, pl.off_scores);
-  P.ent = at<uint32_t>(ws, pl.off_ent);
+  P.hcnt = at<int32_t>(ws, pl.off_hcnt);
+  P.bstar = at<int32_t>(ws, pl.off_bstar);
+  P.cstat = at<float4>(ws, pl.off_cstat);
   P.ccnt = at<uint32_t>(ws, pl.off_ccnt);
-  P.cstat = at<float2>(ws, pl.off_cstat);
+  P.cpos = at<uint32_t>(ws, pl.off_cpos);
+  P.cbin = at<uint2>(ws, pl.off_cbin);
   P.part = at<float>(ws, pl.off_part);
   P.tpart = at<float>(ws, pl.off_tpart);
   P.lpart = at<float>(ws, pl.off_lpart);
@@ -409,6 +458,7 @@ int rtp_decode_step_static(const rtp_layer_desc* desc, const rtp_cache* cache,
                            const uint16_t* q_pre, const float* w_qidx, const int32_t* seq_lens,
                            double p, uint16_t* out, int32_t* sel_counts, rtp_stream_t stream) {
   g_launches = 0;
+  if (const int inj = take_injected()) return inj;
   const size_t need = rtp_workspace_bytes(desc);
   if (need == 0) {
     Plan pl;
@@ -418,6 +468,8 @@ int rtp_decode_step_static(const rtp_layer_desc* desc, const rtp_cache* cache,
   void* ws = nullptr;
   const int rc = static_scratch(&ws);
   if (rc != RTP_OK) return rc;
+  // the status word is not reported by this entry point; clear what an earlier call left
+  if (cudaMemsetAsync(ws, 0, 256, (cudaStream_t)stream) != cudaSuccess) return RTP_ECUDA;
   return rtp_decode_step(desc, cache, q_pre, w_qidx, seq_lens, p, out, sel_counts, nullptr, 0,
                          ws, (size_t)RTP_STATIC_SCRATCH_BYTES, stream);
 }
@@ -433,5 +485,17 @@ int rtp_read_device_status(void* ws, rtp_stream_t stream) {
 }
 
 int32_t rtp_last_launch_count(void) { return g_launches; }
+
+int rtp_debug_set_wait_limit(int64_t cycles) {
+  if (cycles < 0) return RTP_EINVAL;
+  g_spin_limit.store(cycles == 0 ? kSpinLimitDefault : (long long)cycles);
+  return RTP_OK;
+}
+
+int rtp_debug_fail_next_call(int status) {
+  if (status > 0 || status < RTP_EDEVICE) return RTP_EINVAL;
+  g_fail_next.store(status);
+  return RTP_OK;
+}
 
 }  // extern "C"

@@ -1,269 +1,305 @@
-// Exact softmax attention of the G query heads of one KV head over a list of K/V rows
-// ("Full Attention Strikes Back" (paper text) §3.2 eq. (5): O = sum_n softmax(q^T k_n / sqrt(d)) v_n).
+// Exact softmax attention of the G query heads of one KV head over a list of K/V rows, on the
+// tensor cores ("Full Attention Strikes Back" (paper text) §3.2 eq. (5):
+// O = sum_n softmax(q^T k_n / sqrt(d)) v_n over the rows of S).
 //
-// Layout on the SM: a half-warp (16 lanes) owns kRows rows per step, each lane 8 of the 128
-// channels (16 bytes of K and of V per row). Rows are staged in shared memory with cp.async
-// (16 bytes per lane, L2-only), two steps deep, so the loads of step i+1 are in flight while
-// step i is computed and no registers are held by loads in flight. A lane only ever reads the
-// bytes it copied itself, so no barrier is needed between copy and use. The kRows x G partial
-// dot products of a lane are reduced over the 16 lanes by recursive halving (each step
-// exchanges half of the remaining values), so every lane ends with one complete logit; the
-// probabilities are then broadcast for the V update. Softmax state (running max, sum,
-// 8-channel accumulator per head) is kept per half-warp in the log2 domain (q carries
-// log2(e)/sqrt(d)) and merged across half-warps at the end.
+// A warp takes tiles of 16 rows. Logits come from mma.sync m16n8k16 (bf16 x bf16 -> fp32)
+// with the rows as M, the heads as N (G <= 8 real columns) and the channels as K:
+// S^T = K Q^T. The query is split into two bf16 terms (q = q_hi + q_lo, with q_lo the rounded
+// remainder), so the logits carry ~16 significant bits of q instead of 8. The probabilities
+// P of a tile are transposed in registers (movmatrix) into the B operand of O^T += V^T P^T
+// (channels as M, heads as N, the 16 rows as K), again as two bf16 terms, so the result keeps
+// fp32-level accuracy; the softmax state (running max, sum) is fp32 in the log2 domain
+// (the query carries log2(e)/sqrt(d)).
+//
+// Staging: rows are copied with cp.async (16 bytes per lane, L2 only) into the warp's own
+// tile buffer, 16-byte chunks XOR-swizzled by the row index so the ldmatrix reads of eight
+// rows hit eight different bank groups. A warp only reads what it copied itself, so the only
+// synchronisation inside the loop is __syncwarp.
 #pragma once
 
 #include "rtp_common.cuh"
 
 namespace rtp {
 
-template <int G> struct AttnCfg {
-  static constexpr int kRows = 2;                         // rows per half-warp per step
-  static constexpr int kVals = kRows * G;                 // partial dots per lane
-  static constexpr int kStages = 2;
-  // staging bytes for a CTA of nthreads threads
-  static constexpr int stage_bytes(int nthreads) { return kStages * (nthreads / 16) * kRows * 512; }
-};
-
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return (uint32_t)__cvta_generic_to_shared(p);
+}
 __device__ __forceinline__ void cp_async16(void* smem, const void* gmem) {
-  const unsigned s = (unsigned)__cvta_generic_to_shared(smem);
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(s), "l"(gmem) : "memory");
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(smem)), "l"(gmem)
+               : "memory");
 }
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 template <int N>
-__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
-
-// Recursive-halving reduction of n values over the 16 lanes of a half-warp. On exit v[0] of
-// lane hl holds the full sum of value index (hl >> (4 - log2 n)) (n <= 16).
-template <int N>
-__device__ __forceinline__ void halving_reduce(float (&v)[N], int hl) {
-  static_assert(N >= 1 && N <= 16 && (N & (N - 1)) == 0, "power of two up to 16");
-  int n = N;
-#pragma unroll
-  for (int m = 8; m >= 1; m >>= 1) {
-    if (n > 1) {
-      const bool up = (hl & m) != 0;
-#pragma unroll
-      for (int i = 0; i < N / 2; ++i) {
-        if (i < n / 2) {
-          const float send = up ? v[i] : v[i + n / 2];
-          const float keep = up ? v[i + n / 2] : v[i];
-          v[i] = keep + __shfl_xor_sync(0xffffffffu, send, m);
-        }
-      }
-      n >>= 1;
-    } else {
-      v[0] += __shfl_xor_sync(0xffffffffu, v[0], m);
-    }
-  }
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
 }
 
-// Softmax state of one half-warp; the accumulator holds channel pairs (2e, 2e + 1), so the
-// V update is one packed f32x2 multiply-add per pair.
-template <int G> struct AttnState {
-  float m[G], l[G];
-  float2 a2[G][4];
-  __device__ __forceinline__ float& acc(int h, int e) { return (&a2[h][e >> 1].x)[e & 1]; }
-  __device__ __forceinline__ void init() {
-#pragma unroll
-    for (int h = 0; h < G; ++h) {
-      m[h] = -INFINITY;
-      l[h] = 0.f;
-#pragma unroll
-      for (int e = 0; e < 4; ++e) a2[h][e] = make_float2(0.f, 0.f);
-    }
-  }
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t (&r)[4]) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr));
+}
+__device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t (&r)[4]) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr));
+}
+__device__ __forceinline__ uint32_t movm_t(uint32_t a) {
+  uint32_t d;
+  asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(d) : "r"(a));
+  return d;
+}
+// d += A B, m16n8k16, bf16 inputs, fp32 accumulators
+__device__ __forceinline__ void mma_bf16(float (&d)[4], const uint32_t (&a)[4], uint32_t b0,
+                                         uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+      "{%8,%9}, {%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+// two floats -> bf16x2 (x in the low half), round to nearest even
+__device__ __forceinline__ uint32_t pack_bf2(float x, float y) {
+  uint32_t r;
+  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(y), "f"(x));
+  return r;
+}
+// (x, y) = hi + lo with hi = bf16(x, y) and lo = bf16 of the exact float remainders
+__device__ __forceinline__ void split_bf2(float x, float y, uint32_t& hi, uint32_t& lo) {
+  hi = pack_bf2(x, y);
+  lo = pack_bf2(x - __uint_as_float(hi << 16), y - __uint_as_float(hi & 0xffff0000u));
+}
+
+constexpr int kTileRows = 16;
+constexpr int kTileBytes = kTileRows * 512;     // K (16 x 256 B) then V (16 x 256 B)
+constexpr int kAccStride = 132;                  // floats per head row of the merge scratch
+
+// Online-softmax state of one warp: heads h0 = 2 (lane & 3) and h0 + 1 of the thread,
+// O^T fragments of 8 channel tiles. The query's B fragments are read from a shared buffer.
+struct WarpAttn {
+  float acc[8][4];
+  float m[2], l[2];              // running max; this thread's share of the running sum
+  uint32_t qb;                   // shared address of the query buffer (kQBytes)
 };
 
-// 8 bf16 -> 4 packed channel pairs
-__device__ __forceinline__ void unpack_pairs(const uint4& w, float2 (&f)[4]) {
-  f[0] = make_float2(bf_lo(w.x), bf_hi(w.x));
-  f[1] = make_float2(bf_lo(w.y), bf_hi(w.y));
-  f[2] = make_float2(bf_lo(w.z), bf_hi(w.z));
-  f[3] = make_float2(bf_lo(w.w), bf_hi(w.w));
-}
+// Query buffer: q_hi and q_lo as bf16 [8 heads][128] each (rows of heads >= G are zero),
+// 16-byte chunks XOR-swizzled by the head, so one ldmatrix.x4 per 16-channel step gives the
+// B fragments of Q^T (hi: matrices 0, 1; lo: matrices 2, 3).
+constexpr int kQBytes = 2 * 8 * kD * 2;
 
-// One step of kRows staged rows for a half-warp; kw/vw: this lane's 16 bytes of each row
-// (zero for rows no head attends), mask: heads that attend each row.
+// Fills the query buffer from q_s: [G][128] fp32 query rows pre-scaled by log2(e)/sqrt(d).
+// Called by every thread of the CTA; ends with a barrier.
 template <int G>
-__device__ __forceinline__ void attend_step(AttnState<G>& st, const float2 (&q)[G][4],
-                                            const uint4 (&kw)[AttnCfg<G>::kRows],
-                                            const uint4 (&vw)[AttnCfg<G>::kRows],
-                                            const uint32_t (&mask)[AttnCfg<G>::kRows], int hl) {
-  constexpr int R = AttnCfg<G>::kRows;
-  constexpr int V = AttnCfg<G>::kVals;
-  float d[V];
+__device__ __forceinline__ void fill_qbuf(unsigned char* qbuf, const float* q_s, int nthreads) {
+  for (int e = threadIdx.x; e < 8 * kD / 2; e += nthreads) {
+    const int h = e / (kD / 2), c = (e % (kD / 2)) * 2;
+    const float x = h < G ? q_s[h * kD + c] : 0.f;
+    const float y = h < G ? q_s[h * kD + c + 1] : 0.f;
+    uint32_t hi, lo;
+    split_bf2(x, y, hi, lo);
+    const int off = h * 256 + (((c >> 3) ^ h) << 4) + (c & 7) * 2;
+    *reinterpret_cast<uint32_t*>(qbuf + off) = hi;
+    *reinterpret_cast<uint32_t*>(qbuf + 2048 + off) = lo;
+  }
+  __syncthreads();
+}
+
+__device__ __forceinline__ void warp_attn_init(WarpAttn& W, const unsigned char* qbuf) {
 #pragma unroll
-  for (int r = 0; r < R; ++r) {
-    float2 k[4];
-    unpack_pairs(kw[r], k);
+  for (int mt = 0; mt < 8; ++mt)
 #pragma unroll
-    for (int h = 0; h < G; ++h) {
-      float2 a = __fmul2_rn(q[h][0], k[0]);
+    for (int e = 0; e < 4; ++e) W.acc[mt][e] = 0.f;
+  W.m[0] = W.m[1] = -INFINITY;
+  W.l[0] = W.l[1] = 0.f;
+  W.qb = smem_u32(qbuf);
+}
+
+// Copies up to 16 rows into a tile: lane l handles row l / 2 (both K and V, the 16-byte
+// chunks of parity l & 1, XOR-swizzled by the row). Rows with ok = false get zero V (their
+// logits are masked; a zero V keeps stale shared memory out of the P V product).
+__device__ __forceinline__ void tile_copy(unsigned char* tile, const uint16_t* krow,
+                                          const uint16_t* vrow, bool ok) {
+  const int lane = threadIdx.x & 31, i = lane >> 1, part = lane & 1;
+  unsigned char* kd = tile + i * 256;
+  unsigned char* vd = tile + 4096 + i * 256;
+  if (ok) {
 #pragma unroll
-      for (int e = 1; e < 4; ++e) a = __ffma2_rn(q[h][e], k[e], a);
-      d[r * G + h] = a.x + a.y;
+    for (int u = 0; u < 8; ++u) {
+      const int c = 2 * u + part;
+      cp_async16(kd + ((c ^ (i & 7)) << 4), krow + c * 8);
+      cp_async16(vd + ((c ^ (i & 7)) << 4), vrow + c * 8);
     }
-  }
-  halving_reduce<V>(d, hl);
-  // lane hl holds the logit of value index (r, h) = (hl * V / 16) split as r * G + h
-  constexpr int kShift = (V == 16) ? 0 : (V == 8 ? 1 : (V == 4 ? 2 : (V == 2 ? 3 : 4)));
-  const int vi = hl >> kShift;
-  const int my_r = vi / G, my_h = vi % G;
-  uint32_t my_mask = 0;
+  } else {
 #pragma unroll
-  for (int r = 0; r < R; ++r) my_mask = (r == my_r) ? mask[r] : my_mask;
-  const float logit = ((my_mask >> my_h) & 1u) ? d[0] : -INFINITY;
-  // block max per head over the R rows: lanes holding the same head differ in the row bits
-  float bm = logit;
-#pragma unroll
-  for (int o = 1; o < R; o <<= 1) {
-    const int lanebit = (o * G) << kShift;
-    bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, lanebit));
-  }
-  float mnew_my = -INFINITY;
-#pragma unroll
-  for (int h = 0; h < G; ++h) mnew_my = (h == my_h) ? fmaxf(st.m[h], bm) : mnew_my;
-  const float p_my = (logit == -INFINITY) ? 0.f : exp2f(logit - mnew_my);
-  // broadcast: every lane gets p of each (r, h) and the block max of each head
-  const int base = (threadIdx.x & 31) & 16;
-#pragma unroll
-  for (int h = 0; h < G; ++h) {
-    const float bmh = __shfl_sync(0xffffffffu, bm, base + (h << kShift));
-    if (bmh > st.m[h]) {                       // the running max moved: rescale the state
-      const float scale = exp2f(st.m[h] - bmh);  // 0 when the state was empty (m = -inf)
-      st.m[h] = bmh;
-      st.l[h] *= scale;
-      const float2 sc2 = make_float2(scale, scale);
-#pragma unroll
-      for (int e = 0; e < 4; ++e) st.a2[h][e] = __fmul2_rn(st.a2[h][e], sc2);
-    }
-  }
-#pragma unroll
-  for (int r = 0; r < R; ++r) {
-    float2 v[4];
-    unpack_pairs(vw[r], v);
-#pragma unroll
-    for (int h = 0; h < G; ++h) {
-      const float p = __shfl_sync(0xffffffffu, p_my, base + ((r * G + h) << kShift));
-      st.l[h] += p;
-      const float2 p2 = make_float2(p, p);
-#pragma unroll
-      for (int e = 0; e < 4; ++e) st.a2[h][e] = __ffma2_rn(p2, v[e], st.a2[h][e]);
+    for (int u = 0; u < 8; ++u) {
+      const int c = 2 * u + part;
+      *reinterpret_cast<uint4*>(vd + ((c ^ (i & 7)) << 4)) = make_uint4(0, 0, 0, 0);
     }
   }
 }
 
-// Attention of the G heads over rows [0, cnt), row i given by rowfn(i, kp, vp, mask).
-// stage: AttnCfg<G>::stage_bytes(nthreads) bytes of shared memory. Leaves the half-warp
-// states in st (merge with attend_merge).
+// One staged tile: nrows valid rows; mask_row: this lane's row (lane / 2) head mask.
+template <int G>
+__device__ __forceinline__ void tile_attend(WarpAttn& W, const unsigned char* tile, int nrows,
+                                            uint32_t mask_row) {
+  const int lane = threadIdx.x & 31, gid = lane >> 2, tig = lane & 3;
+  const uint32_t tk = smem_u32(tile), tv = tk + 4096;
+  float s[4] = {0.f, 0.f, 0.f, 0.f};
+  {
+    const int r = (lane & 7) + ((lane >> 3) & 1) * 8;     // K row for this lane's address
+    const int chi = lane >> 4;
+    // query matrices: lane l addresses head l & 7 of matrix l >> 3 (hi: chunk 2kk, 2kk+1;
+    // lo: the same chunks 2048 bytes on)
+    const int qh = lane & 7, qm = lane >> 3;
+    const uint32_t qrow = W.qb + (qm >> 1) * 2048 + qh * 256;
+#pragma unroll
+    for (int kk = 0; kk < 8; ++kk) {
+      uint32_t a[4], b[4];
+      ldsm_x4(qrow + (((2 * kk + (qm & 1)) ^ qh) << 4), b);
+      ldsm_x4(tk + r * 256 + (((2 * kk + chi) ^ (r & 7)) << 4), a);
+      mma_bf16(s, a, b[0], b[1]);
+      mma_bf16(s, a, b[2], b[3]);
+    }
+  }
+  // masks of rows gid and gid + 8 (held by lanes 2 gid and 2 gid + 16)
+  const uint32_t mk0 = __shfl_sync(0xffffffffu, mask_row, 2 * gid);
+  const uint32_t mk1 = __shfl_sync(0xffffffffu, mask_row, 2 * gid + 16);
+  const int h0 = 2 * tig;
+  const bool r0 = gid < nrows, r1 = gid + 8 < nrows;
+  float x[4];
+  x[0] = (r0 && ((mk0 >> h0) & 1u)) ? s[0] : -INFINITY;
+  x[1] = (r0 && ((mk0 >> (h0 + 1)) & 1u)) ? s[1] : -INFINITY;
+  x[2] = (r1 && ((mk1 >> h0) & 1u)) ? s[2] : -INFINITY;
+  x[3] = (r1 && ((mk1 >> (h0 + 1)) & 1u)) ? s[3] : -INFINITY;
+  float mx0 = fmaxf(x[0], x[2]), mx1 = fmaxf(x[1], x[3]);
+#pragma unroll
+  for (int o = 4; o < 32; o <<= 1) {
+    mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, o));
+    mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, o));
+  }
+  const float mn0 = fmaxf(W.m[0], mx0), mn1 = fmaxf(W.m[1], mx1);
+  const float al0 = mn0 == -INFINITY ? 1.f : exp2f(W.m[0] - mn0);
+  const float al1 = mn1 == -INFINITY ? 1.f : exp2f(W.m[1] - mn1);
+  float p[4];
+  p[0] = x[0] == -INFINITY ? 0.f : exp2f(x[0] - mn0);
+  p[1] = x[1] == -INFINITY ? 0.f : exp2f(x[1] - mn1);
+  p[2] = x[2] == -INFINITY ? 0.f : exp2f(x[2] - mn0);
+  p[3] = x[3] == -INFINITY ? 0.f : exp2f(x[3] - mn1);
+  W.l[0] = W.l[0] * al0 + (p[0] + p[2]);
+  W.l[1] = W.l[1] * al1 + (p[1] + p[3]);
+  W.m[0] = mn0;
+  W.m[1] = mn1;
+  if (__any_sync(0xffffffffu, al0 != 1.f || al1 != 1.f)) {
+#pragma unroll
+    for (int mt = 0; mt < 8; ++mt) {
+      W.acc[mt][0] *= al0; W.acc[mt][1] *= al1;
+      W.acc[mt][2] *= al0; W.acc[mt][3] *= al1;
+    }
+  }
+  uint32_t h01, l01, h23, l23;
+  split_bf2(p[0], p[1], h01, l01);
+  split_bf2(p[2], p[3], h23, l23);
+  const uint32_t bh0 = movm_t(h01), bh1 = movm_t(h23);
+  const uint32_t bl0 = movm_t(l01), bl1 = movm_t(l23);
+  {
+    const int j = lane >> 3;
+    const int r = (lane & 7) + (j >> 1) * 8;             // V row for this lane's address
+#pragma unroll
+    for (int mt = 0; mt < 8; ++mt) {
+      uint32_t a[4];
+      ldsm_x4_t(tv + r * 256 + (((2 * mt + (j & 1)) ^ (r & 7)) << 4), a);
+      mma_bf16(W.acc[mt], a, bh0, bh1);
+      mma_bf16(W.acc[mt], a, bl0, bl1);
+    }
+  }
+}
+
+// Attention of the G heads over a row list, in three steps so a caller can feed the rows
+// in batches: attn_begin (state from the query), attn_tiles (rows [0, cnt) of one batch,
+// rowfn(i, kp, vp, mask) gives row i), attn_end (merge of the warps' states). Warps
+// [0, nwa) take tiles w, w + nwa, ... with one tile buffer each at stage + w * kTileBytes.
+template <int G>
+__device__ __forceinline__ void attn_begin(WarpAttn& W, unsigned char* qbuf, const float* q_s,
+                                           int nthreads) {
+  fill_qbuf<G>(qbuf, q_s, nthreads);
+  warp_attn_init(W, qbuf);
+}
+
 template <int G, class RowFn>
-__device__ __forceinline__ void attend_rows(AttnState<G>& st, const float2 (&q)[G][4], int cnt,
-                                            RowFn rowfn, unsigned char* stage, int nthreads) {
-  constexpr int R = AttnCfg<G>::kRows;
-  const int t = threadIdx.x, lane = t & 31, warp = t >> 5, hl = lane & 15, hw = t >> 4;
-  const int nhw = nthreads >> 4;
-  const int step = (nthreads >> 5) * 2 * R;                  // rows per CTA step
-  // this half-warp's slot: stage s, row r -> stage + ((s * nhw + hw) * R + r) * 512
-  auto slot = [&](int s, int r) -> unsigned char* {
-    return stage + ((size_t)(s * nhw + hw) * R + r) * 512;
-  };
-  uint32_t mask_cur[R], mask_nxt[R];
-  auto issue = [&](int wb, int s, uint32_t (&mk)[R]) {
-#pragma unroll
-    for (int r = 0; r < R; ++r) {
-      const int i = wb + (lane >> 4) * R + r;
-      const uint16_t* kp = nullptr;
-      const uint16_t* vp = nullptr;
-      mk[r] = 0;
-      if (i < cnt) rowfn(i, kp, vp, mk[r]);
-      if (mk[r]) {
-        cp_async16(slot(s, r) + hl * 16, kp + hl * 8);
-        cp_async16(slot(s, r) + 256 + hl * 16, vp + hl * 8);
-      }
-    }
-    cp_async_commit();
-  };
-  int wb = warp * 2 * R;
-  int s = 0;
-  if (wb < cnt) issue(wb, 0, mask_cur);
+__device__ __forceinline__ void attn_tiles(WarpAttn& W, int cnt, RowFn rowfn,
+                                           unsigned char* stage, int nwa) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  if (warp >= nwa) return;
+  unsigned char* tile = stage + warp * kTileBytes;
+  const int i = lane >> 1;
 #pragma unroll 1
-  for (; wb < cnt; wb += step, s ^= 1) {
-    if (wb + step < cnt) issue(wb + step, s ^ 1, mask_nxt);
-    else cp_async_commit();                                   // keep one group per step
-    cp_async_wait<1>();
-    uint4 kw[R], vw[R];
-#pragma unroll
-    for (int r = 0; r < R; ++r) {
-      if (mask_cur[r]) {
-        kw[r] = *reinterpret_cast<const uint4*>(slot(s, r) + hl * 16);
-        vw[r] = *reinterpret_cast<const uint4*>(slot(s, r) + 256 + hl * 16);
-      } else {
-        kw[r] = make_uint4(0, 0, 0, 0);
-        vw[r] = make_uint4(0, 0, 0, 0);
-      }
-    }
-    attend_step<G>(st, q, kw, vw, mask_cur, hl);
-#pragma unroll
-    for (int r = 0; r < R; ++r) mask_cur[r] = mask_nxt[r];
+  for (int t0 = warp * kTileRows; t0 < cnt; t0 += nwa * kTileRows) {
+    const int nrows = min(kTileRows, cnt - t0);
+    const uint16_t* kp = nullptr;
+    const uint16_t* vp = nullptr;
+    uint32_t mk = 0;
+    if (i < nrows) rowfn(t0 + i, kp, vp, mk);
+    tile_copy(tile, kp, vp, i < nrows && mk != 0);
+    cp_async_commit();
+    cp_async_wait<0>();
+    __syncwarp();
+    tile_attend<G>(W, tile, nrows, mk);
+    __syncwarp();                         // the tile is rewritten by the next copy
   }
-  cp_async_wait<0>();
 }
 
-// Merges the per-half-warp states of a CTA of nthreads threads into res[G][2 + 128]
-// (M, L, A). scratch: >= (nthreads / 32) * G * 128 + 2 * (nthreads / 32) * G floats.
+// Merges the warps' states into res[G][2 + 128] (M, L, A) through scratch (>= 16 *
+// G * (kAccStride + 2) floats; may alias the tile buffers). Every thread of the CTA calls it.
 template <int G>
-__device__ __forceinline__ void attend_merge(AttnState<G>& st, float* scratch, float* res,
-                                             int nthreads) {
-  const int t = threadIdx.x, lane = t & 31, warp = t >> 5, hl = lane & 15;
+__device__ __forceinline__ void attn_end(WarpAttn& W, int nwa, float* res, float* scratch,
+                                         int nthreads) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int nw = nthreads >> 5;
-  // merge the two half-warps of each warp with shuffles
+  const bool active = warp < nwa;
+  if (active) {
+    // a thread's sum covered its own rows: reduce over the 8 row groups
 #pragma unroll
-  for (int h = 0; h < G; ++h) {
-    const float mo = __shfl_xor_sync(0xffffffffu, st.m[h], 16);
-    const float lo = __shfl_xor_sync(0xffffffffu, st.l[h], 16);
-    const float mn = fmaxf(st.m[h], mo);
-    const float fa = (mn == -INFINITY) ? 0.f : exp2f(st.m[h] - mn);
-    const float fb = (mn == -INFINITY) ? 0.f : exp2f(mo - mn);
-    st.l[h] = st.l[h] * fa + lo * fb;
-#pragma unroll
-    for (int e = 0; e < 8; ++e) {
-      const float ao = __shfl_xor_sync(0xffffffffu, st.acc(h, e), 16);
-      st.acc(h, e) = st.acc(h, e) * fa + ao * fb;
+    for (int o = 4; o < 32; o <<= 1) {
+      W.l[0] += __shfl_xor_sync(0xffffffffu, W.l[0], o);
+      W.l[1] += __shfl_xor_sync(0xffffffffu, W.l[1], o);
     }
-    st.m[h] = mn;
   }
-  __syncthreads();                                // scratch may alias the staging buffer
-  float* sm_m = scratch + nw * G * kD;
-  float* sm_l = sm_m + nw * G;
-  if (lane < 16) {
+  __syncthreads();                        // scratch may alias the tile buffers
+  float* sm_ml = scratch + nw * G * kAccStride;           // [nw][G][2]
+  if (active) {
+    const int gid = lane >> 2, tig = lane & 3;
 #pragma unroll
-    for (int h = 0; h < G; ++h)
+    for (int e = 0; e < 2; ++e) {
+      const int h = 2 * tig + e;
+      if (h < G) {
+        float* a = scratch + (warp * G + h) * kAccStride;
 #pragma unroll
-      for (int e = 0; e < 8; ++e) scratch[(warp * G + h) * kD + hl * 8 + e] = st.acc(h, e);
-    if (hl == 0) {
-#pragma unroll
-      for (int h = 0; h < G; ++h) { sm_m[warp * G + h] = st.m[h]; sm_l[warp * G + h] = st.l[h]; }
+        for (int mt = 0; mt < 8; ++mt) {
+          a[mt * 16 + gid] = W.acc[mt][e];
+          a[mt * 16 + gid + 8] = W.acc[mt][2 + e];
+        }
+        if (gid == 0) {
+          sm_ml[(warp * G + h) * 2 + 0] = W.m[e];
+          sm_ml[(warp * G + h) * 2 + 1] = W.l[e];
+        }
+      }
     }
   }
   __syncthreads();
-#pragma unroll 1
-  for (int o = t; o < G * kD; o += nthreads) {
-    const int h = o / kD, dch = o % kD;
+  for (int o = threadIdx.x; o < G * kD; o += nthreads) {
+    const int h = o / kD, c = o % kD;
     float M = -INFINITY;
-#pragma unroll 1
-    for (int w = 0; w < nw; ++w) M = fmaxf(M, sm_m[w * G + h]);
-    float Ls = 0.f, A = 0.f;
+    for (int w = 0; w < nwa; ++w) M = fmaxf(M, sm_ml[(w * G + h) * 2]);
+    float L = 0.f, A = 0.f;
     if (M != -INFINITY) {
-#pragma unroll 1
-      for (int w = 0; w < nw; ++w) {
-        const float f = exp2f(sm_m[w * G + h] - M);
-        Ls += sm_l[w * G + h] * f;
-        A += scratch[(w * G + h) * kD + dch] * f;
+      for (int w = 0; w < nwa; ++w) {
+        const float f = exp2f(sm_ml[(w * G + h) * 2] - M);   // 0 for a warp without rows
+        L += sm_ml[(w * G + h) * 2 + 1] * f;
+        A += scratch[(w * G + h) * kAccStride + c] * f;
       }
     }
-    res[h * (kD + 2) + 2 + dch] = A;
-    if (dch == 0) { res[h * (kD + 2)] = M; res[h * (kD + 2) + 1] = Ls; }
+    res[h * (kD + 2) + 2 + c] = A;
+    if (c == 0) { res[h * (kD + 2)] = M; res[h * (kD + 2) + 1] = L; }
   }
   __syncthreads();
 }
@@ -275,9 +311,7 @@ constexpr int kMaxMerge = 64;
 // other CTAs) into `dst` (same format) or, when out_rows is given, into the bf16 output rows
 // of the G heads. The partials are first copied into shared memory (buf, buf_bytes) with
 // cp.async, as many per batch as fit, so all loads of a batch are in flight together; each
-// thread then folds its output channels over the batch with the online softmax rule. The
-// code is kept small on purpose: it runs once per group at the end of a step, when the
-// instruction cache does not hold it.
+// thread then folds its output channels over the batch with the online softmax rule.
 template <int G>
 __device__ __forceinline__ void merge_partials(const float* parts, int n, float* dst,
                                                uint16_t* out_rows, float* buf, int buf_bytes,

@@ -132,3 +132,15 @@ def rtp_read_device_status(ws, stream=None) -> int:
 
 def rtp_last_launch_count() -> int:
     return int(_lib.load().rtp_last_launch_count())
+
+
+def rtp_debug_set_wait_limit(cycles: int):
+    """Test hook: limit (SM cycles) of every device-side wait of later decode launches;
+    0 restores the default (about one second)."""
+    return _check("rtp_debug_set_wait_limit", _lib.load().rtp_debug_set_wait_limit(int(cycles)))
+
+
+def rtp_debug_fail_next_call(status: int):
+    """Test hook: the next append / decode entry-point call returns ``status`` (a negative
+    RTP_E* code) without enqueueing anything; 0 cancels."""
+    return _check("rtp_debug_fail_next_call", _lib.load().rtp_debug_fail_next_call(int(status)))

@@ -215,11 +215,9 @@ class HeadResult:
     sel: np.ndarray | None     # ascending selected positions (retrieval)
     selection: Selection | None
     scores: np.ndarray | None
-    exact: np.ndarray | None   # exact sorted top-p mask (diagnostic)
 
 
-def retrieval_head(q_pre, w_qidx_h, k_pre, v, w_kidx_g, p: float, base: float = 1e6,
-                   with_exact: bool = False) -> HeadResult:
+def retrieval_head(q_pre, w_qidx_h, k_pre, v, w_kidx_g, p: float, base: float = 1e6) -> HeadResult:
     """One retrieval query head at decode position m = N - 1 ([P] §3.2 eq. (4)-(5)).
 
     k_pre, v: [N][d] pre-RoPE keys and values of the head's KV head (bf16 values as float64).
@@ -233,8 +231,7 @@ def retrieval_head(q_pre, w_qidx_h, k_pre, v, w_kidx_g, p: float, base: float = 
     K = bf16_round(rope_rotate(k_pre[idx], idx, base))
     q = rope_rotate(q_pre, N - 1, base)
     out = attend(q, K, np.asarray(v, np.float64)[idx])
-    ex = topp_exact(s, p) if with_exact else None
-    return HeadResult(out, int(idx.size), idx, sel, s, ex)
+    return HeadResult(out, int(idx.size), idx, sel, s)
 
 
 def local_head(q_pre, k_pre, v, sinks: int, window: int, base: float = 1e6) -> HeadResult:
@@ -245,12 +242,15 @@ def local_head(q_pre, k_pre, v, sinks: int, window: int, base: float = 1e6) -> H
     K = bf16_round(rope_rotate(k_pre[pos], pos, base))
     q = rope_rotate(q_pre, N - 1, base)
     out = attend(q, K, np.asarray(v, np.float64)[pos])
-    return HeadResult(out, int(pos.size), pos, None, None, None)
+    return HeadResult(out, int(pos.size), pos, None, None)
 
 
 def full_attention_mass(q_pre, k_pre, sel_positions, base: float = 1e6) -> float:
-    """Share of the dense softmax(q^T k / sqrt(d)) mass over all N tokens that falls on the
-    selected positions (the retained-mass diagnostic of the paper's notes)."""
+    """Retained mass of a selected set: the share of the dense attention weights
+    softmax(q^T k_n / sqrt(d)) over all N cached tokens (RoPE'd, bf16-stored keys; query at
+    position N - 1) that falls on ``sel_positions``. [DR] "Key Results" reports this share
+    (above 0.93 at 89.2 % sparsity) for the sets the selector keeps; [P] §2.3 compares top-k
+    and top-p sets by the same quantity."""
     k_pre = np.asarray(k_pre, np.float64)
     N = k_pre.shape[0]
     K = bf16_round(rope_rotate(k_pre, np.arange(N), base))
@@ -261,7 +261,7 @@ def full_attention_mass(q_pre, k_pre, sel_positions, base: float = 1e6) -> float
 
 
 def decode_layer(q_pre, w_qidx, w_kidx, k_pre, v, ret_mask, seq_lens, p: float, sinks: int,
-                 window: int, base: float = 1e6, heads=None, with_exact: bool = False):
+                 window: int, base: float = 1e6, heads=None):
     """Whole decode layer over a batch ([P] §3.2): retrieval query heads use eq. (4)-(5),
     local query heads use sinks + window. Query head h reads KV head h // G (GQA).
 
@@ -280,8 +280,7 @@ def decode_layer(q_pre, w_qidx, w_kidx, k_pre, v, ret_mask, seq_lens, p: float, 
         kp = np.asarray(k_pre(b, g), np.float64)[:N]
         vv = np.asarray(v(b, g), np.float64)[:N]
         if ret_mask[g]:
-            res[(b, h)] = retrieval_head(q_pre[b][h], w_qidx[h], kp, vv, w_kidx[g], p, base,
-                                         with_exact)
+            res[(b, h)] = retrieval_head(q_pre[b][h], w_qidx[h], kp, vv, w_kidx[g], p, base)
         else:
             res[(b, h)] = local_head(q_pre[b][h], kp, vv, sinks, window, base)
     return res

@@ -141,3 +141,41 @@ def test_missing_library_fails_loudly(tmp_path):
             _lib.load(str(tmp_path / "nope.so"))
         finally:
             _lib._lib = None
+
+
+def test_injected_failure_returns_before_any_launch():
+    """rtp_debug_fail_next_call: the next entry-point call returns the injected status before
+    looking at its arguments (so nothing reaches a device), once; then calls behave again."""
+    d = _desc()
+    lib = _lib.load()
+    cache = rtp.make_cache(0x1000, 0x1000, 0x1000, 0x1000, 0x1000, 0x1000, 0x1000, 65536)
+    append = lambda: lib.rtp_append_kv(d.ref, ctypes.byref(cache), 0x1000, 0x1000, 0x1000, 0x1000,
+                                       None, 0, None, None)
+    assert append() == _lib.RTP_OK                                  # n_new = 0: nothing to do
+    rtp.rtp_debug_fail_next_call(_lib.RTP_ECUDA)
+    assert append() == _lib.RTP_ECUDA
+    assert append() == _lib.RTP_OK                                  # consumed by one call
+    # decode: the injected code comes before the argument checks (null q_pre would be EINVAL)
+    rtp.rtp_debug_fail_next_call(_lib.RTP_ETIMEOUT)
+    rc = lib.rtp_decode_step(d.ref, ctypes.byref(cache), None, 0x1000, 0x1000, 0.9, 0x1000,
+                             0x1000, None, 0, 0x1000, 1 << 30, None)
+    assert rc == _lib.RTP_ETIMEOUT
+    rc = lib.rtp_decode_step(d.ref, ctypes.byref(cache), None, 0x1000, 0x1000, 0.9, 0x1000,
+                             0x1000, None, 0, 0x1000, 1 << 30, None)
+    assert rc == _lib.RTP_EINVAL
+    rtp.rtp_debug_fail_next_call(_lib.RTP_EDEVICE)
+    rc = lib.rtp_decode_step_static(d.ref, ctypes.byref(cache), 0x1000, 0x1000, 0x1000, 0.9,
+                                    0x1000, 0x1000, None)
+    assert rc == _lib.RTP_EDEVICE
+    rtp.rtp_debug_fail_next_call(_lib.RTP_EWORKSPACE)
+    rtp.rtp_debug_fail_next_call(0)                                 # cancelled
+    assert append() == _lib.RTP_OK
+    for bad in (1, -7):
+        assert lib.rtp_debug_fail_next_call(bad) == _lib.RTP_EINVAL
+
+
+def test_wait_limit_hook_validates():
+    lib = _lib.load()
+    assert lib.rtp_debug_set_wait_limit(-1) == _lib.RTP_EINVAL
+    assert lib.rtp_debug_set_wait_limit(5000) == _lib.RTP_OK
+    assert lib.rtp_debug_set_wait_limit(0) == _lib.RTP_OK            # default restored

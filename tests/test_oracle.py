@@ -390,3 +390,50 @@ def test_decode_layer_bruteforce_tiny(seed):
             assert r.count == len(sel)
             assert list(r.sel) == sel
             np.testing.assert_allclose(r.out, out, rtol=0, atol=1e-12)
+
+
+# ----------------------------------------------------------------------------- retained mass
+def _mass_case(seed, N):
+    rng = np.random.default_rng(300 + seed)
+    q = O.bf16_round(rng.standard_normal(128) * 2.0)
+    kp = O.bf16_round(rng.standard_normal((N, 128)))
+    return rng, q, kp
+
+
+def test_full_attention_mass_of_every_position_is_one():
+    _, q, kp = _mass_case(0, 500)
+    assert abs(O.full_attention_mass(q, kp, np.arange(500)) - 1.0) < 1e-14
+    assert O.full_attention_mass(q, kp, np.array([], np.int64)) == 0.0
+
+
+def test_full_attention_mass_matches_torch_softmax_weights():
+    """The dense attention weights from torch's softmax over the complex-RoPE'd, bf16-stored
+    keys, summed over the subset (and its complement summing to the rest)."""
+    rng, q, kp = _mass_case(1, 700)
+    N = 700
+    K = O.bf16_round(_rope_complex(kp, np.arange(N)))
+    qr = _rope_complex(q, N - 1)
+    wts = torch.softmax(torch.from_numpy(K) @ torch.from_numpy(qr) / math.sqrt(128), dim=0).numpy()
+    sub = np.sort(rng.choice(N, size=90, replace=False))
+    rest = np.setdiff1d(np.arange(N), sub)
+    got = O.full_attention_mass(q, kp, sub)
+    assert abs(got - wts[sub].sum()) < 1e-12
+    assert abs(got + O.full_attention_mass(q, kp, rest) - 1.0) < 1e-12
+
+
+@pytest.mark.parametrize("N", [1, 5, 33, 64])
+def test_full_attention_mass_bruteforce_tiny(N):
+    """Loop-by-loop evaluation of the definition: keys rotated by their own positions and
+    stored in bf16, the query rotated by N - 1, weights exp(q.k / sqrt(128)) normalised over
+    all N tokens, summed over the subset."""
+    rng, q, kp = _mass_case(2 + N, N)
+    sub = sorted(set(int(x) for x in rng.integers(0, N, size=max(1, N // 3))))
+    qr = _bf_rope(q.tolist(), N - 1)
+    z = []
+    for n in range(N):
+        k = [float(x) for x in O.bf16_round(np.array(_bf_rope(kp[n].tolist(), n)))]
+        z.append(sum(qr[d] * k[d] for d in range(128)) / math.sqrt(128))
+    zmax = max(z)
+    w = [math.exp(x - zmax) for x in z]
+    ref = sum(w[n] for n in sub) / sum(w)
+    assert abs(O.full_attention_mass(q, kp, np.array(sub)) - ref) < 1e-12
