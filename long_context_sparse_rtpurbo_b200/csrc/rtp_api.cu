@@ -18,7 +18,6 @@ namespace {
 thread_local int32_t g_launches = 0;
 
 constexpr int kPlanCTAs = 160;      // upper bound on decode CTAs (one per SM; B200 has 148)
-constexpr int kLocRows = 256;       // ring rows per local attention item
 constexpr long long kSpinLimitDefault = 2000000000LL;   // ~1 s of SM clock per device wait
 
 // Test hooks (see include/rtp.h): the device-wait limit of later launches, and an error code
@@ -33,12 +32,12 @@ inline int align16(int x) { return (x + 15) & ~15; }
 
 struct Plan {
   LayerShape L;
-  int C_min, max_nch, NC_max, n_groups, n_lgroups, RL, PL, n_loc_items;
+  int C_min, max_nch, NC_max, n_groups, n_lgroups, n_loc_items;
   int64_t cand_stride;
   size_t off_ctrl, ctrl_bytes;
   size_t off_bar, off_team, off_locarr, off_misc, off_hist, off_hcnt;
-  size_t off_bstar, off_cstat, off_ccnt, off_cpos, off_cbin, off_part, off_tpart, off_lpart,
-      off_trace, total;
+  size_t off_bstar, off_cstat, off_bands, off_ccnt, off_cpos, off_cbin, off_part, off_tpart,
+      off_lpart, off_trace, total;
 };
 
 int check_desc(const rtp_layer_desc* d, LayerShape& L) {
@@ -98,21 +97,10 @@ int make_plan(const rtp_layer_desc* d, Plan& pl) {
                                      int64_t(kMaxSteps) * kPlanCTAs + pl.n_groups);
   pl.NC_max = std::max(pl.NC_max, 1);
   pl.cand_stride = (maxN + 63) / 64 * 64;
+  // local items: at least 64 ring rows each (the split itself depends on the SM count and
+  // is made at launch, see local_split)
   const int64_t loc_rows = std::min<int64_t>(maxN, L.ring);
-  // ring rows per local item: about kLocRows, in whole tiles; in a layer without retrieval
-  // heads the local items are the whole launch, so they are cut to about one per CTA
-  int64_t pl_n = (loc_rows + kLocRows - 1) / kLocRows;
-  if (L.n_ret == 0) {
-    const int64_t per_cta = (int64_t(pl.n_lgroups) * loc_rows + kPlanCTAs - 1) / kPlanCTAs;
-    const int64_t rl = std::max<int64_t>(64, (per_cta + 15) / 16 * 16);
-    pl_n = std::max<int64_t>(pl_n, (loc_rows + rl - 1) / rl);
-  }
-  pl_n = std::max<int64_t>(pl_n, 1);
-  int64_t rl = (loc_rows + pl_n - 1) / pl_n;
-  rl = (rl + 15) / 16 * 16;
-  pl.RL = (int)rl;
-  pl.PL = (int)((loc_rows + rl - 1) / rl);
-  pl.n_loc_items = pl.n_lgroups * pl.PL;
+  pl.n_loc_items = (int)(int64_t(pl.n_lgroups) * ((loc_rows + 63) / 64));
   const size_t part_bytes = sizeof(float) * G * (kD + 2);
   size_t o = 256;                                   // [0, 256): status word
   pl.off_ctrl = o;
@@ -125,6 +113,7 @@ int make_plan(const rtp_layer_desc* d, Plan& pl) {
   pl.ctrl_bytes = o - pl.off_ctrl;
   pl.off_bstar = o;  o = align256(o + sizeof(int32_t) * pl.n_groups * G);
   pl.off_cstat = o;  o = align256(o + 16 * size_t(pl.n_groups) * pl.max_nch * G);
+  pl.off_bands = o;  o = align256(o + 4 * size_t(pl.n_groups) * pl.max_nch * G * kBandRec);
   pl.off_ccnt = o;   o = align256(o + sizeof(uint32_t) * size_t(pl.n_groups) * pl.max_nch);
   pl.off_cpos = o;   o = align256(o + sizeof(uint32_t) * size_t(pl.n_groups) * pl.cand_stride);
   pl.off_cbin = o;   o = align256(o + 8 * size_t(pl.n_groups) * pl.cand_stride);
@@ -166,9 +155,24 @@ int dev_info(DevInfo& di) {
   return RTP_OK;
 }
 
-// Shared-memory layout of the decode kernel: the staging region, the score slot right after
-// it (the two form the free region once the slot is dead), then the small arrays. Returns the
-// bytes, sets C_cap.
+// Ring rows per local item (RL, a multiple of the 16-row tile, at least 64) and items per
+// local group (PL): about 256 rows per item; in a layer without retrieval heads the items
+// are the whole launch, so they are cut to about one per CTA.
+void local_split(const LayerShape& L, int n_lgroups, int n_ret, int P, int& PL, int& RL) {
+  const int64_t rows = std::min<int64_t>(L.maxN, L.ring);
+  int64_t pl = (rows + 255) / 256;
+  if (n_ret == 0 && n_lgroups > 0) pl = std::max<int64_t>(pl, P / n_lgroups);
+  pl = std::max<int64_t>(pl, 1);
+  int64_t rl = (rows + pl - 1) / pl;
+  rl = std::max<int64_t>(64, (rl + 15) / 16 * 16);
+  RL = (int)rl;
+  PL = (int)((rows + rl - 1) / rl);
+}
+
+// Shared-memory layout of the decode kernel: the staging region (index ring, tiles, merge
+// buffers, gather lists), then the small arrays. The kept scores of a CTA's last chunk live in
+// tensor memory (C_cap rows). Returns the bytes, or -1 when the staging region would be too
+// small for the index ring.
 int smem_layout(DecodeParams& P, const Plan& pl, int smem_optin) {
   const int G = P.L.G;
   int small = 0;
@@ -178,18 +182,17 @@ int smem_layout(DecodeParams& P, const Plan& pl, int smem_optin) {
   small += align16(8 * G * kHistStride);                // hist (two 32-bit words per bin)
   small += align16(4 * G * (kD + 2));                   // res
   small += align16(8 * kFThreads);                      // tmp
-  small += align16(4 * 64);                             // ints
+  small += align16(4 * 128);                            // ints
   small += align16(4 * P.L.B);                          // N
   small += align16(4 * (pl.n_groups + 1));              // cbase
   small += align16(8 * kMaxSteps * G);                  // tcache
+  small += align16(4 * G * kBandN * 32);                // mass bands, one word per lane
   const int budget = smem_optin - 1024;
-  int cap = (budget - kStageBytes - small) / (4 * G) - kHeadPad;
-  cap = std::min(cap, 16384) / 64 * 64;
-  if (cap < 512) return -1;
-  P.C_cap = cap;
+  const int stage = (budget - small) / 1024 * 1024;
+  if (stage < DecodeCta<1>::kSRows * 32 * DecodeCta<1>::kSStages) return -1;
+  P.C_cap = kTmemColsPerThread / G * DecodeCta<1>::kSRows;
   int o = 0;
-  P.sm_stage = o; o += kStageBytes;
-  P.sm_slot = o;  o += 4 * G * (cap + kHeadPad);
+  P.sm_stage = o; o += stage;
   P.free_bytes = o;
   P.sm_q = o;     o += align16(4 * G * kD);
   P.sm_qbuf = o;  o += kQBytes;
@@ -197,10 +200,11 @@ int smem_layout(DecodeParams& P, const Plan& pl, int smem_optin) {
   P.sm_hist = o;  o += align16(8 * G * kHistStride);
   P.sm_res = o;   o += align16(4 * G * (kD + 2));
   P.sm_tmp = o;   o += align16(8 * kFThreads);
-  P.sm_int = o;   o += align16(4 * 64);
+  P.sm_int = o;   o += align16(4 * 128);
   P.sm_N = o;     o += align16(4 * P.L.B);
   P.sm_cbase = o; o += align16(4 * (pl.n_groups + 1));
   P.sm_tcache = o; o += align16(8 * kMaxSteps * G);
+  P.sm_band = o;  o += align16(4 * G * kBandN * 32);
   return o;
 }
 
@@ -240,6 +244,9 @@ int launch_decode(DecodeParams& P, const Plan& pl, const DevInfo& di, cudaStream
     return RTP_ECUDA;
   P.P = std::min(di.sms, kPlanCTAs);
   if (pl.n_groups >= kMaxSteps * P.P) return RTP_ESHAPE;
+  // every chunk stays within kMaxChunk rows at kMaxSteps chunks per CTA
+  if (double(pl.n_groups) * double(P.L.maxN) > double(kMaxSteps) * P.P * kMaxChunk * 0.9)
+    return RTP_ESHAPE;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(P.P);
   cfg.blockDim = dim3(kFThreads);
@@ -385,8 +392,9 @@ int decode_impl(const rtp_layer_desc* desc, const rtp_cache* cache, const uint16
   P.L = L;
   P.L.T_total = cache->T_total;
   P.C_min = pl.C_min; P.max_nch = pl.max_nch; P.NC_max = pl.NC_max;
-  P.n_groups = pl.n_groups; P.n_lgroups = pl.n_lgroups; P.PL = pl.PL; P.RL = pl.RL;
-  P.n_loc_items = pl.n_loc_items;
+  P.n_groups = pl.n_groups; P.n_lgroups = pl.n_lgroups;
+  local_split(L, pl.n_lgroups, L.n_ret, std::min(di.sms, kPlanCTAs), P.PL, P.RL);
+  P.n_loc_items = pl.n_lgroups * P.PL;          // <= pl.n_loc_items (RL >= 64)
   P.select_all = p >= 1.0 ? 1 : 0;
   P.p = p;
   P.spin_limit = g_spin_limit.load();
@@ -405,6 +413,7 @@ int decode_impl(const rtp_layer_desc* desc, const rtp_cache* cache, const uint16
   P.hcnt = at<int32_t>(ws, pl.off_hcnt);
   P.bstar = at<int32_t>(ws, pl.off_bstar);
   P.cstat = at<float4>(ws, pl.off_cstat);
+  P.bands = at<float>(ws, pl.off_bands);
   P.ccnt = at<uint32_t>(ws, pl.off_ccnt);
   P.cpos = at<uint32_t>(ws, pl.off_cpos);
   P.cbin = at<uint2>(ws, pl.off_cbin);

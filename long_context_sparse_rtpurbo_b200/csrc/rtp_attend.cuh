@@ -225,9 +225,27 @@ __device__ __forceinline__ void attn_begin(WarpAttn& W, unsigned char* qbuf, con
   warp_attn_init(W, qbuf);
 }
 
+// Issues the copy of each warp's first tile (rows warp * 16 ...), so the loads are in flight
+// while the caller prepares the query; attn_tiles(..., first_issued = true) then uses them.
+template <class RowFn>
+__device__ __forceinline__ void attn_first_copy(int cnt, const RowFn& rowfn, unsigned char* stage,
+                                                int nwa) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int t0 = warp * kTileRows;
+  if (warp >= nwa || t0 >= cnt) return;
+  const int i = lane >> 1;
+  const int nrows = min(kTileRows, cnt - t0);
+  const uint16_t* kp = nullptr;
+  const uint16_t* vp = nullptr;
+  uint32_t mk = 0;
+  if (i < nrows) rowfn(t0 + i, kp, vp, mk);
+  tile_copy(stage + warp * kTileBytes, kp, vp, i < nrows && mk != 0);
+  cp_async_commit();
+}
+
 template <int G, class RowFn>
-__device__ __forceinline__ void attn_tiles(WarpAttn& W, int cnt, RowFn rowfn,
-                                           unsigned char* stage, int nwa) {
+__device__ __forceinline__ void attn_tiles(WarpAttn& W, int cnt, const RowFn& rowfn,
+                                           unsigned char* stage, int nwa, bool first_issued) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   if (warp >= nwa) return;
   unsigned char* tile = stage + warp * kTileBytes;
@@ -239,8 +257,10 @@ __device__ __forceinline__ void attn_tiles(WarpAttn& W, int cnt, RowFn rowfn,
     const uint16_t* vp = nullptr;
     uint32_t mk = 0;
     if (i < nrows) rowfn(t0 + i, kp, vp, mk);
-    tile_copy(tile, kp, vp, i < nrows && mk != 0);
-    cp_async_commit();
+    if (!(first_issued && t0 == warp * kTileRows)) {
+      tile_copy(tile, kp, vp, i < nrows && mk != 0);
+      cp_async_commit();
+    }
     cp_async_wait<0>();
     __syncwarp();
     tile_attend<G>(W, tile, nrows, mk);
