@@ -36,8 +36,8 @@ struct Plan {
   int64_t cand_stride;
   size_t off_ctrl, ctrl_bytes;
   size_t off_bar, off_team, off_locarr, off_misc, off_hist, off_hcnt;
-  size_t off_bstar, off_cstat, off_bands, off_ccnt, off_cpos, off_cbin, off_part, off_tpart,
-      off_lpart, off_trace, total;
+  size_t off_bstar, off_cstat, off_grange, off_sellist, off_part, off_tpart, off_lpart,
+      off_trace, total;
 };
 
 int check_desc(const rtp_layer_desc* d, LayerShape& L) {
@@ -113,10 +113,8 @@ int make_plan(const rtp_layer_desc* d, Plan& pl) {
   pl.ctrl_bytes = o - pl.off_ctrl;
   pl.off_bstar = o;  o = align256(o + sizeof(int32_t) * pl.n_groups * G);
   pl.off_cstat = o;  o = align256(o + 16 * size_t(pl.n_groups) * pl.max_nch * G);
-  pl.off_bands = o;  o = align256(o + 4 * size_t(pl.n_groups) * pl.max_nch * G * kBandRec);
-  pl.off_ccnt = o;   o = align256(o + sizeof(uint32_t) * size_t(pl.n_groups) * pl.max_nch);
-  pl.off_cpos = o;   o = align256(o + sizeof(uint32_t) * size_t(pl.n_groups) * pl.cand_stride);
-  pl.off_cbin = o;   o = align256(o + 8 * size_t(pl.n_groups) * pl.cand_stride);
+  pl.off_grange = o; o = align256(o + 8 * size_t(pl.n_groups) * G);
+  pl.off_sellist = o; o = align256(o + sizeof(uint32_t) * size_t(pl.n_groups) * pl.cand_stride);
   pl.off_part = o;   o = align256(o + part_bytes * pl.NC_max);
   pl.off_tpart = o;  o = align256(o + part_bytes * pl.NC_max);
   pl.off_lpart = o;  o = align256(o + part_bytes * std::max(pl.n_loc_items, 1));
@@ -186,7 +184,7 @@ int smem_layout(DecodeParams& P, const Plan& pl, int smem_optin) {
   small += align16(4 * P.L.B);                          // N
   small += align16(4 * (pl.n_groups + 1));              // cbase
   small += align16(8 * kMaxSteps * G);                  // tcache
-  small += align16(4 * G * kBandN * 32);                // mass bands, one word per lane
+  small += align16(8 * kMaxSteps * G);                  // lcache
   const int budget = smem_optin - 1024;
   const int stage = (budget - small) / 1024 * 1024;
   if (stage < DecodeCta<1>::kSRows * 32 * DecodeCta<1>::kSStages) return -1;
@@ -204,7 +202,7 @@ int smem_layout(DecodeParams& P, const Plan& pl, int smem_optin) {
   P.sm_N = o;     o += align16(4 * P.L.B);
   P.sm_cbase = o; o += align16(4 * (pl.n_groups + 1));
   P.sm_tcache = o; o += align16(8 * kMaxSteps * G);
-  P.sm_band = o;  o += align16(4 * G * kBandN * 32);
+  P.sm_lcache = o; o += align16(8 * kMaxSteps * G);
   return o;
 }
 
@@ -244,9 +242,6 @@ int launch_decode(DecodeParams& P, const Plan& pl, const DevInfo& di, cudaStream
     return RTP_ECUDA;
   P.P = std::min(di.sms, kPlanCTAs);
   if (pl.n_groups >= kMaxSteps * P.P) return RTP_ESHAPE;
-  // every chunk stays within kMaxChunk rows at kMaxSteps chunks per CTA
-  if (double(pl.n_groups) * double(P.L.maxN) > double(kMaxSteps) * P.P * kMaxChunk * 0.9)
-    return RTP_ESHAPE;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(P.P);
   cfg.blockDim = dim3(kFThreads);
@@ -260,7 +255,7 @@ int launch_decode(DecodeParams& P, const Plan& pl, const DevInfo& di, cudaStream
   if (cudaLaunchKernelEx(&cfg, decode_kernel<G>, P) != cudaSuccess) return RTP_ECUDA;
   int n = 1;
   if (sel_idx) {
-    emit_sel_kernel<G><<<P.L.B * P.L.Hq, kThreads, 0, st>>>(P, sel_idx, sel_stride);
+    emit_sel_kernel<G><<<P.L.B * P.L.Hq, kFThreads, 0, st>>>(P, sel_idx, sel_stride);
     ++n;
   }
   g_launches += n;
@@ -413,10 +408,8 @@ int decode_impl(const rtp_layer_desc* desc, const rtp_cache* cache, const uint16
   P.hcnt = at<int32_t>(ws, pl.off_hcnt);
   P.bstar = at<int32_t>(ws, pl.off_bstar);
   P.cstat = at<float4>(ws, pl.off_cstat);
-  P.bands = at<float>(ws, pl.off_bands);
-  P.ccnt = at<uint32_t>(ws, pl.off_ccnt);
-  P.cpos = at<uint32_t>(ws, pl.off_cpos);
-  P.cbin = at<uint2>(ws, pl.off_cbin);
+  P.grange = at<float2>(ws, pl.off_grange);
+  P.sellist = at<uint32_t>(ws, pl.off_sellist);
   P.part = at<float>(ws, pl.off_part);
   P.tpart = at<float>(ws, pl.off_tpart);
   P.lpart = at<float>(ws, pl.off_lpart);

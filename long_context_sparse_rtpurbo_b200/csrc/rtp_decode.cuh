@@ -47,16 +47,6 @@ constexpr int kHistStride = 256 + kHeadPad;
 constexpr int kSplitRows = 64;          // fewest candidates per gather split
 constexpr int kMaxSteps = 32;           // chunks per CTA, upper bound
 constexpr int kListCap = 4096;          // gather entries staged per batch
-// Mass bands of phase S (log2 units, relative to the chunk's first-stage maximum R): band
-// i < kBandN covers (R - i + 3, R - i + 4]; kBandOver: above R + 4; kBandTail: at or below
-// R - kBandN + 4. In shared memory a band i < kBandN holds its masses scaled by 2^(i - 4 + 19)
-// (each rounded up to an integer, so the sum bounds the band's mass from above) in one 32-bit
-// word per lane position ([G][kBandN][32]: the lanes of a warp never collide; at most 2^19 per
-// row and kMaxChunk / 32 = 4096 rows per word); the over and tail bands are kept in registers
-// (the tail as a count). A
-// published record holds the band masses relative to R as floats, and R in slot kBandR.
-constexpr int kBandN = 26, kBandOver = 26, kBandTail = 27, kBandR = 28, kBandRec = 32;
-constexpr int kMaxChunk = 131072;      // rows per chunk, upper bound
 
 struct DecodeParams {
   LayerShape L;
@@ -73,10 +63,10 @@ struct DecodeParams {
   int select_all;    // p >= 1
   double p;
   long long spin_limit;
-  int64_t cand_stride;   // candidate entries per group (>= max_seq_len)
+  int64_t cand_stride;   // list entries per group (>= max_seq_len)
   // shared-memory layout (byte offsets into the dynamic buffer)
   int sm_stage, sm_q, sm_qbuf, sm_qidx, sm_hist, sm_res, sm_tmp, sm_int, sm_N, sm_cbase,
-      sm_tcache, sm_band, free_bytes;
+      sm_tcache, sm_lcache, free_bytes;
   // inputs / outputs
   const uint16_t* q_pre;
   const float* w_qidx;
@@ -99,10 +89,8 @@ struct DecodeParams {
   int32_t* hcnt;               // [n_groups][G]  selected tokens per head            (zeroed)
   int32_t* bstar;              // [n_groups][G]  threshold bins (debug output)
   float4* cstat;               // [n_groups][max_nch][G]  chunk (min, max, sum 2^(y - max))
-  float* bands;                // [n_groups][max_nch][G][kBandRec] chunk mass bands and R
-  uint32_t* ccnt;              // [n_groups][max_nch]     candidates per chunk
-  uint32_t* cpos;              // [n_groups][cand_stride] candidate positions
-  uint2* cbin;                 // [n_groups][cand_stride] candidate bins (byte h: head h)
+  float2* grange;              // [n_groups][G]  group (min score, 256 / (max - min)), debug output
+  uint32_t* sellist;           // [n_groups][cand_stride] selected rows of recomputed chunks
   float* part;                 // [NC_max][G][130]
   float* tpart;                // [NC_max][G][130]
   float* lpart;                // [n_loc_items][G][130]
@@ -113,7 +101,7 @@ struct DecodeParams {
 // Each event keeps its last occurrence; kEvNLocWait / kEvNLocDrain count local items.
 enum TraceEvent { kEvStart, kEvPlan, kEvS0, kEvS1, kEvH0, kEvHw, kEvH1, kEvW0, kEvW1, kEvW2,
                   kEvW3, kEvLoc0, kEvLoc1, kEvDrain, kEvEnd, kEvNLocWait, kEvNLocDrain,
-                  kEvHs, kEvWl, kEvHb, kEvNCand, kEvBch0, kEvBand0, kTraceEvents = 32 };
+                  kEvHs, kEvWl, kTraceEvents = 32 };
 
 // ------------------------------------------------------------------------------ helpers
 __device__ __forceinline__ int seq_len_checked(const DecodeParams& P, int b) {
@@ -221,12 +209,12 @@ template <int G> struct Smem {
   __device__ int* N() const { return (int*)(rtp_smem + P.sm_N); }
   __device__ int* cbase() const { return (int*)(rtp_smem + P.sm_cbase); }
   __device__ double* tcache() const { return (double*)(rtp_smem + P.sm_tcache); }
-  __device__ float* band() const { return (float*)(rtp_smem + P.sm_band); }
+  __device__ float2* lcache() const { return (float2*)(rtp_smem + P.sm_lcache); }
 };
 // ints[]: [0..31] reduction scratch, [32] wait flag, [33] next local item, [36] last-split
 //         flag, [38] local-last flag, [40..47] b*, [48..55] decode token's index row
 //         (16 bf16), [60] tensor-memory base, [64..95] per-warp counts of ordered
-//         compactions (two blocks of 16)
+//         compactions (two blocks of 16), [96..127] tensor-memory column of each chunk
 
 // RoPE'd, pre-scaled query of the G heads of KV head kvh at position N - 1 -> q_s[G][128].
 template <int G>
@@ -439,7 +427,7 @@ struct DecodeCta {
         c = (Tr + den - 1) / den;
         c = max(c, (long long)P.C_min);
         c = (c + 63) / 64 * 64;
-        if ((c > P.C_cap && steps < kMaxSteps) || c > kMaxChunk) { ++steps; continue; }
+        if (c > P.C_cap && steps < kMaxSteps) { ++steps; continue; }
         break;
       }
       C = (int)c;
@@ -524,129 +512,90 @@ struct DecodeCta {
     cp_async_wait<0>();
   }
 
-  // Per-row work of phase S. Per head: min and max; the sum of 2^(y - rf) against a
-  // per-thread reference rf (R below, moved up only when a score exceeds it by 64, so the
-  // terms never overflow); and the mass 2^(y - R) of the row in its band (shared word of
-  // this lane position). R is the maximum of the chunk's first stage, found when that stage
-  // is scored (every thread takes part). When the chunk's scores are kept, each stage's G
-  // scores go to G tensor-memory columns of the thread's lane (a warp-wide store).
+  // Per-row work of phase S. Per head: min, max, and the sum of 2^(y - rf) against a
+  // per-thread reference rf (the first score, moved up only when a score exceeds it by 64, so
+  // the terms never overflow and the common step is one exponential and one add). When the
+  // chunk's scores are kept, each stage's G scores go to G tensor-memory columns of the
+  // thread's lane (a warp-wide store).
   struct SStats {
-    float mn[G], mx[G], rf[G], ls[G], R[G], over[G];
-    int tail[G];
-    int band_off;                  // byte offsets into rtp_smem: [G][kBandN][32] band words,
-    int red_off;                   // [16][G] reduction scratch
+    float mn[G], mx[G], rf[G], ls[G];
     uint32_t tbase;                // tensor-memory base
-    bool use_slot;
-    __device__ __forceinline__ SStats(uint32_t tb, bool u, int bw, int r)
-        : band_off(bw), red_off(r), tbase(tb), use_slot(u) {
+    int col0;                      // first column of this chunk (-1: scores not kept)
+    __device__ __forceinline__ SStats(uint32_t tb, int c) : tbase(tb), col0(c) {
 #pragma unroll
-      for (int k = 0; k < G; ++k) {
-        mn[k] = INFINITY; mx[k] = -INFINITY; rf[k] = INFINITY; ls[k] = 0.f; R[k] = 0.f;
-        over[k] = 0.f; tail[k] = 0;
-      }
+      for (int k = 0; k < G; ++k) { mn[k] = INFINITY; mx[k] = -INFINITY; rf[k] = -INFINITY; ls[k] = 0.f; }
     }
     __device__ __forceinline__ void operator()(int nl, bool ok, const float (&y)[G]) {
-      if (nl < kSRows) {                     // first stage: R = its maximum per head
-        const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-        float* red = smem_at<float>(red_off);
-#pragma unroll
-        for (int h = 0; h < G; ++h) {
-          float v = ok ? y[h] : -INFINITY;
-#pragma unroll
-          for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
-          if (lane == 0) red[warp * G + h] = v;
-        }
-        __syncthreads();
-#pragma unroll
-        for (int h = 0; h < G; ++h) {
-          float v = red[h];
-          for (int w = 1; w < kFThreads / 32; ++w) v = fmaxf(v, red[w * G + h]);
-          R[h] = v;
-          rf[h] = v;
-        }
-        __syncthreads();
-      }
-      if (use_slot) Tmem<G>::st(tmem_addr(tbase, (nl / kSRows) * G), y);   // whole warp
+      if (col0 >= 0) Tmem<G>::st(tmem_addr(tbase, col0 + (nl / kSRows) * G), y);   // whole warp
       if (!ok) return;
-      uint32_t* band = smem_at<uint32_t>(band_off) + (threadIdx.x & 31);
 #pragma unroll
       for (int h = 0; h < G; ++h) {
         mn[h] = fminf(mn[h], y[h]);
         mx[h] = fmaxf(mx[h], y[h]);
-        const float t = R[h] - y[h];
-        const float e = exp2f(-t);
-        // band: kk = floor(t) in [-8, 30] (round-down add of 1.5 * 2^23), i = kk + 4
-        const float tc = fminf(fmaxf(t, -8.f), 30.f);
-        const int kk = __float_as_int(__fadd_rd(tc, 12582912.f)) - 0x4B400000;
-        if (kk < -4) {
-          over[h] += e;
-        } else if (kk >= kBandN - 4) {
-          ++tail[h];
-        } else {                             // e * 2^(kk + 19) lies in (2^18, 2^19]
-          const uint32_t q = (uint32_t)__float2uint_ru(e * __int_as_float((kk + 19 + 127) << 23));
-          atomicAdd(band + (h * kBandN + kk + 4) * 32, q);
+        const float d = y[h] - rf[h];
+        if (d > 64.f) {
+          ls[h] = ls[h] * exp2f(-d) + 1.f;
+          rf[h] = y[h];
+        } else {
+          ls[h] += exp2f(d);
         }
-        if (rf[h] == R[h] && t >= -64.f) {
-          ls[h] += e;
-        } else {                             // a score 64 above R (rare)
-          const float d = y[h] - rf[h];
-          if (d > 64.f) {
-            ls[h] = ls[h] * exp2f(-d) + 1.f;
-            rf[h] = y[h];
-          } else {
-            ls[h] += exp2f(d);
+      }
+    }
+  };
+
+  // Per-row work of phase H: for each head whose score reaches ycut (half a bin below the
+  // cutoff bin's edge), the bin; when it reaches the cutoff, the row's fixed-point mass goes
+  // to the shared histogram (two 32-bit words per bin, exact).
+  struct HHist {
+    float lo[G], hi[G], inv[G], ycut[G];
+    int bch[G];
+    int hist_off;                  // byte offset of the histogram words in rtp_smem
+    __device__ __forceinline__ void operator()(int nl, bool ok, const float (&y)[G]) {
+      (void)nl;
+      if (!ok) return;
+      uint32_t* hlo = smem_at<uint32_t>(hist_off);
+      uint32_t* hhi = hlo + G * kHistStride;
+#pragma unroll
+      for (int h = 0; h < G; ++h) {
+        if (y[h] >= ycut[h]) {
+          const int b = inv[h] > 0.f ? bin_of(y[h], lo[h], inv[h]) : 0;
+          const float ex = y[h] - hi[h];
+          if (b >= bch[h] && ex > -42.f) {   // below 2^-41 the fixed-point mass rounds to 0
+            const unsigned long long q = __float2ull_rn(exp2f(ex) * kMassScale);
+            const int bi = h * kHistStride + b;
+            const uint32_t ql = (uint32_t)q, qh = (uint32_t)(q >> 32);
+            const uint32_t old = atomicAdd(&hlo[bi], ql);
+            const uint32_t up = qh + ((old + ql < old) ? 1u : 0u);
+            if (up) atomicAdd(&hhi[bi], up);
           }
         }
       }
     }
   };
 
-  // Per-row work of phase H: a row whose score reaches ycut for some head is binned; heads
-  // whose bin reaches the cutoff add its fixed-point mass to the shared histogram (two 32-bit
-  // words per bin, exact), and the row becomes a candidate, written in row order.
-  struct HEmit {
-    float lo[G], hi[G], inv[G], ycut[G];
-    int bch[G];
-    int hist_off;                  // byte offsets into rtp_smem: histogram words (lo, hi),
-    int wc_off;                    // per-warp counts of the ordered compaction
-    uint32_t* cpos;
-    uint2* cbin;
-    int n0, run, par;
+  // Per-row work of phase W when the scores are recomputed: the head mask of the row (heads
+  // whose bin reaches b*) and the ordered compaction of the selected rows into a list in
+  // global memory.
+  struct WSel {
+    float lo[G], inv[G];
+    int bs[G];
+    int hc[G];
+    uint32_t* out;                 // the chunk's list (global)
+    int n0, nb, par, wc_off;
     __device__ __forceinline__ void operator()(int nl, bool ok, const float (&y)[G]) {
-      bool pass = false;
-#pragma unroll
-      for (int h = 0; h < G; ++h) pass |= y[h] >= ycut[h];
-      bool cand = false;
-      uint32_t bw0 = 0, bw1 = 0;
-      uint32_t* hlo = smem_at<uint32_t>(hist_off);
-      uint32_t* hhi = hlo + G * kHistStride;
-      if (ok && pass) {
+      uint32_t mask = 0;
+      if (ok) {
 #pragma unroll
         for (int h = 0; h < G; ++h) {
           const int b = inv[h] > 0.f ? bin_of(y[h], lo[h], inv[h]) : 0;
-          if (h < 4) bw0 |= (uint32_t)b << (8 * h); else bw1 |= (uint32_t)b << (8 * (h - 4));
-          if (b >= bch[h]) {
-            cand = true;
-            const float ex = y[h] - hi[h];
-            if (ex > -42.f) {                // below 2^-41 the fixed-point mass rounds to 0
-              const unsigned long long q = __float2ull_rn(exp2f(ex) * kMassScale);
-              const int bi = h * kHistStride + b;
-              const uint32_t ql = (uint32_t)q, qh = (uint32_t)(q >> 32);
-              const uint32_t old = atomicAdd(&hlo[bi], ql);
-              const uint32_t up = qh + ((old + ql < old) ? 1u : 0u);
-              if (up) atomicAdd(&hhi[bi], up);
-            }
-          }
+          if (b >= bs[h]) { mask |= 1u << h; hc[h]++; }
         }
       }
       int before, total;
-      block_flag_prefix(cand, wc_off, par, before, total);
-      if (cand) {
-        cpos[run + before] = (uint32_t)(n0 + nl);
-        cbin[run + before] = make_uint2(bw0, bw1);
-      }
-      run += total;
+      block_flag_prefix(mask != 0, wc_off, par, before, total);
       par ^= 1;
+      if (mask) out[nb + before] = ((uint32_t)(n0 + nl) << 8) | mask;
+      nb += total;
     }
   };
 
@@ -676,19 +625,15 @@ struct DecodeCta {
   };
 
   // ------------------------------------------------------------ phase S
-  // Per head: min, max, and the sum of 2^(y - r) against a per-thread reference r (the first
-  // score, moved up only when a score exceeds it by 64, so 2^(y - r) never overflows and the
-  // common step is one exponential and one add).
-  __device__ __forceinline__ void phase_score(int k, bool use_slot) {
+  // tcol: first tensor-memory column of the chunk's scores, -1 when they are not kept.
+  __device__ __forceinline__ void phase_score(int k, int tcol) {
     const int g = group_of(k), j = k - sm.cbase()[g];
     const int N = gN(g);
     const bool patch = P.k_new && min(N, (j + 1) * C) == N;
-    float* bnd = sm.band();                  // [G][kBandN][32]
-    for (int i = threadIdx.x; i < G * kBandN * 32; i += kFThreads) bnd[i] = 0.f;
-    SStats sst((uint32_t)sm.ints()[60], use_slot, P.sm_band, P.sm_tmp);
+    SStats sst((uint32_t)sm.ints()[60], tcol);
     trace(kEvS0);
-    stream_chunk(g, j, patch, sst);             // begins with a barrier (bands zeroed)
-    if (use_slot) tmem_wait_st();
+    stream_chunk(g, j, patch, sst);
+    if (tcol >= 0) tmem_wait_st();
     trace(kEvS1);
     float (&mn)[G] = sst.mn;
     float (&mx)[G] = sst.mx;
@@ -732,126 +677,7 @@ struct DecodeCta {
       }
       P.cstat[((int64_t)g * P.max_nch + j) * G + h] = make_float4(a, z, (float)l, 0.f);
     }
-    // the chunk's bands: the warps' words (summed in 64 bits and rounded up to float), the
-    // over masses and tail counts reduced from the threads, and R
-    __syncthreads();
-#pragma unroll
-    for (int h = 0; h < G; ++h) {
-      float ov = sst.over[h];
-      int tc = sst.tail[h];
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) {
-        ov += __shfl_xor_sync(0xffffffffu, ov, o);
-        tc += __shfl_xor_sync(0xffffffffu, tc, o);
-      }
-      if (lane == 0) {
-        red[(0 * G + h) * 16 + warp] = ov;
-        reinterpret_cast<int*>(red)[(1 * G + h) * 16 + warp] = tc;
-      }
-    }
-    __syncthreads();
-    float* gb = P.bands + ((int64_t)g * P.max_nch + j) * G * kBandRec;
-    const uint32_t* bnd_u = reinterpret_cast<const uint32_t*>(bnd);
-    for (int i = threadIdx.x; i < G * kBandRec; i += kFThreads) {
-      const int h = i / kBandRec, k = i % kBandRec;
-      float v = 0.f;
-      if (k < kBandN) {
-        unsigned long long sum = 0;
-        for (int l = 0; l < 32; ++l) sum += bnd_u[(h * kBandN + k) * 32 + l];
-        v = __fmul_ru(__ull2float_ru(sum), __int_as_float((127 - (k - 4 + 19)) << 23));
-      } else if (k == kBandOver) {
-        for (int w = 0; w < kFThreads / 32; ++w) v += red[(0 * G + h) * 16 + w];
-        v = __fmul_ru(v, 1.001f);               // bounds the rounding of the float sum
-      } else if (k == kBandTail) {
-        int c = 0;
-        for (int w = 0; w < kFThreads / 32; ++w) c += reinterpret_cast<const int*>(red)[(1 * G + h) * 16 + w];
-        v = (float)c * exp2f(-(float)(kBandN - 4));    // each at most 2^-(kBandN - 4)
-      } else if (k == kBandR) {
-        v = sst.R[h];
-      }
-      gb[i] = v;
-    }
     arrive(P.bar + (int64_t)g * 4 + 0);
-  }
-
-  // A tighter cutoff from the chunks' mass bands. A band of chunk c holds tokens whose
-  // scores lie in an interval (y_low, y_high]; for an edge e the tokens below e are within the
-  // bands with y_low < e, so U(e) = sum of those bands' masses (relative to hi) bounds the
-  // mass below e from above (a small margin on y_low covers the rounding of the band index).
-  // C_b >= T - U(e_b), so every b with T - U(e_b) >= p T satisfies b <= b*; the largest such
-  // b is the cutoff when it exceeds the first bound. U is built per head as a scatter of the
-  // band masses onto their first bin (shared atomics) and a prefix sum (one warp per head).
-  __device__ __forceinline__ void band_cutoff(int g, int nc, int step, HEmit& em) {
-    uint32_t* dU = reinterpret_cast<uint32_t*>(sm.hist());  // [G][257], units of T 2^-27
-    for (int i = threadIdx.x; i < G * 257; i += kFThreads) dU[i] = 0u;
-    __syncthreads();
-    if (!P.select_all) {
-      const float* gb = P.bands + (int64_t)g * P.max_nch * G * kBandRec;
-      const int tot = nc * G * kBandRec;
-      for (int i = threadIdx.x; i < tot; i += kFThreads) {
-        const int k = i % kBandRec, h = (i / kBandRec) % G;
-        if (k >= kBandR) continue;
-        const float v = __ldcg(gb + i);
-        if (!(v > 0.f)) continue;
-        const float Rc = __ldcg(gb + (i - k) + kBandR);
-        float hi = 0.f, lo = 0.f, inv = 0.f;
-#pragma unroll
-        for (int hh = 0; hh < G; ++hh)
-          if (hh == h) { hi = em.hi[hh]; lo = em.lo[hh]; inv = em.inv[hh]; }
-        if (!(inv > 0.f)) continue;
-        const double T = sm.tcache()[step * G + h];
-        // the band's mass relative to the group max, in units of T 2^-27, rounded up (all
-        // bands together stay far below 2^32 units: their mass is at most a few T)
-        const double mu = (double)v * exp2((double)Rc - (double)hi) / T * 134217728.0;
-        const uint32_t q = mu >= 4.0e9 ? 4000000000u : (uint32_t)ceil(mu);
-        int b0 = 0;
-        if (k != kBandTail) {
-          const float ylow = (k == kBandOver ? Rc + 4.f : Rc + 3.f - (float)k) - 0.01f;
-          const float x = (ylow - lo) * inv;
-          b0 = x < 0.f ? 0 : min(256, (int)x + 1);
-        }
-        if (q) atomicAdd(dU + h * 257 + b0, q);
-      }
-    }
-    __syncthreads();
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    if (warp < G && !P.select_all) {
-      const int h = warp;
-      float inv = 0.f;
-#pragma unroll
-      for (int hh = 0; hh < G; ++hh) if (hh == h) inv = em.inv[hh];
-      if (inv > 0.f) {
-        // lane l holds bins 8l .. 8l + 7: inclusive prefix of dU (64-bit sums)
-        unsigned long long v[8], run = 0;
-#pragma unroll
-        for (int e = 0; e < 8; ++e) { run += dU[h * 257 + lane * 8 + e]; v[e] = run; }
-        unsigned long long incl = run;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-          const unsigned long long y = __shfl_up_sync(0xffffffffu, incl, o);
-          if (lane >= o) incl += y;
-        }
-        const unsigned long long base = incl - run;
-        // U(e_b) / T = prefix 2^-27 (each part rounded up); b is certified when
-        // 1 - 1.001 U / T >= p
-        int best = -1;
-#pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          const double u = (double)(base + v[e]) * (1.0 / 134217728.0) * 1.001;
-          if (1.0 - u >= P.p) best = lane * 8 + e;
-        }
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) best = max(best, __shfl_xor_sync(0xffffffffu, best, o));
-        if (lane == 0) sm.ints()[40 + h] = best;
-      } else if (lane == 0) {
-        sm.ints()[40 + h] = -1;
-      }
-    }
-    __syncthreads();
-#pragma unroll
-    for (int h = 0; h < G; ++h)
-      if (!P.select_all) em.bch[h] = max(em.bch[h], sm.ints()[40 + h]);
-    __syncthreads();                       // the scratch is rewritten next
   }
 
   // ------------------------------------------------------------ phase H
@@ -860,11 +686,9 @@ struct DecodeCta {
   // bin(c), c = hi + log2((1 - p) T' / N), T' = T (1 - 1e-3), has mass below (1 - p) T' / N,
   // so together they hold less than (1 - p) of the total, C_bin(c) > p T, and b* can not fall
   // under the cutoff bin (the 1e-3 absorbs the rounding of T, the log and the bin edges).
-  // A token is binned only when a score reaches half a bin below the cutoff bin's edge (so
-  // every token whose bin reaches the cutoff is binned, and the others cost one compare).
-  // Masses are 2^(y - max) in 2^-40 fixed point, summed with two 32-bit shared atomics per
-  // (token, head): the low-word add returns the old value and its carry goes to the high word.
-  __device__ __forceinline__ void phase_hist(int k, int step, bool from_slot) {
+  // Rows whose bin reaches the cutoff add their masses (2^(y - max) in 2^-40 fixed point) to
+  // the group's histogram. The range (lo, 256 / (hi - lo)) and T are kept for phase W.
+  __device__ __forceinline__ void phase_hist(int k, int step, int tcol) {
     const int g = group_of(k), j = k - sm.cbase()[g];
     const int N = gN(g), n0 = j * C, len = min(N, n0 + C) - n0;
     const int nc = nch(g);
@@ -899,9 +723,12 @@ struct DecodeCta {
           lo = fminf(lo, pf[w * G + t]);
           hi = fmaxf(hi, pf[512 + w * G + t]);
         }
+        const float inv = (hi > lo && !P.select_all) ? (float)kBins / (hi - lo) : 0.f;
         st3[t * 3 + 0] = lo;
         st3[t * 3 + 1] = hi;
-        st3[t * 3 + 2] = (hi > lo && !P.select_all) ? (float)kBins / (hi - lo) : 0.f;
+        st3[t * 3 + 2] = inv;
+        sm.lcache()[step * G + t] = make_float2(lo, inv);
+        if (j == 0) P.grange[(int64_t)g * G + t] = make_float2(lo, inv);
       }
       __syncthreads();
       const float hih = st3[h * 3 + 1];
@@ -921,74 +748,48 @@ struct DecodeCta {
       __syncthreads();
     }
     trace(kEvHs);
-    uint32_t* hlo = sm.hist();
-    uint32_t* hhi = hlo + G * kHistStride;
-    HEmit em;
+    HHist hh;
 #pragma unroll
     for (int h = 0; h < G; ++h) {
-      em.lo[h] = st3[h * 3 + 0];
-      em.hi[h] = st3[h * 3 + 1];
-      em.inv[h] = st3[h * 3 + 2];
-      em.bch[h] = 0;
-      if (P.p < 1.0 && em.inv[h] > 0.f) {
+      hh.lo[h] = st3[h * 3 + 0];
+      hh.hi[h] = st3[h * 3 + 1];
+      hh.inv[h] = st3[h * 3 + 2];
+      hh.bch[h] = 0;
+      if (P.p < 1.0 && hh.inv[h] > 0.f) {
         const double T = sm.tcache()[step * G + h];
         const float arg = (float)((1.0 - P.p) * T * (1.0 - 1e-3) / (double)N);
-        const float c = em.hi[h] + log2f(arg);
-        em.bch[h] = c > em.lo[h] ? bin_of(c, em.lo[h], em.inv[h]) : 0;
+        const float c = hh.hi[h] + log2f(arg);
+        hh.bch[h] = c > hh.lo[h] ? bin_of(c, hh.lo[h], hh.inv[h]) : 0;
       }
+      hh.ycut[h] = hh.bch[h] > 0 ? hh.lo[h] + ((float)hh.bch[h] - 0.5f) / hh.inv[h] : -INFINITY;
     }
-    const int bch_first = em.bch[0];
-    band_cutoff(g, nc, step, em);
-#ifdef RTP_TRACE
-    if (threadIdx.x == 0 && P.trace) {
-      P.trace[(int64_t)blockIdx.x * kTraceEvents + kEvBch0] = (unsigned long long)bch_first;
-      P.trace[(int64_t)blockIdx.x * kTraceEvents + kEvBand0] = (unsigned long long)em.bch[0];
-    }
-#endif
-    (void)bch_first;
-#pragma unroll
-    for (int h = 0; h < G; ++h)
-      em.ycut[h] = em.bch[h] > 0 ? em.lo[h] + ((float)em.bch[h] - 0.5f) / em.inv[h] : -INFINITY;
-    em.hist_off = P.sm_hist;
-    em.cpos = P.cpos + (int64_t)g * P.cand_stride + n0;
-    em.cbin = P.cbin + (int64_t)g * P.cand_stride + n0;
-    em.wc_off = P.sm_int + 64 * 4;          // [2][16]
-    em.n0 = n0;
-    em.run = 0;
-    em.par = 0;
+    hh.hist_off = P.sm_hist;
+    uint32_t* hlo = sm.hist();
+    uint32_t* hhi = hlo + G * kHistStride;
     for (int i = threadIdx.x; i < 2 * G * kHistStride; i += kFThreads) hlo[i] = 0u;
     __syncthreads();
-    if (from_slot) {
+    if (tcol >= 0) {
       const uint32_t tb = (uint32_t)sm.ints()[60];
 #pragma unroll 1
       for (int i0 = 0; i0 < len; i0 += kFThreads) {
         const int nl = i0 + threadIdx.x;
         float y[G];
-        Tmem<G>::ld(tmem_addr(tb, (i0 / kSRows) * G), y);     // whole warp
+        Tmem<G>::ld(tmem_addr(tb, tcol + (i0 / kSRows) * G), y);     // whole warp
         tmem_wait_ld();
-        if (nl >= len) {
-#pragma unroll
-          for (int h = 0; h < G; ++h) y[h] = -INFINITY;
-        }
-        em(nl, nl < len, y);
-        if (i0 == 0) trace(kEvHb);
+        hh(nl, nl < len, y);
       }
     } else {
-      stream_chunk(g, j, false, em);
+      stream_chunk(g, j, false, hh);
     }
     __syncthreads();
     trace(kEvH1);
     unsigned long long* gh = P.hist + (int64_t)g * G * kBins;
     for (int i = threadIdx.x; i < G * kBins; i += kFThreads) {
-      const int hh = i / kBins, b = i % kBins;
+      const int hd = i / kBins, b = i % kBins;
       const unsigned long long v =
-          ((unsigned long long)hhi[hh * kHistStride + b] << 32) | hlo[hh * kHistStride + b];
+          ((unsigned long long)hhi[hd * kHistStride + b] << 32) | hlo[hd * kHistStride + b];
       if (v) atomicAdd(gh + i, v);
     }
-    if (threadIdx.x == 0) P.ccnt[(int64_t)g * P.max_nch + j] = (uint32_t)em.run;
-#ifdef RTP_TRACE
-    if (threadIdx.x == 0 && P.trace) P.trace[(int64_t)blockIdx.x * kTraceEvents + kEvNCand] += (unsigned long long)em.run;
-#endif
     arrive(P.bar + (int64_t)g * 4 + 1);
   }
 
@@ -999,40 +800,30 @@ struct DecodeCta {
   }
 
   // ------------------------------------------------------------ phase W
-  // Split j of group g: candidates [e0, e1) of the group's list (chunk after chunk), loaded
-  // in batches of kListCap; a candidate is kept when a head's bin reaches its b*, with the
-  // mask of those heads, in candidate order. The list and the chunk prefix sit at the end of
-  // the free region (the score slot is dead by now); the tiles use its start. The rotated
-  // query is formed before the wait.
-  static constexpr int kEPer = kListCap / kFThreads;        // entries per thread per batch
-  __device__ __forceinline__ void phase_attend(int k, int step) {
+  // The chunk's own rows with bin >= b* for some head (from its kept scores, or recomputed
+  // from the index rows), with the mask of those heads, in row order; their K/V rows are
+  // gathered once for all G heads. Kept scores: the list is built in shared memory at the
+  // end of the staging region and handed to the attention loop whenever it fills up.
+  // Recomputed scores: the list is written to global memory first (the index ring and the
+  // tiles share the staging region), then read back in batches. The rotated query is formed
+  // before the wait. Partials merge in teams of kTeam by the last arrivals.
+  __device__ __forceinline__ void phase_attend(int k, int step, int tcol) {
     const int g = group_of(k), j = k - sm.cbase()[g];
     const int b = g / P.L.n_ret, r = g % P.L.n_ret, kvh = P.L.ret_kv[r];
-    const int N = gN(g);
+    const int N = gN(g), n0 = j * C, len = min(N, n0 + C) - n0;
     const int S = nch(g);
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     rope_query<G>(P, b, kvh, N, sm.q());
     if (!wait_for(P.bar + (int64_t)g * 4 + 1, (uint32_t)S)) { abort_ = true; return; }
     trace(kEvW0);
-    const int pref_bytes = ((S + 1) * 4 + 15) / 16 * 16;
-    int* pref = reinterpret_cast<int*>(sm.stage() + P.free_bytes - pref_bytes);
-    uint32_t* list = reinterpret_cast<uint32_t*>(reinterpret_cast<unsigned char*>(pref) - kListCap * 4);
-    // one round trip: the group histogram (warp h: head h) and the chunks' candidate counts
-    unsigned long long hv[8];
-    if (warp < G && !P.select_all) {
-      const unsigned long long* gh = P.hist + ((int64_t)g * G + warp) * kBins + lane * 8;
-#pragma unroll
-      for (int e = 0; e < 8; ++e) hv[e] = __ldcg(gh + e);
-    }
-    for (int c = threadIdx.x; c < S; c += kFThreads)
-      pref[c] = (int)__ldcg(P.ccnt + (int64_t)g * P.max_nch + c);
-    // b* per head: the highest bin whose mass from the top reaches p T
+    // b* per head (warp h: head h): the highest bin whose mass from the top reaches p T
     if (warp < G) {
       int best = 0;
       if (!P.select_all) {
-        unsigned long long lt = 0;
+        const unsigned long long* gh = P.hist + ((int64_t)g * G + warp) * kBins + lane * 8;
+        unsigned long long hv[8], lt = 0;
 #pragma unroll
-        for (int e = 0; e < 8; ++e) lt += hv[e];
+        for (int e = 0; e < 8; ++e) { hv[e] = __ldcg(gh + e); lt += hv[e]; }
         unsigned long long x = lt;            // inclusive suffix sum over lanes
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
@@ -1054,80 +845,84 @@ struct DecodeCta {
       if (lane == 0) sm.ints()[40 + warp] = best;
     }
     __syncthreads();
-    int bs[G];
+    WSel ws;
 #pragma unroll
-    for (int h = 0; h < G; ++h) bs[h] = sm.ints()[40 + h];
-    if (j == 0 && threadIdx.x < G) P.bstar[(int64_t)g * G + threadIdx.x] = bs[threadIdx.x];
-    const int U = block_scan_excl(pref, S, sm.ints());
-    const int nsplit = min(min(S, kTeam), max(1, (U + kSplitRows - 1) / kSplitRows));
-    if (j >= nsplit) return;
-    const int e0 = (int)(((long long)U * j) / nsplit), e1 = (int)(((long long)U * (j + 1)) / nsplit);
+    for (int h = 0; h < G; ++h) {
+      ws.bs[h] = sm.ints()[40 + h];
+      const float2 li = sm.lcache()[step * G + h];
+      ws.lo[h] = li.x;
+      ws.inv[h] = li.y;
+      ws.hc[h] = 0;
+    }
+    if (j == 0 && threadIdx.x < G) P.bstar[(int64_t)g * G + threadIdx.x] = ws.bs[threadIdx.x];
+    ws.n0 = n0;
+    ws.nb = 0;
+    ws.par = 0;
+    ws.wc_off = P.sm_int + 64 * 4;
     const int64_t rowbase = (int64_t)r * P.L.T_total + P.cache.seq_off[b];
     const uint16_t* kb = P.cache.k_ret + rowbase * kD;
     const uint16_t* vb = P.cache.v_ret + rowbase * kD;
-    const uint32_t* gpos = P.cpos + (int64_t)g * P.cand_stride;
-    const uint2* gbin = P.cbin + (int64_t)g * P.cand_stride;
-    const int nwa = min(kFThreads / 32, (P.free_bytes - pref_bytes - kListCap * 4) / kTileBytes);
-    int hc[G];
-#pragma unroll
-    for (int h = 0; h < G; ++h) hc[h] = 0;
+    uint32_t* list = reinterpret_cast<uint32_t*>(sm.stage() + P.free_bytes - kListCap * 4);
+    const int nwa = min(kFThreads / 32, (P.free_bytes - kListCap * 4) / kTileBytes);
+    const ListRows rows{list, kb, vb};
     WarpAttn W;
-    attn_begin<G>(W, sm.qbuf(), sm.q(), kFThreads);
-    trace(kEvW1);
-    const int wc_off = P.sm_int + 64 * 4;
-    int par = 0;
+    if (tcol >= 0) {
+      attn_begin<G>(W, sm.qbuf(), sm.q(), kFThreads);
+      trace(kEvW1);
+      const uint32_t tb = (uint32_t)sm.ints()[60];
 #pragma unroll 1
-    for (int b0 = e0; b0 < e1; b0 += kListCap) {
-      const int b1 = min(e1, b0 + kListCap);
-      // all of this thread's entries of the batch in flight at once
-      uint32_t pos[kEPer];
-      uint2 bw[kEPer];
-#pragma unroll
-      for (int u = 0; u < kEPer; ++u) {
-        const int e = b0 + u * kFThreads + threadIdx.x;
-        pos[u] = 0;
-        bw[u] = make_uint2(0, 0);
-        if (e < b1) {
-          const int c = upper_index(pref, S, e);
-          const int64_t o = (int64_t)c * C + (e - pref[c]);
-          pos[u] = __ldcg(gpos + o);
-          bw[u] = __ldcg(gbin + o);
+      for (int i0 = 0; i0 < len; i0 += kFThreads) {
+        if (ws.nb > kListCap - kFThreads) {   // the list is full: attend to it first
+          __syncthreads();
+          attn_tiles<G>(W, ws.nb, rows, sm.stage(), nwa, false);
+          __syncthreads();
+          ws.nb = 0;
         }
-      }
-      __syncthreads();                    // the previous batch's list is no longer read
-      int nb = 0;                         // kept entries of this batch (every thread)
-      const int nu = (b1 - b0 + kFThreads - 1) / kFThreads;   // uniform over the CTA
+        const int nl = i0 + threadIdx.x;
+        float y[G];
+        Tmem<G>::ld(tmem_addr(tb, tcol + (i0 / kSRows) * G), y);     // whole warp
+        tmem_wait_ld();
+        uint32_t mask = 0;
+        if (nl < len) {
 #pragma unroll
-      for (int u = 0; u < kEPer; ++u) {
-        if (u < nu) {
-          const int e = b0 + u * kFThreads + threadIdx.x;
-          uint32_t mask = 0;
-          if (e < b1) {
-#pragma unroll
-            for (int h = 0; h < G; ++h) {
-              const int bb = (int)(((h < 4 ? bw[u].x : bw[u].y) >> (8 * (h & 3))) & 0xffu);
-              if (bb >= bs[h]) { mask |= 1u << h; hc[h]++; }
-            }
+          for (int h = 0; h < G; ++h) {
+            const int bb = ws.inv[h] > 0.f ? bin_of(y[h], ws.lo[h], ws.inv[h]) : 0;
+            if (bb >= ws.bs[h]) { mask |= 1u << h; ws.hc[h]++; }
           }
-          int before, total;
-          block_flag_prefix(mask != 0, wc_off, par, before, total);
-          par ^= 1;
-          if (mask) list[nb + before] = (pos[u] << 8) | mask;
-          nb += total;
         }
+        int before, total;
+        block_flag_prefix(mask != 0, ws.wc_off, ws.par, before, total);
+        ws.par ^= 1;
+        if (mask) list[ws.nb + before] = ((uint32_t)(n0 + nl) << 8) | mask;
+        ws.nb += total;
       }
       __syncthreads();
       trace(kEvWl);
-      const ListRows rows{list, kb, vb};
-      attn_tiles<G>(W, nb, rows, sm.stage(), nwa, false);
+      attn_tiles<G>(W, ws.nb, rows, sm.stage(), nwa, false);
+    } else {
+      uint32_t* gl = P.sellist + (int64_t)g * P.cand_stride + n0;
+      ws.out = gl;
+      stream_chunk(g, j, false, ws);
+      __syncthreads();
+      attn_begin<G>(W, sm.qbuf(), sm.q(), kFThreads);
+      trace(kEvWl);
+      const int total = ws.nb;
+#pragma unroll 1
+      for (int b0 = 0; b0 < total; b0 += kListCap) {
+        const int nb = min(kListCap, total - b0);
+        __syncthreads();
+        for (int i = threadIdx.x; i < nb; i += kFThreads) list[i] = __ldcg(gl + b0 + i);
+        __syncthreads();
+        attn_tiles<G>(W, nb, rows, sm.stage(), nwa, false);
+      }
     }
     attn_end<G>(W, nwa, sm.res(), reinterpret_cast<float*>(sm.stage()), kFThreads);
     trace(kEvW2);
-    // per-head counts of this split
+    // per-head counts of this chunk
     int* red = reinterpret_cast<int*>(sm.tmp());              // [16][G]
 #pragma unroll
     for (int h = 0; h < G; ++h) {
-      int v = hc[h];
+      int v = ws.hc[h];
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
       if (lane == 0) red[warp * G + h] = v;
@@ -1138,20 +933,36 @@ struct DecodeCta {
       for (int w = 0; w < kFThreads / 32; ++w) v += red[w * G + threadIdx.x];
       if (v) atomicAdd(P.hcnt + (int64_t)g * G + threadIdx.x, v);
     }
-    // partial -> workspace; the last split merges the group's partials
+    // partial -> workspace; team / group merge by the last arrivals
     const int stride = G * (kD + 2);
     float* mine = P.part + (int64_t)k * stride;
     for (int o = threadIdx.x; o < stride; o += kFThreads) mine[o] = sm.res()[o];
+    const int team = j / kTeam, nteams = (S + kTeam - 1) / kTeam;
+    const int tcount = min(kTeam, S - team * kTeam);
     __syncthreads();
     if (threadIdx.x == 0) {
       __threadfence();
-      sm.ints()[36] = atomicAdd(P.team_arr + sm.cbase()[g], 1u) == (uint32_t)(nsplit - 1);
+      sm.ints()[36] = atomicAdd(P.team_arr + sm.cbase()[g] + team, 1u) == (uint32_t)(tcount - 1);
     }
     __syncthreads();
     if (!sm.ints()[36]) return;
     __threadfence();
-    merge(P.part + (int64_t)sm.cbase()[g] * stride, nsplit, nullptr,
-          P.out + ((int64_t)b * P.L.Hq + kvh * G) * kD, P.free_bytes);
+    uint16_t* orow = P.out + ((int64_t)b * P.L.Hq + kvh * G) * kD;
+    const float* tparts = P.part + (int64_t)(sm.cbase()[g] + team * kTeam) * stride;
+    if (nteams == 1) {
+      merge(tparts, tcount, nullptr, orow, P.free_bytes);
+    } else {
+      merge(tparts, tcount, P.tpart + (int64_t)(sm.cbase()[g] + team) * stride, nullptr, P.free_bytes);
+      __syncthreads();
+      if (threadIdx.x == 0) {
+        __threadfence();
+        sm.ints()[37] = atomicAdd(P.bar + (int64_t)g * 4 + 2, 1u) == (uint32_t)(nteams - 1);
+      }
+      __syncthreads();
+      if (!sm.ints()[37]) return;
+      __threadfence();
+      merge(P.tpart + (int64_t)sm.cbase()[g] * stride, nteams, nullptr, orow, P.free_bytes);
+    }
     if (threadIdx.x < G)
       P.sel_counts[(int64_t)b * P.L.Hq + kvh * G + threadIdx.x] =
           __ldcg(P.hcnt + (int64_t)g * G + threadIdx.x);
@@ -1228,38 +1039,45 @@ struct DecodeCta {
   // Chunks k_t = blockIdx.x + t P_ret of a chunk CTA, in group order. Phase S runs for every
   // chunk in turn; the chunks of a group get their phase H once the CTA has scored the first
   // chunk of the next group (or at the end), so the wait for the group's other chunks
-  // overlaps that scoring. Phase H of every chunk but the last recomputes its scores; the
-  // last chunk keeps them in the shared-memory slot when it fits. Then phase W of every
-  // chunk, then local items until the queue is empty. CTAs [P_ret, P) only run local items.
+  // overlaps that scoring. The scores of the first chunks are kept in tensor memory as long
+  // as its columns last (kTmemColsPerThread / G stages of kSRows rows per thread); phases H
+  // and W of later chunks recompute them from the index rows. Then phase W of every chunk,
+  // then local items until the queue is empty. CTAs [P_ret, P) only run local items.
   __device__ void run() {
     trace(kEvStart);
     plan();
     trace(kEvPlan);
     const int i = blockIdx.x;
     const int m = (i < P_ret && i < NC) ? (NC - i + P_ret - 1) / P_ret : 0;
-    bool last_in_slot = false;
-    if (m > 0) {
-      const int kl = i + (m - 1) * P_ret, gl = group_of(kl), jl = kl - sm.cbase()[gl];
-      last_in_slot = min(gN(gl), (jl + 1) * C) - jl * C <= P.C_cap;
+    int* tcols = sm.ints() + 96;                              // [kMaxSteps]
+    if (threadIdx.x == 0) {
+      int col = 0;
+      for (int t = 0; t < m; ++t) {
+        const int k = i + t * P_ret, g = group_of(k), j = k - sm.cbase()[g];
+        const int len = min(gN(g), (j + 1) * C) - j * C;
+        const int need = (len + kSRows - 1) / kSRows * G;
+        if (col + need <= kTmemColsPerThread) { tcols[t] = col; col += need; } else { tcols[t] = -1; }
+      }
     }
+    __syncthreads();
     int pstart = 0;
     for (int t = 0; t < m; ++t) {
       const int k = i + t * P_ret;
-      phase_score(k, t == m - 1 && last_in_slot);
+      phase_score(k, tcols[t]);
       if (pstart < t && group_of(i + pstart * P_ret) != group_of(k)) {
         for (int s = pstart; s < t; ++s) {
-          phase_hist(i + s * P_ret, s, false);
+          phase_hist(i + s * P_ret, s, tcols[s]);
           if (abort_) return;
         }
         pstart = t;
       }
     }
     for (int s = pstart; s < m; ++s) {
-      phase_hist(i + s * P_ret, s, s == m - 1 && last_in_slot);
+      phase_hist(i + s * P_ret, s, tcols[s]);
       if (abort_) return;
     }
     for (int t = 0; t < m; ++t) {
-      phase_attend(i + t * P_ret, t);
+      phase_attend(i + t * P_ret, t, tcols[t]);
       if (abort_) return;
     }
     local_items();
@@ -1285,76 +1103,58 @@ __global__ void __launch_bounds__(kFThreads, 1) decode_kernel(const __grid_const
 }
 
 // ------------------------------------------------------------------------------ sel_idx
-// Debug output: ascending positions each query head attended to. One CTA per (b, h): the
-// selected candidates of the head are marked in a shared-memory bitmap window of kEmitBits
-// positions, which is then read in order.
-constexpr int kEmitBits = 1 << 18;
+// Debug output: ascending positions each query head attended to. One CTA of kFThreads threads
+// per (b, h): a retrieval head's scores are recomputed with the decode kernel's own routines
+// (the same index query, the same per-row arithmetic, so the same bits), binned with the
+// group's range and compared with its b*; the selected positions are compacted in order.
 template <int G>
-__global__ void __launch_bounds__(kThreads) emit_sel_kernel(DecodeParams P, int32_t* sel_idx,
-                                                            int64_t sel_stride) {
-  __shared__ uint32_t bm[kEmitBits / 32];
-  __shared__ int wsum[kThreads / 32];
+__global__ void __launch_bounds__(kFThreads) emit_sel_kernel(DecodeParams P, int32_t* sel_idx,
+                                                             int64_t sel_stride) {
+  __shared__ float qidx[G * kR];
+  __shared__ float tmp[kFThreads];
+  __shared__ int wc[32];
   const int b = blockIdx.x / P.L.Hq, h = blockIdx.x % P.L.Hq;
   const int kvh = h / G, jh = h % G;
   const int N = seq_len_checked(P, b);
   int32_t* dst = sel_idx + ((int64_t)b * P.L.Hq + h) * sel_stride;
   if (N == 0) return;
   const int slot = P.L.slot[kvh];
-  const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
+  const int t = threadIdx.x;
   if (slot < 0) {
     const int s1 = min(N, P.L.sinks);
     const int w0 = max(P.L.sinks, N - P.L.window);
     const int cnt = s1 + max(0, N - w0);
-    for (int k = t; k < cnt; k += kThreads) dst[k] = k < s1 ? k : w0 + (k - s1);
+    for (int k = t; k < cnt; k += kFThreads) dst[k] = k < s1 ? k : w0 + (k - s1);
     return;
   }
   const int g = b * P.L.n_ret + slot;
-  const int C = (int)__ldcg(P.misc + 2);
-  const int nchg = (N + C - 1) / C;
   const int bst = __ldcg(P.bstar + (int64_t)g * G + jh);
-  const uint32_t* gpos = P.cpos + (int64_t)g * P.cand_stride;
-  const uint2* gbin = P.cbin + (int64_t)g * P.cand_stride;
-  int base = 0;
-  constexpr int kWords = kEmitBits / 32, kPer = kWords / kThreads;
-  for (int w0 = 0; w0 < N; w0 += kEmitBits) {
-    for (int i = t; i < kWords; i += kThreads) bm[i] = 0u;
-    __syncthreads();
-    for (int c = 0; c < nchg; ++c) {
-      const int cnt = (int)__ldcg(P.ccnt + (int64_t)g * P.max_nch + c);
-      for (int e = t; e < cnt; e += kThreads) {
-        const int64_t o = (int64_t)c * C + e;
-        const uint2 bw = __ldcg(gbin + o);
-        const int bb = (int)(((jh < 4 ? bw.x : bw.y) >> (8 * (jh & 3))) & 0xffu);
-        const int pos = (int)__ldcg(gpos + o) - w0;
-        if (bb >= bst && pos >= 0 && pos < kEmitBits) atomicOr(&bm[pos >> 5], 1u << (pos & 31));
-      }
-    }
-    __syncthreads();
-    int cnt = 0;
-#pragma unroll 1
-    for (int q = 0; q < kPer; ++q) cnt += __popc(bm[t * kPer + q]);
-    int incl = cnt;
+  const float2 li = __ldcg(P.grange + (int64_t)g * G + jh);
+  index_query<G>(P, b, kvh, qidx, tmp);
+  float2 qi[G][kR / 2];
 #pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int y = __shfl_up_sync(0xffffffffu, incl, o);
-      if (lane >= o) incl += y;
-    }
-    if (lane == 31) wsum[warp] = incl;
-    __syncthreads();
-    int before = 0, total = 0;
-    for (int w = 0; w < kThreads / 32; ++w) { before += w < warp ? wsum[w] : 0; total += wsum[w]; }
-    int o = base + before + incl - cnt;
+  for (int hh = 0; hh < G; ++hh)
+#pragma unroll
+    for (int jj = 0; jj < kR / 2; ++jj)
+      qi[hh][jj] = make_float2(qidx[hh * kR + 2 * jj], qidx[hh * kR + 2 * jj + 1]);
+  const unsigned char* src = (const unsigned char*)(
+      P.cache.idx + ((int64_t)slot * P.L.T_total + P.cache.seq_off[b]) * kR);
+  int base = 0, par = 0;
 #pragma unroll 1
-    for (int q = 0; q < kPer; ++q) {
-      uint32_t word = bm[t * kPer + q];
-      while (word) {
-        const int bit = __ffs(word) - 1;
-        word &= word - 1;
-        dst[o++] = w0 + (t * kPer + q) * 32 + bit;
-      }
+  for (int i0 = 0; i0 < N; i0 += kFThreads) {
+    const int n = i0 + t;
+    bool keep = false;
+    if (n < N) {
+      float y[G];
+      score_row<G>(qi, src + (int64_t)n * 32, y);
+      const int bb = li.y > 0.f ? bin_of(y[jh], li.x, li.y) : 0;
+      keep = bb >= bst;
     }
+    int before, total;
+    block_flag_prefix_impl(keep, wc + par * 16, before, total);
+    par ^= 1;
+    if (keep) dst[base + before] = n;
     base += total;
-    __syncthreads();
   }
 }
 
