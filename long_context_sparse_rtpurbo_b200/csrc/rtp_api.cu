@@ -35,8 +35,8 @@ struct Plan {
   int C_min, max_nch, NC_max, n_groups, n_lgroups, n_loc_items;
   int64_t cand_stride;
   size_t off_ctrl, ctrl_bytes;
-  size_t off_bar, off_team, off_locarr, off_misc, off_hist, off_hcnt;
-  size_t off_bstar, off_cstat, off_grange, off_sellist, off_part, off_tpart, off_lpart,
+  size_t off_bar, off_locarr, off_misc, off_hist, off_hcnt;
+  size_t off_bstar, off_cstat, off_grange, off_sellist, off_part, off_lpart,
       off_trace, total;
 };
 
@@ -101,22 +101,20 @@ int make_plan(const rtp_layer_desc* d, Plan& pl) {
   // is made at launch, see local_split)
   const int64_t loc_rows = std::min<int64_t>(maxN, L.ring);
   pl.n_loc_items = (int)(int64_t(pl.n_lgroups) * ((loc_rows + 63) / 64));
-  const size_t part_bytes = sizeof(float) * G * (kD + 2);
+  const size_t part_bytes = size_t((8 * G + 15) / 16 * 16 + 2 * G * kD);   // Part<G>::kBytes
   size_t o = 256;                                   // [0, 256): status word
   pl.off_ctrl = o;
   pl.off_bar = o;    o = align256(o + sizeof(uint32_t) * pl.n_groups * 4);
-  pl.off_team = o;   o = align256(o + sizeof(uint32_t) * pl.NC_max);
   pl.off_locarr = o; o = align256(o + sizeof(uint32_t) * std::max(pl.n_lgroups, 1));
   pl.off_misc = o;   o = align256(o + sizeof(uint32_t) * 16);
-  pl.off_hist = o;   o = align256(o + sizeof(unsigned long long) * pl.n_groups * G * kBins);
-  pl.off_hcnt = o;   o = align256(o + sizeof(int32_t) * pl.n_groups * G);
   pl.ctrl_bytes = o - pl.off_ctrl;
+  pl.off_hist = o;   o = align256(o + sizeof(unsigned long long) * pl.n_groups * G * kBins * kHistPad);
+  pl.off_hcnt = o;   o = align256(o + sizeof(int32_t) * pl.n_groups * G);
   pl.off_bstar = o;  o = align256(o + sizeof(int32_t) * pl.n_groups * G);
   pl.off_cstat = o;  o = align256(o + 16 * size_t(pl.n_groups) * pl.max_nch * G);
   pl.off_grange = o; o = align256(o + 8 * size_t(pl.n_groups) * G);
   pl.off_sellist = o; o = align256(o + sizeof(uint32_t) * size_t(pl.n_groups) * pl.cand_stride);
   pl.off_part = o;   o = align256(o + part_bytes * pl.NC_max);
-  pl.off_tpart = o;  o = align256(o + part_bytes * pl.NC_max);
   pl.off_lpart = o;  o = align256(o + part_bytes * std::max(pl.n_loc_items, 1));
 #ifdef RTP_TRACE
   pl.off_trace = o;  o = align256(o + sizeof(unsigned long long) * kPlanCTAs * kTraceEvents);
@@ -168,9 +166,10 @@ void local_split(const LayerShape& L, int n_lgroups, int n_ret, int P, int& PL, 
 }
 
 // Shared-memory layout of the decode kernel: the staging region (index ring, tiles, merge
-// buffers, gather lists), then the small arrays. The kept scores of a CTA's last chunk live in
-// tensor memory (C_cap rows). Returns the bytes, or -1 when the staging region would be too
-// small for the index ring.
+// buffers; at its end the per-warp lists and row masks of phase W and the candidate queues of
+// phase H), then the small arrays. The kept scores of a CTA's chunks live in tensor memory
+// (C_cap rows per CTA). Returns the bytes, or -1 when the staging region would be too small
+// for the index ring and the tails.
 int smem_layout(DecodeParams& P, const Plan& pl, int smem_optin) {
   const int G = P.L.G;
   int small = 0;
@@ -180,15 +179,15 @@ int smem_layout(DecodeParams& P, const Plan& pl, int smem_optin) {
   small += align16(8 * G * kHistStride);                // hist (two 32-bit words per bin)
   small += align16(4 * G * (kD + 2));                   // res
   small += align16(8 * kFThreads);                      // tmp
-  small += align16(4 * 128);                            // ints
+  small += align16(4 * kIntsWords);                     // ints
   small += align16(4 * P.L.B);                          // N
   small += align16(4 * (pl.n_groups + 1));              // cbase
   small += align16(8 * kMaxSteps * G);                  // tcache
-  small += align16(8 * kMaxSteps * G);                  // lcache
+  small += align16(16 * kMaxSteps * G);                 // lcache
   const int budget = smem_optin - 1024;
   const int stage = (budget - small) / 1024 * 1024;
-  if (stage < DecodeCta<1>::kSRows * 32 * DecodeCta<1>::kSStages) return -1;
-  P.C_cap = kTmemColsPerThread / G * DecodeCta<1>::kSRows;
+  if (stage < kStageBytes * kSStages + kTailMax) return -1;   // ring + phase H/W tails
+  P.C_cap = kTmemColsPerThread / (G == 8 ? 8 : 4) * kSRows;
   int o = 0;
   P.sm_stage = o; o += stage;
   P.free_bytes = o;
@@ -198,11 +197,11 @@ int smem_layout(DecodeParams& P, const Plan& pl, int smem_optin) {
   P.sm_hist = o;  o += align16(8 * G * kHistStride);
   P.sm_res = o;   o += align16(4 * G * (kD + 2));
   P.sm_tmp = o;   o += align16(8 * kFThreads);
-  P.sm_int = o;   o += align16(4 * 128);
+  P.sm_int = o;   o += align16(4 * kIntsWords);
   P.sm_N = o;     o += align16(4 * P.L.B);
   P.sm_cbase = o; o += align16(4 * (pl.n_groups + 1));
   P.sm_tcache = o; o += align16(8 * kMaxSteps * G);
-  P.sm_lcache = o; o += align16(8 * kMaxSteps * G);
+  P.sm_lcache = o; o += align16(16 * kMaxSteps * G);
   return o;
 }
 
@@ -401,7 +400,6 @@ int decode_impl(const rtp_layer_desc* desc, const rtp_cache* cache, const uint16
   P.out = out; P.sel_counts = sel_counts;
   P.status = at<int>(ws, 0);
   P.bar = at<uint32_t>(ws, pl.off_bar);
-  P.team_arr = at<uint32_t>(ws, pl.off_team);
   P.loc_arr = at<uint32_t>(ws, pl.off_locarr);
   P.misc = at<uint32_t>(ws, pl.off_misc);
   P.hist = at<unsigned long long>(ws, pl.off_hist);
@@ -410,9 +408,8 @@ int decode_impl(const rtp_layer_desc* desc, const rtp_cache* cache, const uint16
   P.cstat = at<float4>(ws, pl.off_cstat);
   P.grange = at<float2>(ws, pl.off_grange);
   P.sellist = at<uint32_t>(ws, pl.off_sellist);
-  P.part = at<float>(ws, pl.off_part);
-  P.tpart = at<float>(ws, pl.off_tpart);
-  P.lpart = at<float>(ws, pl.off_lpart);
+  P.part = at<unsigned char>(ws, pl.off_part);
+  P.lpart = at<unsigned char>(ws, pl.off_lpart);
   P.trace = pl.off_trace ? at<unsigned long long>(ws, pl.off_trace) : nullptr;
   if (cudaMemsetAsync(at<char>(ws, pl.off_ctrl), 0, pl.ctrl_bytes, st) != cudaSuccess)
     return RTP_ECUDA;

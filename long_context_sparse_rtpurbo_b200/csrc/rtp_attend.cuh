@@ -17,6 +17,8 @@
 // synchronisation inside the loop is __syncwarp.
 #pragma once
 
+#include <cuda_fp16.h>
+
 #include "rtp_common.cuh"
 
 namespace rtp {
@@ -27,6 +29,15 @@ __device__ __forceinline__ uint32_t smem_u32(const void* p) {
 __device__ __forceinline__ void cp_async16(void* smem, const void* gmem) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(smem)), "l"(gmem)
                : "memory");
+}
+__device__ __forceinline__ void cp_async16_s(uint32_t saddr, const void* gmem) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(saddr), "l"(gmem) : "memory");
+}
+__device__ __forceinline__ void st_shared_zero16(uint32_t saddr) {
+  asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(saddr), "r"(0u) : "memory");
+}
+__device__ __forceinline__ void st_shared_u32(uint32_t saddr, uint32_t v) {
+  asm volatile("st.shared.u32 [%0], %1;" ::"r"(saddr), "r"(v) : "memory");
 }
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 template <int N>
@@ -324,69 +335,143 @@ __device__ __forceinline__ void attn_end(WarpAttn& W, int nwa, float* res, float
   __syncthreads();
 }
 
-// Largest number of partial states one merge combines (the host plan sizes splits by it).
-constexpr int kMaxMerge = 64;
-
-// Merges n partial states (contiguous in global memory, stride G*(2+128) floats, written by
-// other CTAs) into `dst` (same format) or, when out_rows is given, into the bf16 output rows
-// of the G heads. The partials are first copied into shared memory (buf, buf_bytes) with
-// cp.async, as many per batch as fit, so all loads of a batch are in flight together; each
-// thread then folds its output channels over the batch with the online softmax rule.
+// Partial softmax state of the G heads in global memory: per head (m, L) as floats (the
+// block padded to 16 bytes), then per head the 128 normalised outputs A / L as fp16 (0 for a
+// partial without rows).
 template <int G>
-__device__ __forceinline__ void merge_partials(const float* parts, int n, float* dst,
-                                               uint16_t* out_rows, float* buf, int buf_bytes,
-                                               int nthreads) {
-  constexpr int S = G * (kD + 2);                    // floats per partial
-  constexpr int kPer = (G * kD + 511) / 512;         // outputs per thread for 512 threads
-  const int per = max(1, buf_bytes / (S * 4));       // partials per batch
-  const int t = threadIdx.x;
-  float M[kPer], Ls[kPer], A[kPer];
+struct Part {
+  static constexpr int kMLBytes = (8 * G + 15) / 16 * 16;
+  static constexpr int kBytes = kMLBytes + 2 * G * kD;
+};
+
+// res[G][130] (m, L, A) in shared memory -> the partial at dst. Every thread of the CTA
+// calls it (NT threads).
+template <int G, int NT>
+__device__ __forceinline__ void write_partial(const float* res, unsigned char* dst) {
+  float* ml = reinterpret_cast<float*>(dst);
+  __half* o = reinterpret_cast<__half*>(dst + Part<G>::kMLBytes);
+  for (int i = threadIdx.x; i < G * kD; i += NT) {
+    const int h = i / kD, c = i % kD;
+    const float L = res[h * (kD + 2) + 1];
+    o[i] = __float2half_rn(L > 0.f ? res[h * (kD + 2) + 2 + c] / L : 0.f);
+    if (c == 0) { ml[2 * h] = res[h * (kD + 2)]; ml[2 * h + 1] = L; }
+  }
+}
+
+// Merges n partials (contiguous in global memory, Part<G>::kBytes each, written by other
+// CTAs) into the bf16 output rows of the G heads: with M = max_i m_i per head and weights
+// w_i = 2^(m_i - M) L_i, O = sum_i w_i O_i / sum_i w_i. When the n partials fit in buf they
+// are copied into shared memory with cp.async, all copies in flight at once, and everything
+// is read from there: warp h finds M, the weights and their sum for head h (lanes over the
+// partials, a fixed butterfly for the sum), then every thread sums its output channels (four
+// running sums, added in a fixed order). Otherwise the partials are processed in batches,
+// M and the sum of the weights first from global memory. A partial without rows has
+// m = -inf and weight 0. sml: G floats of shared memory. Every thread of the CTA calls it;
+// NT threads.
+template <int G, int NT>
+__device__ __forceinline__ void merge_all(const unsigned char* parts, int n, uint16_t* out_rows,
+                                          unsigned char* buf, int buf_bytes, float* sml) {
+  constexpr int PB = Part<G>::kBytes, ML = Part<G>::kMLBytes;
+  constexpr int kPer = (G * kD + NT - 1) / NT;       // outputs per thread
+  const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
+  const int per = max(1, buf_bytes / (PB + 4 * G));  // partials per batch (data + weights)
+  float* wbuf = reinterpret_cast<float*>(buf + per * PB);
+  const bool one = n <= per;
+  {
+    const int nb = min(per, n);
+    for (int i = t; i < nb * (PB / 16); i += NT) cp_async16(buf + 16 * i, parts + 16 * i);
+    cp_async_commit();
+  }
+  if (one) {
+    cp_async_wait<0>();
+    __syncthreads();
+    if (warp < G) {
+      float m = -INFINITY;
+      for (int i = lane; i < n; i += 32)
+        m = fmaxf(m, reinterpret_cast<const float*>(buf + i * PB)[2 * warp]);
 #pragma unroll
-  for (int u = 0; u < kPer; ++u) { M[u] = -INFINITY; Ls[u] = 0.f; A[u] = 0.f; }
+      for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+      float W = 0.f;
+      for (int i = lane; i < n; i += 32) {
+        const float* ml = reinterpret_cast<const float*>(buf + i * PB);
+        const float w = ml[2 * warp] == -INFINITY ? 0.f : exp2f(ml[2 * warp] - m) * ml[2 * warp + 1];
+        wbuf[i * G + warp] = w;
+        W += w;
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) W += __shfl_xor_sync(0xffffffffu, W, o);
+      if (lane == 0) sml[warp] = W;
+    }
+  } else if (warp < G) {
+    float m = -INFINITY;
+    for (int i = lane; i < n; i += 32)
+      m = fmaxf(m, __ldcg(reinterpret_cast<const float*>(parts + (int64_t)i * PB) + 2 * warp));
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    float W = 0.f;
+    for (int i = lane; i < n; i += 32) {
+      const float* ml = reinterpret_cast<const float*>(parts + (int64_t)i * PB);
+      const float mi = __ldcg(ml + 2 * warp);
+      if (mi != -INFINITY) W += exp2f(mi - m) * __ldcg(ml + 2 * warp + 1);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) W += __shfl_xor_sync(0xffffffffu, W, o);
+    if (lane == 0) { sml[warp] = W; sml[G + warp] = m; }
+  }
+  float acc[kPer][4];
+#pragma unroll
+  for (int u = 0; u < kPer; ++u)
+#pragma unroll
+    for (int k = 0; k < 4; ++k) acc[u][k] = 0.f;
 #pragma unroll 1
   for (int b0 = 0; b0 < n; b0 += per) {
     const int nb = min(per, n - b0);
-    __syncthreads();                                 // the buffer is free
-    const float* src = parts + (int64_t)b0 * S;
-    if constexpr (S % 4 == 0) {                      // 16-byte partials (G >= 2): cp.async
-      for (int i = t; i < nb * (S / 4); i += nthreads) cp_async16(buf + 4 * i, src + 4 * i);
-      cp_async_commit();
+    if (!one) {
+      if (b0 > 0) {
+        for (int i = t; i < nb * (PB / 16); i += NT)
+          cp_async16(buf + 16 * i, parts + (int64_t)b0 * PB + 16 * i);
+        cp_async_commit();
+      }
+      __syncthreads();                               // sml (first batch) is ready
+      for (int idx = t; idx < nb * G; idx += NT) {
+        const int i = idx / G, h = idx % G;
+        const float* ml = reinterpret_cast<const float*>(parts + (int64_t)(b0 + i) * PB);
+        const float M = sml[G + h], mi = __ldcg(ml + 2 * h);
+        wbuf[idx] = (mi == -INFINITY || M == -INFINITY) ? 0.f : exp2f(mi - M) * __ldcg(ml + 2 * h + 1);
+      }
       cp_async_wait<0>();
-    } else {                                         // G = 1: 520-byte partials, plain loads
-      for (int i = t; i < nb * S; i += nthreads) buf[i] = __ldcg(src + i);
     }
     __syncthreads();
+    const __half* ob = reinterpret_cast<const __half*>(buf + ML);
 #pragma unroll
     for (int u = 0; u < kPer; ++u) {
-      const int o = t + u * nthreads;
-      if (o >= G * kD) break;
-      const int h = o / kD, dch = o % kD;
+      const int o = t + u * NT;
+      if (o < G * kD) {
+        const int h = o / kD;
+        const __half* src = ob + o;
+        int i = 0;
 #pragma unroll 1
-      for (int i = 0; i < nb; ++i) {
-        const float* pp = buf + i * S + h * (kD + 2);
-        const float mi = pp[0];
-        if (mi == -INFINITY) continue;               // a split without rows
-        const float mn = fmaxf(M[u], mi);
-        const float fo = exp2f(M[u] - mn), fi = exp2f(mi - mn);   // exp2(-inf) = 0
-        A[u] = A[u] * fo + pp[2 + dch] * fi;
-        Ls[u] = Ls[u] * fo + pp[1] * fi;
-        M[u] = mn;
+        for (; i + 4 <= nb; i += 4) {
+#pragma unroll
+          for (int k = 0; k < 4; ++k)
+            acc[u][k] = fmaf(__half2float(src[(i + k) * (PB / 2)]), wbuf[(i + k) * G + h], acc[u][k]);
+        }
+        for (; i < nb; ++i) acc[u][0] = fmaf(__half2float(src[i * (PB / 2)]), wbuf[i * G + h], acc[u][0]);
       }
     }
+    __syncthreads();                                 // buf is rewritten by the next batch
   }
 #pragma unroll
   for (int u = 0; u < kPer; ++u) {
-    const int o = t + u * nthreads;
-    if (o >= G * kD) break;
-    const int h = o / kD, dch = o % kD;
-    if (out_rows) {
-      out_rows[(int64_t)h * kD + dch] = f2bf_rn(Ls[u] > 0.f ? A[u] / Ls[u] : 0.f);
-    } else {
-      dst[h * (kD + 2) + 2 + dch] = A[u];
-      if (dch == 0) { dst[h * (kD + 2)] = M[u]; dst[h * (kD + 2) + 1] = Ls[u]; }
+    const int o = t + u * NT;
+    if (o < G * kD) {
+      const int h = o / kD;
+      const float A = (acc[u][0] + acc[u][1]) + (acc[u][2] + acc[u][3]);
+      const float W = sml[h];
+      out_rows[o] = f2bf_rn(W > 0.f ? A / W : 0.f);
     }
   }
-  __syncthreads();                                   // the caller may reuse the buffer
+  __syncthreads();                                   // the caller may reuse buf and sml
 }
 
 }  // namespace rtp

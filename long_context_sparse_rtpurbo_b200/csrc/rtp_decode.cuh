@@ -13,21 +13,23 @@
 // heads at once, P_ret following the byte share of the two sides). Per group the chunks pass
 // three phases, separated by arrival counters in global memory (two device-wide
 // dependencies):
-//   S  the chunk's index rows are streamed once from HBM; G scores per row (in log2 units:
-//      the index query carries log2(e)); per-chunk (min, max, sum 2^(y - max)) per head. The
-//      CTA's last chunk keeps its scores in shared memory; the scores of earlier chunks are
-//      recomputed from the index rows, which are still in L2, when their phase H comes.
+//   S  the chunk's index rows are streamed once from HBM, each warp through its own slots of
+//      a ring (no block barrier per stage), and scored on the tensor cores, 32 rows per warp
+//      tile, in log2 units (the index query carries log2(e)); per-chunk (min, max,
+//      sum 2^(y - max)) per head. The scores stay in tensor memory as long as its columns
+//      last; later chunks of the CTA recompute them from the index rows when needed.
 //   H  from the group's (min, max, total mass): the 256 linear bins and a cutoff bin under
-//      which no token can be selected (their total mass is below (1 - p) of the total); per
-//      bin fixed-point masses of the tokens at or above the cutoff go to the group's
-//      histogram (exact 64-bit sums), and these tokens are emitted as candidates with their
-//      bins, in token order. Phase H of a group runs after phase S of the CTA's next group,
-//      which hides the wait for the other chunks.
-//   W  b* per head from the group's histogram; the group's candidates are split evenly over
-//      at most kTeam of the chunks' CTAs; each keeps the candidates with bin >= b* for some
-//      head, gathers their K/V rows once for all G heads (tensor-core tiles, a head that did
-//      not select a row masks it) and writes a partial softmax state; the last split merges
-//      them into the output rows and the selected counts.
+//      which no token can be selected (their total mass is below (1 - p) of the total). A
+//      score reaches a bin exactly when it reaches the bin's lower edge, found once per head
+//      by bisection over the floats, so the test per score is one compare; the scores at or
+//      above the cutoff are compacted per warp and added (fixed-point masses) to the group's
+//      histogram (exact integer sums). Phase H of a group runs after phase S of the CTA's
+//      next group, which hides the wait for the other chunks.
+//   W  b* per head from the group's histogram; each chunk selects its rows with a score at
+//      or above the edge of b* for some head (per-warp compaction, batches of 8 stages),
+//      gathers their K/V rows once for all G heads (tensor-core tiles, a head that did not
+//      select a row masks it) and writes a partial softmax state; the last chunk to finish
+//      merges all partials of the group into the output rows and the selected counts.
 // Local items (a slice of one local head's ring) come from a global queue; the chunk CTAs
 // drain it when their chunks are done.
 // Every wait is bounded (clock64 limit): on expiry the kernel records RTP_ETIMEOUT, raises
@@ -36,17 +38,33 @@
 
 #include "rtp_append.cuh"
 #include "rtp_attend.cuh"
+#include "rtp_score.cuh"
 #include "rtp_tmem.cuh"
 
 namespace rtp {
 
 constexpr int kFThreads = 512;          // threads of the decode kernel
-constexpr int kTeam = 32;               // partials merged per team (gather splits per group)
+constexpr int kWarps = kFThreads / 32;
 constexpr int kHeadPad = 8;             // words between the heads' rows of shared buffers
 constexpr int kHistStride = 256 + kHeadPad;
-constexpr int kSplitRows = 64;          // fewest candidates per gather split
 constexpr int kMaxSteps = 32;           // chunks per CTA, upper bound
-constexpr int kListCap = 4096;          // gather entries staged per batch
+constexpr int kSRows = kWarps * kWRows; // index rows per stage (one 32-row tile per warp)
+constexpr int kSStages = 8;             // ring depth (stages in flight: kSStages - 1)
+constexpr int kSlotBytes = kWRows * 32; // one warp's slot of a stage
+constexpr int kStageBytes = kSRows * 32;
+constexpr int kWBatch = 16;             // stages per selection batch of phase W
+constexpr int kHistPad = 4;             // u64 words per bin of the global histogram: one
+                                        // 32-byte sector per bin spreads the CTAs' atomic
+                                        // adds over more L2 lines
+constexpr int kWListCap = kWBatch * kWRows;           // list entries per warp and batch
+constexpr int kHQueueMax = 32 * 9;      // per-warp candidate queue of phase H (entries)
+constexpr int kIntsWords = 256;         // words of the shared ints[] array
+// tail of the staging region (bytes back from its end): phase W's lists and row-mask bytes,
+// phase H's candidate queues (different phases, so they may overlap)
+constexpr int kTailList = kWarps * kWListCap * 4;
+constexpr int kTailRm = kTailList + kWarps * kWRows * 8;
+constexpr int kTailHq = kWarps * kHQueueMax * 8;
+constexpr int kTailMax = kTailHq > kTailRm ? kTailHq : kTailRm;
 
 struct DecodeParams {
   LayerShape L;
@@ -81,19 +99,18 @@ struct DecodeParams {
   int32_t* sel_counts;
   // workspace
   int* status;
-  uint32_t* bar;               // [n_groups][4]  S arrivals, H arrivals, teams done  (zeroed)
-  uint32_t* team_arr;          // [NC_max]       team arrivals                      (zeroed)
+  uint32_t* bar;               // [n_groups][4]  S arrivals, H arrivals, W arrivals     (zeroed)
   uint32_t* loc_arr;           // [n_lgroups]    local item arrivals                (zeroed)
   uint32_t* misc;              // [0] local queue head, [1] abort, [2] chunk size     (zeroed)
-  unsigned long long* hist;    // [n_groups][G][256] fixed-point bin masses          (zeroed)
-  int32_t* hcnt;               // [n_groups][G]  selected tokens per head            (zeroed)
+  unsigned long long* hist;    // [n_groups][G][256][kHistPad] fixed-point bin masses (word 0;
+                               //   zeroed by the group's first chunk in phase S)
+  int32_t* hcnt;               // [n_groups][G]  selected tokens per head (zeroed likewise)
   int32_t* bstar;              // [n_groups][G]  threshold bins (debug output)
   float4* cstat;               // [n_groups][max_nch][G]  chunk (min, max, sum 2^(y - max))
   float2* grange;              // [n_groups][G]  group (min score, 256 / (max - min)), debug output
   uint32_t* sellist;           // [n_groups][cand_stride] selected rows of recomputed chunks
-  float* part;                 // [NC_max][G][130]
-  float* tpart;                // [NC_max][G][130]
-  float* lpart;                // [n_loc_items][G][130]
+  unsigned char* part;         // [NC_max] partials (Part<G>::kBytes each)
+  unsigned char* lpart;        // [n_loc_items] partials
   unsigned long long* trace;   // [P][kTraceEvents] %globaltimer stamps (tracing builds only)
 };
 
@@ -101,7 +118,7 @@ struct DecodeParams {
 // Each event keeps its last occurrence; kEvNLocWait / kEvNLocDrain count local items.
 enum TraceEvent { kEvStart, kEvPlan, kEvS0, kEvS1, kEvH0, kEvHw, kEvH1, kEvW0, kEvW1, kEvW2,
                   kEvW3, kEvLoc0, kEvLoc1, kEvDrain, kEvEnd, kEvNLocWait, kEvNLocDrain,
-                  kEvHs, kEvWl, kTraceEvents = 32 };
+                  kEvHs, kEvWl, kEvWb, kEvWh, kTraceEvents = 32 };
 
 // ------------------------------------------------------------------------------ helpers
 __device__ __forceinline__ int seq_len_checked(const DecodeParams& P, int b) {
@@ -188,13 +205,6 @@ extern __shared__ __align__(16) unsigned char rtp_smem[];
 template <class T>
 __device__ __forceinline__ T* smem_at(int off) { return reinterpret_cast<T*>(rtp_smem + off); }
 
-__device__ __forceinline__ void block_flag_prefix_impl(bool flag, int* w, int& before,
-                                                       int& total);
-__device__ __forceinline__ void block_flag_prefix(bool flag, int wc_off, int par, int& before,
-                                                  int& total) {
-  block_flag_prefix_impl(flag, smem_at<int>(wc_off) + par * 16, before, total);
-}
-
 template <int G> struct Smem {
   const DecodeParams& P;
   __device__ explicit Smem(const DecodeParams& p) : P(p) {}
@@ -209,12 +219,15 @@ template <int G> struct Smem {
   __device__ int* N() const { return (int*)(rtp_smem + P.sm_N); }
   __device__ int* cbase() const { return (int*)(rtp_smem + P.sm_cbase); }
   __device__ double* tcache() const { return (double*)(rtp_smem + P.sm_tcache); }
-  __device__ float2* lcache() const { return (float2*)(rtp_smem + P.sm_lcache); }
+  __device__ float4* lcache() const { return (float4*)(rtp_smem + P.sm_lcache); }
 };
 // ints[]: [0..31] reduction scratch, [32] wait flag, [33] next local item, [36] last-split
 //         flag, [38] local-last flag, [40..47] b*, [48..55] decode token's index row
-//         (16 bf16), [60] tensor-memory base, [64..95] per-warp counts of ordered
-//         compactions (two blocks of 16), [96..127] tensor-memory column of each chunk
+//         (16 bf16), [60] tensor-memory base, [96..127] tensor-memory column of each chunk,
+//         [128..144] prefix of the per-warp list counts, [160..167] selected rows per head,
+//         [176..183] (float) per-head score edge of the cutoff / threshold bin,
+//         [192..223] (float4) per-head lo, 256 / (hi - lo), hi
+constexpr int kIntPre = 128, kIntCnt = 160, kIntEdge = 176, kIntHp = 192;
 
 // RoPE'd, pre-scaled query of the G heads of KV head kvh at position N - 1 -> q_s[G][128].
 template <int G>
@@ -266,12 +279,8 @@ __device__ __forceinline__ void index_query(const DecodeParams& P, int b, int kv
 
 // Every thread gets the number of set flags among the CTA's threads before its own (in
 // thread order) and the block total, for an ordered compaction of one block of kFThreads
-// items. wc: two arrays of 16 ints used alternately (par = block parity), so one barrier
-// per block suffices.
-__device__ __forceinline__ void block_flag_prefix(bool flag, int wc_off, int par, int& before,
-                                                  int& total);
-__device__ __forceinline__ void block_flag_prefix_impl(bool flag, int* w, int& before,
-                                                       int& total) {
+// items. w: one of two arrays of 16 ints used alternately, so one barrier per block suffices.
+__device__ __forceinline__ void block_flag_prefix(bool flag, int* w, int& before, int& total) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const uint32_t bal = __ballot_sync(0xffffffffu, flag);
   if (lane == 0) w[warp] = __popc(bal);
@@ -289,29 +298,42 @@ __device__ __forceinline__ void block_flag_prefix_impl(bool flag, int* w, int& b
   before = upto - mine + __popc(bal & ((1u << lane) - 1u));
 }
 
-// G scores of one 32-byte index row (channel pairs in packed f32x2 multiply-adds, even and
-// odd channel sums added at the end). Phases S and H call this same routine, so a recomputed
-// score is bit-identical to the first one.
-template <int G>
-__device__ __forceinline__ void score_row(const float2 (&qi)[G][kR / 2], const unsigned char* row,
-                                          float (&s)[G]) {
-  const uint4 a = *reinterpret_cast<const uint4*>(row);
-  const uint4 c2 = *reinterpret_cast<const uint4*>(row + 16);
-  const uint32_t w[8] = {a.x, a.y, a.z, a.w, c2.x, c2.y, c2.z, c2.w};
-  float2 x[kR / 2];
-#pragma unroll
-  for (int jj = 0; jj < kR / 2; ++jj) x[jj] = make_float2(bf_lo(w[jj]), bf_hi(w[jj]));
-#pragma unroll
-  for (int h = 0; h < G; ++h) {
-    float2 a2 = __fmul2_rn(qi[h][0], x[0]);
-#pragma unroll
-    for (int jj = 1; jj < kR / 2; ++jj) a2 = __ffma2_rn(qi[h][jj], x[jj], a2);
-    s[h] = a2.x + a2.y;
-  }
-}
-
 __device__ __forceinline__ int bin_of(float s, float lo, float inv) {
   return min(kBins - 1, (int)((s - lo) * inv));
+}
+
+// Lower edge of bin b as a score: the smallest float y in [lo, hi] with bin_of(y) >= b
+// (-inf for b <= 0). bin_of is non-decreasing in y (a rounded subtraction, a rounded product
+// with inv > 0, truncation), so for every score y in [lo, hi]: bin_of(y) >= b <=> y >= edge.
+// Warp-collective search over the order-preserving integer images of the floats in
+// (lo, hi]: the lanes test 32 candidates per round, first the 32 floats around the rounded
+// guess lo + b / inv, then 32-way splits of the remaining interval (a, z] with
+// bin_of(a) < b <= bin_of(z), until it holds one float. Every lane returns the edge.
+__device__ __forceinline__ float bin_edge_warp(int b, float lo, float hi, float inv) {
+  if (b <= 0) return -INFINITY;
+  if (!(inv > 0.f) || bin_of(hi, lo, inv) < b) return INFINITY;
+  const int lane = threadIdx.x & 31;
+  uint32_t a = f2ord(lo), z = f2ord(hi);                      // bin_of(lo) = 0 < b
+  const uint32_t g = f2ord(fminf(fmaxf(lo + (float)b / inv, lo), hi));
+  uint32_t base = g > a + 16u ? g - 16u : a + 1u, step = 1u;
+#pragma unroll 1
+  for (int round = 0; round < 16 && z - a > 1u; ++round) {
+    const uint64_t c64 = (uint64_t)base + (uint64_t)step * (uint32_t)lane;
+    const uint32_t c = c64 >= (uint64_t)z ? z : (c64 <= (uint64_t)a ? a + 1u : (uint32_t)c64);
+    const bool up = bin_of(ord2f(c), lo, inv) >= b;
+    const uint32_t bal = __ballot_sync(0xffffffffu, up);   // a suffix of the lanes
+    if (bal) z = min(z, __shfl_sync(0xffffffffu, c, __ffs(bal) - 1));
+    if (~bal) a = max(a, __shfl_sync(0xffffffffu, c, 31 - __clz(~bal)));
+    step = max(1u, (z - a) / 32u);
+    base = a + step;
+  }
+  return ord2f(z);
+}
+
+__device__ __forceinline__ float ex2_approx(float x) {
+  float r;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
+  return r;
 }
 
 // ------------------------------------------------------------------------------ kernel
@@ -449,168 +471,269 @@ struct DecodeCta {
     __syncthreads();
   }
 
-  // ------------------------------------------------------------ index streaming
-  // The chunk's index rows (32 B each, contiguous) stream through a ring of kSStages stages
-  // of kSRows rows in the staging region with cp.async (seven stages, 112 KB, in flight);
-  // thread t takes row t of each stage and calls fn(nl, ok, y[G]) with its G scores (nl: row
-  // within the chunk; ok: the row exists). Every thread calls fn for every stage.
-  static constexpr int kSRows = 512, kSStages = 8;
-  __device__ __forceinline__ void stream_issue(unsigned char* stage, const unsigned char* src,
-                                               int st, int nst, int len) {
+  // ------------------------------------------------------------ chunks and streaming
+  // Chunk j of a group with nc chunks is the set of its 32-row tiles j, j + nc, j + 2 nc, ...
+  // (of the group's ceil(N / 32) tiles): interleaved, so a run of selected tokens is spread
+  // over many chunks (and CTAs). In local stage st, warp w takes the chunk's tile 16 st + w.
+  __device__ __forceinline__ static int chunk_tiles(int N, int nc, int j) {
+    return ((N + kWRows - 1) / kWRows - j + nc - 1) / nc;
+  }
+  __device__ __forceinline__ static int chunk_stages(int N, int nc, int j) {
+    return (chunk_tiles(N, nc, j) + kWarps - 1) / kWarps;
+  }
+  // first group row of the tile of warp w in local stage st (N when the warp has none)
+  __device__ __forceinline__ static int tile_row(int N, int nc, int j, int ntl, int st, int w) {
+    const int i = st * kWarps + w;
+    return i < ntl ? (j + i * nc) * kWRows : N;
+  }
+
+  // The chunk's index rows stream through a ring of kSStages stages; warp w copies its tile
+  // of each stage itself into its 1 KB slot (cp.async, two 16-byte pieces per lane, the
+  // halves of rows 4..7 mod 8 swapped; rows past the group end are zeroed) and scores it on
+  // the tensor cores, so a stage needs no block barrier. fn(st, rb, c, T) gets the warp's tile
+  // scores (rb: group row of the tile's row 0, N when the warp has no tile this stage; rows
+  // at or past N score 0 and are masked by the callers).
+  __device__ __forceinline__ void slot_issue(uint32_t ring, const unsigned char* src, int st,
+                                             int nst, int N, int nc, int j, int ntl) {
     if (st < nst) {
-      unsigned char* dst = stage + (st % kSStages) * (kSRows * 32);
-      const int rows = min(kSRows, len - st * kSRows);
-      for (int piece = threadIdx.x; piece < rows * 2; piece += kFThreads)
-        cp_async16(dst + piece * 16, src + ((int64_t)st * kSRows * 32) + piece * 16);
+      const int lane = threadIdx.x & 31;
+      const int rb = tile_row(N, nc, j, ntl, st, threadIdx.x >> 5);
+      const uint32_t slot = ring + (st % kSStages) * kStageBytes;
+#pragma unroll
+      for (int u = 0; u < 2; ++u) {
+        const int p = lane + 32 * u, r = p >> 1, hh = p & 1;
+        if (rb + r < N)
+          cp_async16_s(slot + idx_half_off(r, hh), src + (int64_t)(rb + r) * 32 + hh * 16);
+        else      // zero rows: a stale inf or NaN times a zero query column would poison the
+                  // other half-tile's scores
+          st_shared_zero16(slot + idx_half_off(r, hh));
+      }
     }
     cp_async_commit();
   }
   template <class Fn>
   __device__ __forceinline__ void stream_chunk(int g, int j, bool patch, Fn& fn) {
     const int b = g / P.L.n_ret, r = g % P.L.n_ret, kvh = P.L.ret_kv[r];
-    const int N = gN(g);
-    const int n0 = j * C, n1 = min(N, n0 + C), len = n1 - n0;
+    const int N = gN(g), nc = nch(g);
+    const int ntl = chunk_tiles(N, nc, j), nst = chunk_stages(N, nc, j);
     const unsigned char* src = (const unsigned char*)(
-        P.cache.idx + ((int64_t)r * P.L.T_total + P.cache.seq_off[b] + n0) * kR);
-    const int nst = (len + kSRows - 1) / kSRows;
-    unsigned char* stage = sm.stage();
+        P.cache.idx + ((int64_t)r * P.L.T_total + P.cache.seq_off[b]) * kR);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint32_t ring = smem_u32(sm.stage()) + warp * kSlotBytes;
     __syncthreads();                       // the staging region may still be in use
 #pragma unroll
-    for (int st = 0; st < kSStages - 1; ++st) stream_issue(stage, src, st, nst, len);
+    for (int st = 0; st < kSStages - 1; ++st) slot_issue(ring, src, st, nst, N, nc, j, ntl);
     index_query<G>(P, b, kvh, sm.qidx(), reinterpret_cast<float*>(sm.tmp()));
     // The chunk holding the decode token writes it while the first stages are in flight; a
-    // copy of its index row may still be stale, so the stage holding it is patched below.
+    // copy of its index row may be stale, so the warp holding it patches its slot.
     uint16_t* idx_patch = reinterpret_cast<uint16_t*>(sm.ints() + 48);   // 16 bf16
-    if (patch) append_new(b, kvh, N, idx_patch);
-    float2 qi[G][kR / 2];                    // index query, channel pairs (2j, 2j + 1)
-#pragma unroll
-    for (int h = 0; h < G; ++h)
-#pragma unroll
-      for (int jj = 0; jj < kR / 2; ++jj)
-        qi[h][jj] = make_float2(sm.qidx()[h * kR + 2 * jj], sm.qidx()[h * kR + 2 * jj + 1]);
+    if (patch) {
+      append_new(b, kvh, N, idx_patch);
+      __syncthreads();
+    }
+    ScoreTile<G> T;
+    T.init(sm.qidx());
+    const int prow = patch ? N - 1 : -1;
 #pragma unroll 1
     for (int st = 0; st < nst; ++st) {
-      stream_issue(stage, src, st + kSStages - 1, nst, len);
+      slot_issue(ring, src, st + kSStages - 1, nst, N, nc, j, ntl);
       cp_async_wait<kSStages - 1>();
-      __syncthreads();
-      const int rows = min(kSRows, len - st * kSRows);
-      unsigned char* buf = stage + (st % kSStages) * (kSRows * 32);
-      if (patch && st == nst - 1) {        // the last row of the chunk is the decode token
-        if (threadIdx.x < kR / 2)
-          reinterpret_cast<uint32_t*>(buf + (rows - 1) * 32)[threadIdx.x] =
-              reinterpret_cast<const uint32_t*>(idx_patch)[threadIdx.x];
-        __syncthreads();
+      __syncwarp();
+      const uint32_t slot = ring + (st % kSStages) * kStageBytes;
+      const int rb = tile_row(N, nc, j, ntl, st, warp);
+      if (prow >= rb && prow < rb + kWRows) {
+        const int rr = prow - rb;
+        if (lane < 8)
+          st_shared_u32(slot + idx_half_off(rr, lane >> 2) + (lane & 3) * 4,
+                        reinterpret_cast<const uint32_t*>(idx_patch)[lane]);
+        __syncwarp();
       }
-      const int i = threadIdx.x;
-      float y[G];
-#pragma unroll
-      for (int h = 0; h < G; ++h) y[h] = -INFINITY;
-      if (i < rows) score_row<G>(qi, buf + i * 32, y);
-      fn(st * kSRows + i, i < rows, y);
-      __syncthreads();                     // before the stage is refilled
+      float c[ScoreTile<G>::V];
+      T.score(slot, c);
+      fn(st, rb, c, T);
+      __syncwarp();                        // the slot is refilled by the next issue
     }
     cp_async_wait<0>();
   }
 
-  // Per-row work of phase S. Per head: min, max, and the sum of 2^(y - rf) against a
-  // per-thread reference rf (the first score, moved up only when a score exceeds it by 64, so
-  // the terms never overflow and the common step is one exponential and one add). When the
-  // chunk's scores are kept, each stage's G scores go to G tensor-memory columns of the
-  // thread's lane (a warp-wide store).
-  struct SStats {
-    float mn[G], mx[G], rf[G], ls[G];
-    uint32_t tbase;                // tensor-memory base
-    int col0;                      // first column of this chunk (-1: scores not kept)
-    __device__ __forceinline__ SStats(uint32_t tb, int c) : tbase(tb), col0(c) {
-#pragma unroll
-      for (int k = 0; k < G; ++k) { mn[k] = INFINITY; mx[k] = -INFINITY; rf[k] = -INFINITY; ls[k] = 0.f; }
-    }
-    __device__ __forceinline__ void operator()(int nl, bool ok, const float (&y)[G]) {
-      if (col0 >= 0) Tmem<G>::st(tmem_addr(tbase, col0 + (nl / kSRows) * G), y);   // whole warp
-      if (!ok) return;
-#pragma unroll
-      for (int h = 0; h < G; ++h) {
-        mn[h] = fminf(mn[h], y[h]);
-        mx[h] = fmaxf(mx[h], y[h]);
-        const float d = y[h] - rf[h];
-        if (d > 64.f) {
-          ls[h] = ls[h] * exp2f(-d) + 1.f;
-          rf[h] = y[h];
-        } else {
-          ls[h] += exp2f(d);
-        }
-      }
-    }
-  };
+  static constexpr int V = ScoreTile<G>::V;
 
-  // Per-row work of phase H: for each head whose score reaches ycut (half a bin below the
-  // cutoff bin's edge), the bin; when it reaches the cutoff, the row's fixed-point mass goes
-  // to the shared histogram (two 32-bit words per bin, exact).
-  struct HHist {
-    float lo[G], hi[G], inv[G], ycut[G];
-    int bch[G];
-    int hist_off;                  // byte offset of the histogram words in rtp_smem
-    __device__ __forceinline__ void operator()(int nl, bool ok, const float (&y)[G]) {
-      (void)nl;
-      if (!ok) return;
-      uint32_t* hlo = smem_at<uint32_t>(hist_off);
-      uint32_t* hhi = hlo + G * kHistStride;
+  // Per-tile work of phase S: the scores go to V tensor-memory columns of the lane (when the
+  // chunk's scores are kept); per slot (one head per slot): min, max, and the sum of
+  // 2^(y - rf) against a per-lane reference rf (the first score, moved up only when a score
+  // exceeds it by 64, so the terms never overflow).
+  struct SStats {
+    float mn[2], mx[2], rf[2], ls[2];
+    uint32_t taddr;                // tensor-memory address of the chunk's first column
+    bool keep;
+    int N;                         // group rows (rows at or past N are not the group's)
+    __device__ __forceinline__ SStats(uint32_t ta, bool k, int n) : taddr(ta), keep(k), N(n) {
 #pragma unroll
-      for (int h = 0; h < G; ++h) {
-        if (y[h] >= ycut[h]) {
-          const int b = inv[h] > 0.f ? bin_of(y[h], lo[h], inv[h]) : 0;
-          const float ex = y[h] - hi[h];
-          if (b >= bch[h] && ex > -42.f) {   // below 2^-41 the fixed-point mass rounds to 0
-            const unsigned long long q = __float2ull_rn(exp2f(ex) * kMassScale);
-            const int bi = h * kHistStride + b;
-            const uint32_t ql = (uint32_t)q, qh = (uint32_t)(q >> 32);
-            const uint32_t old = atomicAdd(&hlo[bi], ql);
-            const uint32_t up = qh + ((old + ql < old) ? 1u : 0u);
-            if (up) atomicAdd(&hhi[bi], up);
+      for (int e = 0; e < 2; ++e) { mn[e] = INFINITY; mx[e] = -INFINITY; rf[e] = -INFINITY; ls[e] = 0.f; }
+    }
+    // (min, max, rf, ls) of slot e combined with another state
+    __device__ __forceinline__ void combine(int e, float mn2, float mx2, float r2, float l2) {
+      mn[e] = fminf(mn[e], mn2);
+      mx[e] = fmaxf(mx[e], mx2);
+      const float rr = fmaxf(rf[e], r2);
+      ls[e] = (rr == -INFINITY) ? 0.f : ls[e] * exp2f(rf[e] - rr) + l2 * exp2f(r2 - rr);
+      rf[e] = rr;
+    }
+    __device__ __forceinline__ void merge_slots() { combine(0, mn[1], mx[1], rf[1], ls[1]); }
+    __device__ __forceinline__ void merge_lanes(int o) {
+#pragma unroll
+      for (int e = 0; e < 2; ++e)
+        combine(e, __shfl_xor_sync(0xffffffffu, mn[e], o), __shfl_xor_sync(0xffffffffu, mx[e], o),
+                __shfl_xor_sync(0xffffffffu, rf[e], o), __shfl_xor_sync(0xffffffffu, ls[e], o));
+    }
+    __device__ __forceinline__ void operator()(int st, int rb, const float (&c)[V],
+                                               const ScoreTile<G>& T) {
+      if (keep) Tmem<V>::st(taddr + st * V, c);          // whole warp
+#pragma unroll
+      for (int v = 0; v < V; ++v) {
+        const int e = v & 1;
+        if (T.ok[e] && rb + T.row[v] < N) {
+          const float y = c[v];
+          mn[e] = fminf(mn[e], y);
+          mx[e] = fmaxf(mx[e], y);
+          const float d = y - rf[e];
+          if (d > 64.f) {
+            ls[e] = ls[e] * ex2_approx(-d) + 1.f;
+            rf[e] = y;
+          } else {
+            ls[e] += ex2_approx(d);
           }
         }
       }
     }
   };
 
-  // Per-row work of phase W when the scores are recomputed: the head mask of the row (heads
-  // whose bin reaches b*) and the ordered compaction of the selected rows into a list in
-  // global memory.
-  struct WSel {
-    float lo[G], inv[G];
-    int bs[G];
-    int hc[G];
-    uint32_t* out;                 // the chunk's list (global)
-    int n0, nb, par, wc_off;
-    __device__ __forceinline__ void operator()(int nl, bool ok, const float (&y)[G]) {
-      uint32_t mask = 0;
-      if (ok) {
-#pragma unroll
-        for (int h = 0; h < G; ++h) {
-          const int b = inv[h] > 0.f ? bin_of(y[h], lo[h], inv[h]) : 0;
-          if (b >= bs[h]) { mask |= 1u << h; hc[h]++; }
-        }
+  // Per-tile work of phase H: scores at or above their head's cutoff edge are compacted into
+  // the warp's queue (score, head); every 32 queued entries are binned and their fixed-point
+  // masses added to the shared histogram (two 32-bit words per bin, exact).
+  struct HComp {
+    float thr[2];                  // per slot: cutoff edge (+inf for a padding column)
+    int hd[2];
+    int N, qn, qoff, hp_off, hist_off;
+    __device__ __forceinline__ void add(float y, int h) const {
+      const float4 p = smem_at<float4>(hp_off)[h];           // lo, inv, hi
+      const int b = p.y > 0.f ? bin_of(y, p.x, p.y) : 0;
+      const float ex = y - p.z;
+      if (ex > -42.f) {                     // below 2^-41 the fixed-point mass rounds to 0
+        const unsigned long long q = __float2ull_rn(exp2f(ex) * kMassScale);
+        uint32_t* hlo = smem_at<uint32_t>(hist_off);
+        uint32_t* hhi = hlo + G * kHistStride;
+        const int bi = h * kHistStride + b;
+        const uint32_t ql = (uint32_t)q, qh = (uint32_t)(q >> 32);
+        const uint32_t old = atomicAdd(&hlo[bi], ql);
+        const uint32_t up = qh + ((old + ql < old) ? 1u : 0u);
+        if (up) atomicAdd(&hhi[bi], up);
       }
-      int before, total;
-      block_flag_prefix(mask != 0, wc_off, par, before, total);
-      par ^= 1;
-      if (mask) out[nb + before] = ((uint32_t)(n0 + nl) << 8) | mask;
-      nb += total;
+    }
+    __device__ __forceinline__ void operator()(int st, int rb, const float (&c)[V],
+                                               const ScoreTile<G>& T) {
+      (void)st;
+      const int lane = threadIdx.x & 31;
+      const uint32_t lt = (1u << lane) - 1u;
+      float2* q = smem_at<float2>(qoff);
+#pragma unroll
+      for (int v = 0; v < V; ++v) {
+        const int e = v & 1;
+        const bool cand = rb + T.row[v] < N && c[v] >= thr[e];
+        const uint32_t bal = __ballot_sync(0xffffffffu, cand);
+        if (cand) q[qn + __popc(bal & lt)] = make_float2(c[v], __int_as_float(hd[e]));
+        qn += __popc(bal);
+      }
+      __syncwarp();
+      while (qn >= 32) {
+        qn -= 32;
+        const float2 x = q[qn + lane];
+        add(x.x, __float_as_int(x.y));
+        __syncwarp();                       // the entries are overwritten by the next tile
+      }
+    }
+    __device__ __forceinline__ void finish() {
+      const int lane = threadIdx.x & 31;
+      if (lane < qn) {
+        const float2 x = smem_at<float2>(qoff)[lane];
+        add(x.x, __float_as_int(x.y));
+      }
+      qn = 0;
     }
   };
 
-  // Rows of the attention loop: the gather list (position << 8 | head mask) or a contiguous
-  // range of ring rows.
-  struct ListRows {
+  // Selection of one tile in phase W: each (lane, value) writes its (row, head) byte, then
+  // lane r forms row r's head mask. hc: selected scores per slot.
+  __device__ __forceinline__ static uint32_t tile_select(const float (&c)[V], int rb, int N,
+                                                         const float (&ts)[2],
+                                                         const ScoreTile<G>& T, int rm_off,
+                                                         int (&hc)[2]) {
+    unsigned char* rm = smem_at<unsigned char>(rm_off);
+#pragma unroll
+    for (int v = 0; v < V; ++v) {
+      const int e = v & 1;
+      if (T.ok[e]) {
+        const bool s = rb + T.row[v] < N && c[v] >= ts[e];
+        hc[e] += s;
+        rm[T.row[v] * 8 + T.head[e]] = s;
+      }
+    }
+    __syncwarp();
+    const uint2 x = smem_at<uint2>(rm_off)[threadIdx.x & 31];
+    uint32_t mask = 0;
+#pragma unroll
+    for (int h = 0; h < G; ++h) {
+      const uint32_t w = h < 4 ? x.x : x.y;
+      mask |= ((w >> ((h & 3) * 8)) & 1u) << h;
+    }
+    __syncwarp();                           // the bytes are rewritten by the next tile
+    return mask;
+  }
+
+  // Per-tile work of phase W when the scores are recomputed: the selected rows of the warp
+  // go, in row order, to the group's list in global memory: the warp's q-th entry to the
+  // slot of the q-th row of its own tiles (row 32 * tile(q / 32) + q % 32), so the chunks'
+  // and warps' regions never overlap.
+  struct WSel {
+    float ts[2];
+    int hc[2];
+    int N, nc, j, ntl, rm_off, nw;
+    uint32_t* gl;                  // the group's list (global)
+    __device__ __forceinline__ void operator()(int st, int rb, const float (&c)[V],
+                                               const ScoreTile<G>& T) {
+      (void)st;
+      const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+      const uint32_t mask = tile_select(c, rb, N, ts, T, rm_off, hc);
+      const uint32_t bal = __ballot_sync(0xffffffffu, mask != 0);
+      if (mask) {
+        const int q = nw + __popc(bal & ((1u << lane) - 1u));
+        gl[tile_row(N, nc, j, ntl, q / kWRows, warp) + q % kWRows] = ((uint32_t)(rb + lane) << 8) | mask;
+      }
+      nw += __popc(bal);
+    }
+  };
+
+  // Rows of the attention loop: the concatenation of the warps' lists (entry i of the
+  // concatenation is entry q = i - pre[w] of the warp w with pre[w] <= i < pre[w + 1]; it
+  // sits at w * stride + q of `list`, or, in the group's global list of a recomputed chunk,
+  // at the slot WSel gave it), or a contiguous range of ring rows.
+  struct WarpListRows {
     const uint32_t* list;
     const uint16_t* kb;
     const uint16_t* vb;
+    int pre_off;                   // byte offset of pre[17] in rtp_smem
+    int stride;                    // > 0: fixed per-warp stride; 0: WSel slots
+    int N, nc, j, ntl;
     __device__ __forceinline__ void operator()(int i, const uint16_t*& kp, const uint16_t*& vp,
                                                uint32_t& mk) const {
-      const uint32_t w = list[i];
-      kp = kb + (int64_t)(w >> 8) * kD;
-      vp = vb + (int64_t)(w >> 8) * kD;
-      mk = w & 0xffu;
+      const int* pre = smem_at<int>(pre_off);
+      const int w = upper_index(pre, kWarps, i);
+      const int q = i - pre[w];
+      const int at = stride > 0 ? w * stride + q : tile_row(N, nc, j, ntl, q / kWRows, w) + q % kWRows;
+      const uint32_t e = list[at];
+      kp = kb + (int64_t)(e >> 8) * kD;
+      vp = vb + (int64_t)(e >> 8) * kD;
+      mk = e & 0xffu;
     }
   };
   struct RangeRows {
@@ -624,58 +747,83 @@ struct DecodeCta {
     }
   };
 
+  __device__ __forceinline__ int tail(int bytes_back) const { return P.sm_stage + P.free_bytes - bytes_back; }
+  __device__ __forceinline__ uint32_t chunk_taddr(int tcol) const {
+    return tmem_addr((uint32_t)sm.ints()[60], tcol);
+  }
+
+  // Per-warp list counts -> prefix pre[0..16] in ints[kIntPre...] (block-wide; ends with a
+  // barrier). Returns the total.
+  __device__ __forceinline__ int list_prefix(int nw) {
+    int* pre = sm.ints() + kIntPre;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    __syncthreads();
+    if (lane == 0) pre[1 + warp] = nw;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      pre[0] = 0;
+      for (int w = 0; w < kWarps; ++w) pre[1 + w] += pre[w];
+    }
+    __syncthreads();
+    return pre[kWarps];
+  }
+
   // ------------------------------------------------------------ phase S
   // tcol: first tensor-memory column of the chunk's scores, -1 when they are not kept.
   __device__ __forceinline__ void phase_score(int k, int tcol) {
     const int g = group_of(k), j = k - sm.cbase()[g];
     const int N = gN(g);
-    const bool patch = P.k_new && min(N, (j + 1) * C) == N;
-    SStats sst((uint32_t)sm.ints()[60], tcol);
+    const bool patch = P.k_new && ((N - 1) / kWRows) % nch(g) == j;   // holds row N - 1
+    SStats sst(tcol >= 0 ? chunk_taddr(tcol) : 0u, tcol >= 0, N);
     trace(kEvS0);
     stream_chunk(g, j, patch, sst);
     if (tcol >= 0) tmem_wait_st();
     trace(kEvS1);
-    float (&mn)[G] = sst.mn;
-    float (&mx)[G] = sst.mx;
-    float (&rf)[G] = sst.rf;
-    float (&ls)[G] = sst.ls;
-    // chunk statistics per head: min, max, sum 2^(y - max); warp shuffles, then a fixed-order
-    // pass over the warps
+    // chunk statistics per head: lanes of one tig hold the same heads (reduce over gid),
+    // then a fixed-order pass over (warp, tig, slot)
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    float* red = reinterpret_cast<float*>(sm.tmp());         // [4][G][16]
 #pragma unroll
-    for (int h = 0; h < G; ++h) {
+    for (int o = 4; o < 32; o <<= 1) sst.merge_lanes(o);
+    // complete the warp's stats of each head in one lane: G = 1: both slots of tig 0;
+    // G = 2: tig 0 and 1; G = 4: tig t and t + 2 (G = 8: every (tig, slot) is one head)
+    {
+      const int tig = lane & 3;
+      if (G < 8) {
 #pragma unroll
-      for (int o = 16; o > 0; o >>= 1) {
-        mn[h] = fminf(mn[h], __shfl_xor_sync(0xffffffffu, mn[h], o));
-        mx[h] = fmaxf(mx[h], __shfl_xor_sync(0xffffffffu, mx[h], o));
-        const float r2 = __shfl_xor_sync(0xffffffffu, rf[h], o);
-        const float l2 = __shfl_xor_sync(0xffffffffu, ls[h], o);
-        const float rr = fmaxf(rf[h], r2);
-        ls[h] = (rr == -INFINITY) ? 0.f : ls[h] * exp2f(rf[h] - rr) + l2 * exp2f(r2 - rr);
-        rf[h] = rr;
+        for (int e = 0; e < 2; ++e)
+          if (2 * tig + e >= 2 * G) { sst.mn[e] = INFINITY; sst.mx[e] = -INFINITY; sst.rf[e] = -INFINITY; sst.ls[e] = 0.f; }
       }
-      if (lane == 0) {
-        red[(0 * G + h) * 16 + warp] = mn[h];
-        red[(1 * G + h) * 16 + warp] = mx[h];
-        red[(2 * G + h) * 16 + warp] = rf[h];
-        red[(3 * G + h) * 16 + warp] = ls[h];
+      if (G == 1) sst.merge_slots();
+      if (G == 2) sst.merge_lanes(1);
+      if (G == 4) sst.merge_lanes(2);
+    }
+    float4* red = reinterpret_cast<float4*>(sm.tmp());       // [16 warps][8 heads]
+    if (lane < 4) {
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const int n = 2 * lane + e;
+        const bool own = G == 8 ? true : (G == 4 ? n < 4 : (G == 2 ? n < 2 : n == 0));
+        if (own) red[warp * 8 + n] = make_float4(sst.mn[e], sst.mx[e], sst.rf[e], sst.ls[e]);
       }
     }
     __syncthreads();
-    if (threadIdx.x < G) {
-      const int h = threadIdx.x;
-      float a = INFINITY, z = -INFINITY;
-      for (int w = 0; w < kFThreads / 32; ++w) {
-        a = fminf(a, red[(0 * G + h) * 16 + w]);
-        z = fmaxf(z, red[(1 * G + h) * 16 + w]);
+    if (warp < G) {                        // warp h: lanes over the warps, fixed shuffle tree
+      const float4 x = lane < kWarps ? red[lane * 8 + warp] : make_float4(INFINITY, -INFINITY, -INFINITY, 0.f);
+      float a = x.x, z = x.y;
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        a = fminf(a, __shfl_xor_sync(0xffffffffu, a, o));
+        z = fmaxf(z, __shfl_xor_sync(0xffffffffu, z, o));
       }
-      double l = 0.0;                        // references never exceed the chunk max
-      for (int w = 0; w < kFThreads / 32; ++w) {
-        const float rw = red[(2 * G + h) * 16 + w];
-        if (rw != -INFINITY) l += (double)red[(3 * G + h) * 16 + w] * (double)exp2f(rw - z);
-      }
-      P.cstat[((int64_t)g * P.max_nch + j) * G + h] = make_float4(a, z, (float)l, 0.f);
+      double l = x.z != -INFINITY ? (double)x.w * (double)exp2f(x.z - z) : 0.0;   // rf <= max
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) l += __shfl_xor_sync(0xffffffffu, l, o);
+      if (lane == 0) P.cstat[((int64_t)g * P.max_nch + j) * G + warp] = make_float4(a, z, (float)l, 0.f);
+    }
+    if (j == 0) {   // the group's histogram and counts, before any chunk of it reaches phase H
+      unsigned long long* gh = P.hist + (int64_t)g * G * kBins * kHistPad;
+      for (int i = threadIdx.x; i < G * kBins * kHistPad; i += kFThreads) gh[i] = 0ull;
+      if (threadIdx.x < G) P.hcnt[(int64_t)g * G + threadIdx.x] = 0;
     }
     arrive(P.bar + (int64_t)g * 4 + 0);
   }
@@ -686,144 +834,169 @@ struct DecodeCta {
   // bin(c), c = hi + log2((1 - p) T' / N), T' = T (1 - 1e-3), has mass below (1 - p) T' / N,
   // so together they hold less than (1 - p) of the total, C_bin(c) > p T, and b* can not fall
   // under the cutoff bin (the 1e-3 absorbs the rounding of T, the log and the bin edges).
-  // Rows whose bin reaches the cutoff add their masses (2^(y - max) in 2^-40 fixed point) to
-  // the group's histogram. The range (lo, 256 / (hi - lo)) and T are kept for phase W.
+  // Scores in bins at or above the cutoff add their masses (2^(y - max) in 2^-40 fixed point)
+  // to the group's histogram. The range (lo, 256 / (hi - lo), hi) and T are kept for phase W.
   __device__ __forceinline__ void phase_hist(int k, int step, int tcol) {
     const int g = group_of(k), j = k - sm.cbase()[g];
-    const int N = gN(g), n0 = j * C, len = min(N, n0 + C) - n0;
+    const int N = gN(g);
     const int nc = nch(g);
     trace(kEvH0);
     if (!wait_for(P.bar + (int64_t)g * 4 + 0, (uint32_t)nc)) { abort_ = true; return; }
     trace(kEvHw);
-    // group statistics: thread t folds chunks t / G, t / G + kFThreads / G, ... of head t % G
-    double* part = sm.tmp();                                 // [kFThreads]
-    float* st3 = sm.res();                                   // [G][3] lo, hi, inv
+    // group statistics in one pass: thread t folds chunks t / G, t / G + kFThreads / G, ... of
+    // head t % G into (min, max, mass relative to its running max); lanes of one head, then
+    // the warps, combine in a fixed order (every CTA gets the same values)
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     {
       const int t = threadIdx.x, h = t % G;
       float a = INFINITY, z = -INFINITY;
+      double m = 0.0;                      // sum 2^(y - z) over the folded chunks
       for (int c = t / G; c < nc; c += kFThreads / G) {
         const float4 v = __ldcg(P.cstat + ((int64_t)g * P.max_nch + c) * G + h);
         a = fminf(a, v.x);
-        z = fmaxf(z, v.y);
+        if (v.y > z) {
+          m = (z == -INFINITY ? 0.0 : m * (double)exp2f(z - v.y)) + (double)v.z;
+          z = v.y;
+        } else {
+          m += (double)v.z * (double)exp2f(v.y - z);
+        }
       }
 #pragma unroll
       for (int o = G; o < 32; o <<= 1) {
-        a = fminf(a, __shfl_xor_sync(0xffffffffu, a, o));
-        z = fmaxf(z, __shfl_xor_sync(0xffffffffu, z, o));
+        const float a2 = __shfl_xor_sync(0xffffffffu, a, o);
+        const float z2 = __shfl_xor_sync(0xffffffffu, z, o);
+        const double m2 = __shfl_xor_sync(0xffffffffu, m, o);
+        const float zz = fmaxf(z, z2);
+        m = zz == -INFINITY ? 0.0
+                            : m * (double)exp2f(z - zz) + m2 * (double)exp2f(z2 - zz);
+        a = fminf(a, a2);
+        z = zz;
       }
-      float* pf = reinterpret_cast<float*>(part);
-      if ((t & 31) < G) {
-        pf[(t >> 5) * G + h] = a;
-        pf[512 + (t >> 5) * G + h] = z;
-      }
-      __syncthreads();
-      if (t < G) {
-        float lo = INFINITY, hi = -INFINITY;
-        for (int w = 0; w < kFThreads / 32; ++w) {
-          lo = fminf(lo, pf[w * G + t]);
-          hi = fmaxf(hi, pf[512 + w * G + t]);
-        }
-        const float inv = (hi > lo && !P.select_all) ? (float)kBins / (hi - lo) : 0.f;
-        st3[t * 3 + 0] = lo;
-        st3[t * 3 + 1] = hi;
-        st3[t * 3 + 2] = inv;
-        sm.lcache()[step * G + t] = make_float2(lo, inv);
-        if (j == 0) P.grange[(int64_t)g * G + t] = make_float2(lo, inv);
-      }
-      __syncthreads();
-      const float hih = st3[h * 3 + 1];
-      double acc = 0.0;
-      for (int c = t / G; c < nc; c += kFThreads / G) {
-        const float4 v = __ldcg(P.cstat + ((int64_t)g * P.max_nch + c) * G + h);
-        acc += (double)v.z * (double)exp2f(v.y - hih);
-      }
-      __syncthreads();
-      part[t] = acc;
-      __syncthreads();
-      if (t < G) {
-        double v = 0.0;
-        for (int i = t; i < kFThreads; i += G) v += part[i];
-        sm.tcache()[step * G + t] = v;
+      double* pd = sm.tmp();                                 // [16 warps][G] (a, z, m)
+      if (lane < G) {
+        pd[(warp * G + h) * 3 + 0] = (double)a;
+        pd[(warp * G + h) * 3 + 1] = (double)z;
+        pd[(warp * G + h) * 3 + 2] = m;
       }
       __syncthreads();
     }
-    trace(kEvHs);
-    HHist hh;
+    if (warp < G) {                        // warp h: lanes over the warps, fixed shuffle trees
+      const double* pd = sm.tmp();
+      const int h = warp;
+      float a = INFINITY, z = -INFINITY;
+      double m = 0.0;
+      if (lane < kWarps) {
+        a = (float)pd[(lane * G + h) * 3 + 0];
+        z = (float)pd[(lane * G + h) * 3 + 1];
+        m = pd[(lane * G + h) * 3 + 2];
+      }
+      float lo = a, hi = z;
 #pragma unroll
-    for (int h = 0; h < G; ++h) {
-      hh.lo[h] = st3[h * 3 + 0];
-      hh.hi[h] = st3[h * 3 + 1];
-      hh.inv[h] = st3[h * 3 + 2];
-      hh.bch[h] = 0;
-      if (P.p < 1.0 && hh.inv[h] > 0.f) {
-        const double T = sm.tcache()[step * G + h];
-        const float arg = (float)((1.0 - P.p) * T * (1.0 - 1e-3) / (double)N);
-        const float c = hh.hi[h] + log2f(arg);
-        hh.bch[h] = c > hh.lo[h] ? bin_of(c, hh.lo[h], hh.inv[h]) : 0;
+      for (int o = 16; o > 0; o >>= 1) {
+        lo = fminf(lo, __shfl_xor_sync(0xffffffffu, lo, o));
+        hi = fmaxf(hi, __shfl_xor_sync(0xffffffffu, hi, o));
       }
-      hh.ycut[h] = hh.bch[h] > 0 ? hh.lo[h] + ((float)hh.bch[h] - 0.5f) / hh.inv[h] : -INFINITY;
+      double T = z != -INFINITY ? m * (double)exp2f(z - hi) : 0.0;
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) T += __shfl_xor_sync(0xffffffffu, T, o);
+      const float inv = (hi > lo && !P.select_all) ? (float)kBins / (hi - lo) : 0.f;
+      // cutoff bin, its score edge; per-head parameters of the binning
+      int bch = 0;
+      if (P.p < 1.0 && inv > 0.f) {
+        const float arg = (float)((1.0 - P.p) * T * (1.0 - 1e-3) / (double)N);
+        const float c = hi + log2f(arg);
+        bch = c > lo ? bin_of(c, lo, inv) : 0;
+      }
+      const float e = bin_edge_warp(bch, lo, hi, inv);
+      if (lane == 0) {
+        sm.lcache()[step * G + h] = make_float4(lo, inv, hi, 0.f);
+        if (j == 0) P.grange[(int64_t)g * G + h] = make_float2(lo, inv);
+        sm.tcache()[step * G + h] = T;
+        reinterpret_cast<float4*>(sm.ints() + kIntHp)[h] = make_float4(lo, inv, hi, 0.f);
+        reinterpret_cast<float*>(sm.ints())[kIntEdge + h] = e;
+      }
     }
-    hh.hist_off = P.sm_hist;
     uint32_t* hlo = sm.hist();
     uint32_t* hhi = hlo + G * kHistStride;
     for (int i = threadIdx.x; i < 2 * G * kHistStride; i += kFThreads) hlo[i] = 0u;
     __syncthreads();
+    trace(kEvHs);
+    HComp hc;
+    {
+      const int tig = threadIdx.x & 3;
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const int n = 2 * tig + e;
+        const bool ok = G == 8 ? true : n < 2 * G;
+        hc.hd[e] = G == 8 ? n : n % G;
+        hc.thr[e] = ok ? reinterpret_cast<const float*>(sm.ints())[kIntEdge + hc.hd[e]] : INFINITY;
+      }
+    }
+    hc.N = N;
+    hc.qn = 0;
+    hc.qoff = tail(kTailHq) + warp * kHQueueMax * 8;
+    hc.hp_off = P.sm_int + kIntHp * 4;
+    hc.hist_off = P.sm_hist;
     if (tcol >= 0) {
-      const uint32_t tb = (uint32_t)sm.ints()[60];
+      ScoreTile<G> T;                      // lane layout only (no query needed)
+      T.init(sm.qidx());
+      const uint32_t ta = chunk_taddr(tcol);
+      const int ntl = chunk_tiles(N, nc, j), nst = chunk_stages(N, nc, j);
 #pragma unroll 1
-      for (int i0 = 0; i0 < len; i0 += kFThreads) {
-        const int nl = i0 + threadIdx.x;
-        float y[G];
-        Tmem<G>::ld(tmem_addr(tb, tcol + (i0 / kSRows) * G), y);     // whole warp
+      for (int st = 0; st < nst; ++st) {
+        float c[V];
+        Tmem<V>::ld(ta + st * V, c);       // whole warp
         tmem_wait_ld();
-        hh(nl, nl < len, y);
+        hc(st, tile_row(N, nc, j, ntl, st, warp), c, T);
       }
     } else {
-      stream_chunk(g, j, false, hh);
+      stream_chunk(g, j, false, hc);
     }
+    hc.finish();
     __syncthreads();
     trace(kEvH1);
-    unsigned long long* gh = P.hist + (int64_t)g * G * kBins;
+    unsigned long long* gh = P.hist + (int64_t)g * G * kBins * kHistPad;
     for (int i = threadIdx.x; i < G * kBins; i += kFThreads) {
       const int hd = i / kBins, b = i % kBins;
       const unsigned long long v =
           ((unsigned long long)hhi[hd * kHistStride + b] << 32) | hlo[hd * kHistStride + b];
-      if (v) atomicAdd(gh + i, v);
+      if (v) atomicAdd(gh + (int64_t)i * kHistPad, v);
     }
     arrive(P.bar + (int64_t)g * 4 + 1);
   }
 
-  __device__ __forceinline__ void merge(const float* parts, int n, float* dst, uint16_t* out_rows,
-                                        int buf_bytes) {
-    merge_partials<G>(parts, n, dst, out_rows, reinterpret_cast<float*>(sm.stage()), buf_bytes,
-                      kFThreads);
-  }
-
   // ------------------------------------------------------------ phase W
-  // The chunk's own rows with bin >= b* for some head (from its kept scores, or recomputed
-  // from the index rows), with the mask of those heads, in row order; their K/V rows are
-  // gathered once for all G heads. Kept scores: the list is built in shared memory at the
-  // end of the staging region and handed to the attention loop whenever it fills up.
-  // Recomputed scores: the list is written to global memory first (the index ring and the
-  // tiles share the staging region), then read back in batches. The rotated query is formed
-  // before the wait. Partials merge in teams of kTeam by the last arrivals.
+  // b* per head from the group's histogram and the score edge of b*; the chunk's rows with a
+  // score at or above the edge for some head (from the kept scores, or recomputed from the
+  // index rows), with the mask of those heads; their K/V rows are gathered once for all G
+  // heads. Kept scores: per-warp lists in shared memory, attended every kWBatch stages.
+  // Recomputed scores: per-warp regions of the chunk's list in global memory (the index
+  // ring and the tiles share the staging region), attended after the pass. The rotated query
+  // is formed before the wait. The partials of the group are merged by the last arrival.
   __device__ __forceinline__ void phase_attend(int k, int step, int tcol) {
     const int g = group_of(k), j = k - sm.cbase()[g];
     const int b = g / P.L.n_ret, r = g % P.L.n_ret, kvh = P.L.ret_kv[r];
-    const int N = gN(g), n0 = j * C, len = min(N, n0 + C) - n0;
+    const int N = gN(g);
     const int S = nch(g);
+    const int ntl = chunk_tiles(N, S, j), nst = chunk_stages(N, S, j);
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     rope_query<G>(P, b, kvh, N, sm.q());
+    __syncthreads();
+    WarpAttn W;
+    attn_begin<G>(W, sm.qbuf(), sm.q(), kFThreads);
+    ScoreTile<G> T;
+    T.init(sm.qidx());                     // lane layout; its query part is not used here
     if (!wait_for(P.bar + (int64_t)g * 4 + 1, (uint32_t)S)) { abort_ = true; return; }
     trace(kEvW0);
     // b* per head (warp h: head h): the highest bin whose mass from the top reaches p T
     if (warp < G) {
       int best = 0;
       if (!P.select_all) {
-        const unsigned long long* gh = P.hist + ((int64_t)g * G + warp) * kBins + lane * 8;
+        const unsigned long long* gh =
+            P.hist + (((int64_t)g * G + warp) * kBins + lane * 8) * kHistPad;
         unsigned long long hv[8], lt = 0;
 #pragma unroll
-        for (int e = 0; e < 8; ++e) { hv[e] = __ldcg(gh + e); lt += hv[e]; }
+        for (int e = 0; e < 8; ++e) { hv[e] = __ldcg(gh + e * kHistPad); lt += hv[e]; }
         unsigned long long x = lt;            // inclusive suffix sum over lanes
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
@@ -842,132 +1015,103 @@ struct DecodeCta {
         for (int o = 16; o > 0; o >>= 1) best = max(best, __shfl_xor_sync(0xffffffffu, best, o));
         best = max(best, 0);
       }
-      if (lane == 0) sm.ints()[40 + warp] = best;
+      trace(kEvWh);
+      const float4 li = sm.lcache()[step * G + warp];
+      const float e = bin_edge_warp(best, li.x, li.z, li.y);
+      if (lane == 0) {
+        sm.ints()[40 + warp] = best;
+        reinterpret_cast<float*>(sm.ints())[kIntEdge + warp] = e;
+        sm.ints()[kIntCnt + warp] = 0;
+      }
     }
     __syncthreads();
-    WSel ws;
+    trace(kEvWb);
+    if (j == 0 && threadIdx.x < G) P.bstar[(int64_t)g * G + threadIdx.x] = sm.ints()[40 + threadIdx.x];
+    float ts[2];
+    int hc[2] = {0, 0};
 #pragma unroll
-    for (int h = 0; h < G; ++h) {
-      ws.bs[h] = sm.ints()[40 + h];
-      const float2 li = sm.lcache()[step * G + h];
-      ws.lo[h] = li.x;
-      ws.inv[h] = li.y;
-      ws.hc[h] = 0;
-    }
-    if (j == 0 && threadIdx.x < G) P.bstar[(int64_t)g * G + threadIdx.x] = ws.bs[threadIdx.x];
-    ws.n0 = n0;
-    ws.nb = 0;
-    ws.par = 0;
-    ws.wc_off = P.sm_int + 64 * 4;
+    for (int e = 0; e < 2; ++e)
+      ts[e] = T.ok[e] ? reinterpret_cast<const float*>(sm.ints())[kIntEdge + T.head[e]] : INFINITY;
     const int64_t rowbase = (int64_t)r * P.L.T_total + P.cache.seq_off[b];
     const uint16_t* kb = P.cache.k_ret + rowbase * kD;
     const uint16_t* vb = P.cache.v_ret + rowbase * kD;
-    uint32_t* list = reinterpret_cast<uint32_t*>(sm.stage() + P.free_bytes - kListCap * 4);
-    const int nwa = min(kFThreads / 32, (P.free_bytes - kListCap * 4) / kTileBytes);
-    const ListRows rows{list, kb, vb};
-    WarpAttn W;
+    const int rm_off = tail(kTailRm) + warp * kWRows * 8;
+    const int nwa = min(kFThreads / 32, (P.free_bytes - kTailRm) / kTileBytes);
     if (tcol >= 0) {
-      attn_begin<G>(W, sm.qbuf(), sm.q(), kFThreads);
+      uint32_t* list = smem_at<uint32_t>(tail(kTailList));
+      uint32_t* wl = list + warp * kWListCap;
+      const WarpListRows rows{list, kb, vb, P.sm_int + kIntPre * 4, kWListCap, N, S, j, ntl};
       trace(kEvW1);
-      const uint32_t tb = (uint32_t)sm.ints()[60];
+      const uint32_t ta = chunk_taddr(tcol);
 #pragma unroll 1
-      for (int i0 = 0; i0 < len; i0 += kFThreads) {
-        if (ws.nb > kListCap - kFThreads) {   // the list is full: attend to it first
-          __syncthreads();
-          attn_tiles<G>(W, ws.nb, rows, sm.stage(), nwa, false);
-          __syncthreads();
-          ws.nb = 0;
+      for (int s0 = 0; s0 < nst; s0 += kWBatch) {
+        int nw = 0;
+        const int s1 = min(nst, s0 + kWBatch);
+#pragma unroll 1
+        for (int st = s0; st < s1; ++st) {
+          float c[V];
+          Tmem<V>::ld(ta + st * V, c);     // whole warp
+          tmem_wait_ld();
+          const int rb = tile_row(N, S, j, ntl, st, warp);
+          const uint32_t mask = tile_select(c, rb, N, ts, T, rm_off, hc);
+          const uint32_t bal = __ballot_sync(0xffffffffu, mask != 0);
+          if (mask) wl[nw + __popc(bal & ((1u << lane) - 1u))] = ((uint32_t)(rb + lane) << 8) | mask;
+          nw += __popc(bal);
         }
-        const int nl = i0 + threadIdx.x;
-        float y[G];
-        Tmem<G>::ld(tmem_addr(tb, tcol + (i0 / kSRows) * G), y);     // whole warp
-        tmem_wait_ld();
-        uint32_t mask = 0;
-        if (nl < len) {
-#pragma unroll
-          for (int h = 0; h < G; ++h) {
-            const int bb = ws.inv[h] > 0.f ? bin_of(y[h], ws.lo[h], ws.inv[h]) : 0;
-            if (bb >= ws.bs[h]) { mask |= 1u << h; ws.hc[h]++; }
-          }
-        }
-        int before, total;
-        block_flag_prefix(mask != 0, ws.wc_off, ws.par, before, total);
-        ws.par ^= 1;
-        if (mask) list[ws.nb + before] = ((uint32_t)(n0 + nl) << 8) | mask;
-        ws.nb += total;
+        const int total = list_prefix(nw);
+        trace(kEvWl);
+        attn_tiles<G>(W, total, rows, sm.stage(), nwa, false);
+        __syncthreads();                   // the lists are rewritten by the next batch
       }
-      __syncthreads();
-      trace(kEvWl);
-      attn_tiles<G>(W, ws.nb, rows, sm.stage(), nwa, false);
     } else {
-      uint32_t* gl = P.sellist + (int64_t)g * P.cand_stride + n0;
-      ws.out = gl;
-      stream_chunk(g, j, false, ws);
-      __syncthreads();
-      attn_begin<G>(W, sm.qbuf(), sm.q(), kFThreads);
+      uint32_t* gl = P.sellist + (int64_t)g * P.cand_stride;
+      WSel wsel;
+      wsel.ts[0] = ts[0]; wsel.ts[1] = ts[1];
+      wsel.hc[0] = 0; wsel.hc[1] = 0;
+      wsel.N = N; wsel.nc = S; wsel.j = j; wsel.ntl = ntl;
+      wsel.rm_off = rm_off;
+      wsel.nw = 0;
+      wsel.gl = gl;
+      stream_chunk(g, j, false, wsel);
+      hc[0] = wsel.hc[0]; hc[1] = wsel.hc[1];
+      __threadfence_block();
+      const int total = list_prefix(wsel.nw);
       trace(kEvWl);
-      const int total = ws.nb;
-#pragma unroll 1
-      for (int b0 = 0; b0 < total; b0 += kListCap) {
-        const int nb = min(kListCap, total - b0);
-        __syncthreads();
-        for (int i = threadIdx.x; i < nb; i += kFThreads) list[i] = __ldcg(gl + b0 + i);
-        __syncthreads();
-        attn_tiles<G>(W, nb, rows, sm.stage(), nwa, false);
-      }
+      const WarpListRows rows{gl, kb, vb, P.sm_int + kIntPre * 4, 0, N, S, j, ntl};
+      attn_tiles<G>(W, total, rows, sm.stage(), nwa, false);
     }
     attn_end<G>(W, nwa, sm.res(), reinterpret_cast<float*>(sm.stage()), kFThreads);
     trace(kEvW2);
     // per-head counts of this chunk
-    int* red = reinterpret_cast<int*>(sm.tmp());              // [16][G]
 #pragma unroll
-    for (int h = 0; h < G; ++h) {
-      int v = ws.hc[h];
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-      if (lane == 0) red[warp * G + h] = v;
-    }
+    for (int e = 0; e < 2; ++e)
+      if (T.ok[e] && hc[e]) atomicAdd(sm.ints() + kIntCnt + T.head[e], hc[e]);
     __syncthreads();
     if (threadIdx.x < G) {
-      int v = 0;
-      for (int w = 0; w < kFThreads / 32; ++w) v += red[w * G + threadIdx.x];
+      const int v = sm.ints()[kIntCnt + threadIdx.x];
       if (v) atomicAdd(P.hcnt + (int64_t)g * G + threadIdx.x, v);
     }
-    // partial -> workspace; team / group merge by the last arrivals
-    const int stride = G * (kD + 2);
-    float* mine = P.part + (int64_t)k * stride;
-    for (int o = threadIdx.x; o < stride; o += kFThreads) mine[o] = sm.res()[o];
-    const int team = j / kTeam, nteams = (S + kTeam - 1) / kTeam;
-    const int tcount = min(kTeam, S - team * kTeam);
+    // partial -> workspace; the last chunk of the group to finish merges all of them
+    write_partial<G, kFThreads>(sm.res(), P.part + (int64_t)k * Part<G>::kBytes);
     __syncthreads();
     if (threadIdx.x == 0) {
       __threadfence();
-      sm.ints()[36] = atomicAdd(P.team_arr + sm.cbase()[g] + team, 1u) == (uint32_t)(tcount - 1);
+      sm.ints()[36] = atomicAdd(P.bar + (int64_t)g * 4 + 2, 1u) == (uint32_t)(S - 1);
     }
     __syncthreads();
     if (!sm.ints()[36]) return;
     __threadfence();
-    uint16_t* orow = P.out + ((int64_t)b * P.L.Hq + kvh * G) * kD;
-    const float* tparts = P.part + (int64_t)(sm.cbase()[g] + team * kTeam) * stride;
-    if (nteams == 1) {
-      merge(tparts, tcount, nullptr, orow, P.free_bytes);
-    } else {
-      merge(tparts, tcount, P.tpart + (int64_t)(sm.cbase()[g] + team) * stride, nullptr, P.free_bytes);
-      __syncthreads();
-      if (threadIdx.x == 0) {
-        __threadfence();
-        sm.ints()[37] = atomicAdd(P.bar + (int64_t)g * 4 + 2, 1u) == (uint32_t)(nteams - 1);
-      }
-      __syncthreads();
-      if (!sm.ints()[37]) return;
-      __threadfence();
-      merge(P.tpart + (int64_t)sm.cbase()[g] * stride, nteams, nullptr, orow, P.free_bytes);
-    }
+    merge(P.part + (int64_t)sm.cbase()[g] * Part<G>::kBytes, S,
+          P.out + ((int64_t)b * P.L.Hq + kvh * G) * kD);
     if (threadIdx.x < G)
       P.sel_counts[(int64_t)b * P.L.Hq + kvh * G + threadIdx.x] =
           __ldcg(P.hcnt + (int64_t)g * G + threadIdx.x);
     trace(kEvW3);
     __syncthreads();
+  }
+
+  __device__ __forceinline__ void merge(const unsigned char* parts, int n, uint16_t* out_rows) {
+    merge_all<G, kFThreads>(parts, n, out_rows, sm.stage(), P.free_bytes, sm.res());
   }
 
   // ------------------------------------------------------------ local items
@@ -998,9 +1142,7 @@ struct DecodeCta {
     attn_begin<G>(W, sm.qbuf(), sm.q(), kFThreads);
     attn_tiles<G>(W, nrows, rowfn, sm.stage(), nwa, true);
     attn_end<G>(W, nwa, sm.res(), reinterpret_cast<float*>(sm.stage()), kFThreads);
-    const int stride = G * (kD + 2);
-    float* mine = P.lpart + (int64_t)li * stride;
-    for (int o = threadIdx.x; o < stride; o += kFThreads) mine[o] = sm.res()[o];
+    write_partial<G, kFThreads>(sm.res(), P.lpart + (int64_t)li * Part<G>::kBytes);
     __syncthreads();
     if (threadIdx.x == 0) {
       __threadfence();
@@ -1009,8 +1151,8 @@ struct DecodeCta {
     __syncthreads();
     if (sm.ints()[38]) {
       __threadfence();
-      merge(P.lpart + (int64_t)lg * P.PL * stride, P.PL, nullptr,
-            P.out + ((int64_t)b * P.L.Hq + kvh * G) * kD, P.free_bytes);
+      merge(P.lpart + (int64_t)lg * P.PL * Part<G>::kBytes, P.PL,
+            P.out + ((int64_t)b * P.L.Hq + kvh * G) * kD);
       if (threadIdx.x < G) P.sel_counts[(int64_t)b * P.L.Hq + kvh * G + threadIdx.x] = nrows_all;
     }
     __syncthreads();
@@ -1054,8 +1196,7 @@ struct DecodeCta {
       int col = 0;
       for (int t = 0; t < m; ++t) {
         const int k = i + t * P_ret, g = group_of(k), j = k - sm.cbase()[g];
-        const int len = min(gN(g), (j + 1) * C) - j * C;
-        const int need = (len + kSRows - 1) / kSRows * G;
+        const int need = chunk_stages(gN(g), nch(g), j) * V;
         if (col + need <= kTmemColsPerThread) { tcols[t] = col; col += need; } else { tcols[t] = -1; }
       }
     }
@@ -1105,21 +1246,25 @@ __global__ void __launch_bounds__(kFThreads, 1) decode_kernel(const __grid_const
 // ------------------------------------------------------------------------------ sel_idx
 // Debug output: ascending positions each query head attended to. One CTA of kFThreads threads
 // per (b, h): a retrieval head's scores are recomputed with the decode kernel's own routines
-// (the same index query, the same per-row arithmetic, so the same bits), binned with the
-// group's range and compared with its b*; the selected positions are compacted in order.
+// (the same index query, the same tensor-core tile, so the same bits), binned with the
+// group's range and compared with its b* (through bin_of, not the score edge the decode
+// kernel compares with, so a test of the two sets also checks the edge); the selected
+// positions are compacted in order.
 template <int G>
 __global__ void __launch_bounds__(kFThreads) emit_sel_kernel(DecodeParams P, int32_t* sel_idx,
                                                              int64_t sel_stride) {
   __shared__ float qidx[G * kR];
   __shared__ float tmp[kFThreads];
   __shared__ int wc[32];
+  __shared__ __align__(16) unsigned char rows_s[kWarps][kSlotBytes];
+  __shared__ unsigned char keep_s[kWarps][kWRows];
   const int b = blockIdx.x / P.L.Hq, h = blockIdx.x % P.L.Hq;
   const int kvh = h / G, jh = h % G;
   const int N = seq_len_checked(P, b);
   int32_t* dst = sel_idx + ((int64_t)b * P.L.Hq + h) * sel_stride;
   if (N == 0) return;
   const int slot = P.L.slot[kvh];
-  const int t = threadIdx.x;
+  const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
   if (slot < 0) {
     const int s1 = min(N, P.L.sinks);
     const int w0 = max(P.L.sinks, N - P.L.window);
@@ -1131,30 +1276,41 @@ __global__ void __launch_bounds__(kFThreads) emit_sel_kernel(DecodeParams P, int
   const int bst = __ldcg(P.bstar + (int64_t)g * G + jh);
   const float2 li = __ldcg(P.grange + (int64_t)g * G + jh);
   index_query<G>(P, b, kvh, qidx, tmp);
-  float2 qi[G][kR / 2];
-#pragma unroll
-  for (int hh = 0; hh < G; ++hh)
-#pragma unroll
-    for (int jj = 0; jj < kR / 2; ++jj)
-      qi[hh][jj] = make_float2(qidx[hh * kR + 2 * jj], qidx[hh * kR + 2 * jj + 1]);
+  ScoreTile<G> T;
+  T.init(qidx);
   const unsigned char* src = (const unsigned char*)(
       P.cache.idx + ((int64_t)slot * P.L.T_total + P.cache.seq_off[b]) * kR);
+  const uint32_t sa = smem_u32(rows_s[warp]);
   int base = 0, par = 0;
 #pragma unroll 1
-  for (int i0 = 0; i0 < N; i0 += kFThreads) {
-    const int n = i0 + t;
-    bool keep = false;
-    if (n < N) {
-      float y[G];
-      score_row<G>(qi, src + (int64_t)n * 32, y);
-      const int bb = li.y > 0.f ? bin_of(y[jh], li.x, li.y) : 0;
-      keep = bb >= bst;
+  for (int i0 = 0; i0 < N; i0 += kSRows) {
+    const int rb = i0 + warp * kWRows;
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      const int p = lane + 32 * u, r = p >> 1, hh = p & 1;
+      *reinterpret_cast<uint4*>(rows_s[warp] + idx_half_off(r, hh)) =
+          rb + r < N ? __ldg(reinterpret_cast<const uint4*>(src + (int64_t)(rb + r) * 32 + hh * 16))
+                     : make_uint4(0u, 0u, 0u, 0u);
     }
+    __syncwarp();
+    float c[ScoreTile<G>::V];
+    T.score(sa, c);
+#pragma unroll
+    for (int v = 0; v < ScoreTile<G>::V; ++v) {
+      const int e = v & 1;
+      if (T.ok[e] && T.head[e] == jh) {
+        const int bb = li.y > 0.f ? bin_of(c[v], li.x, li.y) : 0;
+        keep_s[warp][T.row[v]] = (rb + T.row[v] < N) && bb >= bst;
+      }
+    }
+    __syncwarp();
+    const bool keep = keep_s[warp][lane] != 0;
     int before, total;
-    block_flag_prefix_impl(keep, wc + par * 16, before, total);
+    block_flag_prefix(keep, wc + par * 16, before, total);
     par ^= 1;
-    if (keep) dst[base + before] = n;
+    if (keep) dst[base + before] = rb + lane;
     base += total;
+    __syncwarp();                          // rows_s / keep_s are rewritten next round
   }
 }
 

@@ -116,6 +116,15 @@ def run_layer_parity(workload_index=1, layer=0, p=None, check_sets=True, heads=N
     out, cnt, sel = decode(lay, q, wq, seq_lens, p, device, with_sel=check_sets)
     st = lay.status()
     assert st == 0, f"device status {st}"
+    report = check_outputs(w, layer, seq_lens, p, out, cnt, sel, heads)
+    report["layer"] = lay
+    return report
+
+
+def check_outputs(w, layer, seq_lens, p, out, cnt, sel=None, heads=None) -> dict:
+    """Compares one decode's outputs (device tensors) with the oracle under the rules above,
+    for the (b, h) pairs in ``heads`` (every head when None). Raises AssertionError."""
+    seq_lens = np.asarray(seq_lens, np.int64)
     out = out.float().cpu().numpy()
     cnt = cnt.cpu().numpy()
     sel = sel.cpu().numpy() if sel is not None else None
@@ -160,5 +169,4 @@ def run_layer_parity(workload_index=1, layer=0, p=None, check_sets=True, heads=N
         report["mean_abs"] = max(report["mean_abs"], entry["mean_abs"])
         assert entry["max_abs"] <= MAX_ABS and entry["mean_abs"] <= MEAN_ABS, entry
         report["heads"].append(entry)
-    report["layer"] = lay
     return report

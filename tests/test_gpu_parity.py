@@ -134,9 +134,9 @@ def test_qwen_layer_32k_parity():
 
 @pytest.mark.parametrize("G,N", [(8, 600_000), (4, 700_000)])
 def test_two_wave_schedule(G, N):
-    """Two retrieval groups whose chunks at the shared-memory score capacity (at most
-    227 KB / (4 G) tokens per CTA) need more than one wave of 148 CTAs: the chunks run in two
-    waves, and a group's phases wait on chunks of both waves."""
+    """Two retrieval groups with more rows than one chunk per CTA holds at the tensor-memory
+    score capacity (16384 rows per CTA for G <= 4, 8192 for G = 8; 1.2-1.4M rows over at most
+    148 CTAs): CTAs take two chunks, and a group's phases wait on chunks of both waves."""
     w = _small(G=G, Hkv=2, seq=(N,), window=2048, ret=(True, True))
     heads = [(0, 0), (0, G - 1), (0, G), (0, 2 * G - 1)]
     rep = _parity().run_layer_parity(w=w, layer=0, source="gpu", heads=heads)
@@ -155,36 +155,89 @@ def _kv(w, layer, retrieval):
 
 def test_full_size_128k_b4_layer():
     """128K x 4 (Qwen3-8B shape), a layer with three retrieval KV heads: twelve groups whose
-    chunks need two waves; heads of the last and first groups and one local head."""
+    chunks need two waves; every query head of two groups (the last sequence's last group,
+    the first sequence's first group) and one local head."""
     w = workloads.workload(3)
     layer = _layer_with(w, 3)
     ret, loc = _kv(w, layer, True), _kv(w, layer, False)
-    heads = [(3, ret[-1] * w.G), (3, ret[-1] * w.G + w.G - 1), (0, ret[0] * w.G + 1),
-             (2, loc[0] * w.G)]
+    heads = [(3, ret[-1] * w.G + i) for i in range(w.G)] + \
+            [(0, ret[0] * w.G + i) for i in range(w.G)] + [(2, loc[0] * w.G)]
     rep = _parity().run_layer_parity(w=w, layer=layer, source="gpu", heads=heads)
     assert all(e["count"] > 0 for e in rep["heads"])
 
 
 def test_full_size_1m_layer():
-    """1M tokens (B = 1), a layer with two retrieval KV heads (chunks in two waves): two query
-    heads of the second group."""
+    """1M tokens (B = 1), a layer with two retrieval KV heads (chunks in two waves): every
+    query head of the second group."""
     w = workloads.workload(4)
     layer = _layer_with(w, 2)
     g = _kv(w, layer, True)[-1]
-    heads = [(0, g * w.G), (0, g * w.G + w.G - 1)]
+    heads = [(0, g * w.G + i) for i in range(w.G)]
     rep = _parity().run_layer_parity(w=w, layer=layer, source="gpu", heads=heads)
     assert all(e["retrieval"] and e["count"] > 0 for e in rep["heads"])
 
 
-def test_full_size_ragged_b64_layer():
-    """Ragged batch of 64 sequences (8K-64K tokens): retrieval heads of the first and last
-    sequences and a local head of a middle one."""
+def test_recomputed_scores_1m_four_groups():
+    """1M tokens, a layer with four retrieval KV heads: 4M index rows over at most 148 CTAs
+    is more than the 16384 rows whose scores one CTA's tensor memory holds, so the CTAs' later
+    chunks recompute their scores from the index rows in phases H and W (the recompute path
+    and its global per-warp lists). Every query head of the last group (whose chunks come
+    last on each CTA) and one head of the first."""
+    w = workloads.workload(4)
+    layer = _layer_with(w, 4)
+    ret = _kv(w, layer, True)
+    assert len(ret) == 4 and w.G == 4
+    assert 4 * int(w.seq_lens[0]) > 148 * 16384
+    heads = [(0, ret[-1] * w.G + i) for i in range(w.G)] + [(0, ret[0] * w.G)]
+    rep = _parity().run_layer_parity(w=w, layer=layer, source="gpu", heads=heads)
+    assert all(e["retrieval"] and e["count"] > 0 for e in rep["heads"])
+
+
+@pytest.mark.parametrize("p", [0.8, 0.95])
+def test_full_size_ragged_b64_other_p(p):
+    """The ragged batch of 64 sequences at the other two top-p values the workload draws
+    from: the retrieval heads of three sequences (first, middle, last)."""
     w = workloads.workload(5)
     layer = _layer_with(w, 1)
-    ret, loc = _kv(w, layer, True), _kv(w, layer, False)
-    heads = [(0, ret[0] * w.G), (63, ret[0] * w.G + 1), (31, loc[0] * w.G + 2)]
-    rep = _parity().run_layer_parity(w=w, layer=layer, source="gpu", heads=heads)
+    ret = _kv(w, layer, True)
+    heads = [(b, ret[0] * w.G + i) for b in (0, 31, 63) for i in (0, w.G - 1)]
+    rep = _parity().run_layer_parity(w=w, layer=layer, p=p, source="gpu", heads=heads)
     assert all(e["count"] > 0 for e in rep["heads"])
+
+
+def test_wait_timeout_then_recovery():
+    """A device-side wait that runs out: with the wait limit at one SM cycle, a fused
+    decode + append (the CTA holding the decode token appends it before it arrives, so the
+    group's other CTAs reach their wait first) returns through RTP_ETIMEOUT in the status
+    word, without hanging; after rtp_workspace_init and with the default limit, the same
+    layer (the token appended again, the same rows) decodes with parity."""
+    from long_context_sparse_rtpurbo_b200 import rtp
+    from long_context_sparse_rtpurbo_b200._lib import RTP_ETIMEOUT
+    P = _parity()
+    w = _small(G=4, Hkv=2, seq=(300_000,), window=2048, ret=(True, False))
+    seq = np.asarray(w.seq_lens, np.int64)
+    q, wq, wk = P.layer_inputs(w, 0, DEV)
+    kb, vb = _token_bits(w, 0, seq)
+    k_new, v_new = P.bits_to_torch(kb, DEV), P.bits_to_torch(vb, DEV)
+    sl = torch.as_tensor(seq.astype(np.int32), device=DEV)
+    lay = P.make_layer(w, 0, DEV)
+    P.fill_layer(w, 0, lay, wk, seq - 1, source="gpu", device=DEV)
+    out = torch.zeros((w.B, w.Hq, 128), dtype=torch.bfloat16, device=DEV)
+    cnt = torch.zeros((w.B, w.Hq), dtype=torch.int32, device=DEV)
+    try:
+        rtp.rtp_debug_set_wait_limit(1)
+        lay.decode_append(k_new, v_new, wk, q, wq, sl, w.p, out, cnt)
+        st = lay.status()
+    finally:
+        rtp.rtp_debug_set_wait_limit(0)
+    assert st == RTP_ETIMEOUT
+    rtp.rtp_workspace_init(lay.ws)
+    lay.append(k_new.view(w.B, 1, w.Hkv, 128), v_new.view(w.B, 1, w.Hkv, 128), wk,
+               torch.as_tensor((seq - 1).astype(np.int32), device=DEV))
+    out, cnt, sel = P.decode(lay, q, wq, seq, w.p, DEV, with_sel=True)
+    assert lay.status() == 0
+    heads = [(0, i) for i in range(w.G)] + [(0, w.G)]
+    P.check_outputs(w, 0, seq, w.p, out, cnt, sel, heads)
 
 
 def _token_bits(w, layer, seq_lens):
@@ -199,7 +252,7 @@ def _token_bits(w, layer, seq_lens):
     return kb, vb
 
 
-@pytest.mark.parametrize("case", ["mix", "ragged", "waves"])
+@pytest.mark.parametrize("case", ["mix", "ragged", "waves", "local", "local_ragged"])
 def test_fused_append_equals_two_calls(case):
     """rtp_decode_step_append equals rtp_append_kv (n_new = 1) followed by rtp_decode_step:
     identical caches, counts and outputs, bit for bit (the same arithmetic runs in both)."""
@@ -208,8 +261,12 @@ def test_fused_append_equals_two_calls(case):
         w = _small(G=4, Hkv=2, seq=(5000,))
     elif case == "ragged":      # N = 1, N < sinks, N around the ring's wrap, a long one
         w = _small(B=6, Hkv=2, seq=(1, 3, 259, 260, 261, 5000), kind="needle")
-    else:                       # two groups in two waves
+    elif case == "waves":       # two groups in two waves
         w = _small(G=8, Hkv=2, seq=(600_000,), window=2048, ret=(True, True))
+    elif case == "local":       # no retrieval head: only local items
+        w = _small(G=4, Hkv=2, seq=(5000,), ret=(False, False))
+    else:                       # only local heads, ragged lengths
+        w = _small(B=6, Hkv=2, seq=(1, 3, 259, 260, 261, 5000), kind="needle", ret=(False, False))
     seq = np.asarray(w.seq_lens, np.int64)
     q, wq, wk = P.layer_inputs(w, 0, DEV)
     kb, vb = _token_bits(w, 0, seq)
