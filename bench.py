@@ -6,8 +6,12 @@ current token and the decode step, for the whole batch, in one launch (rtp_decod
 graph. Metric: decode layer-steps/s (a layer-step is one layer over the whole batch), plus the
 achieved HBM bandwidth of the algorithmic bytes the step must move.
 
-  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload 2] [--impl ours|reference]
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload 4] [--extra 2,3,5]
+                  [--impl ours|reference]
 
+The headline line is the 1M-token workload (4); the 32K (2), 128K x 4 (3) and ragged B = 64
+(5, at p = 0.8, 0.9 and 0.95) workloads are measured in the same run and reported under
+"extra", each with its own roofline and ms_per_step (--extra "" skips them).
 With N > 1 (torchrun), every rank runs an independent replica of the workload on its GPU
 (no data-path collective); value = layer-steps of all ranks / max-over-ranks time.
 """
@@ -174,6 +178,61 @@ def oracle_layer_steps(w, prepared, budget_s: float, max_steps=None):
             return done, spent
 
 
+def _layer_inputs_f64(w, l, pairs):
+    from synth import gen
+    q = gen.bf16_bits_to_f32(w.q_pre_bits(l)).astype(np.float64)
+    kp = {(b, g): gen.bf16_bits_to_f32(w.kpre_bits(l, b, g, 0, int(w.seq_lens[b]))).astype(np.float64)
+          for b, g in pairs}
+    vv = {(b, g): gen.bf16_bits_to_f32(w.v_bits(l, b, g, 0, int(w.seq_lens[b]))).astype(np.float64)
+          for b, g in pairs}
+    return q, kp, vv
+
+
+def oracle_full_step(w):
+    """Times the oracle on one whole step: every layer, every head of every sequence (the
+    inputs of each layer generated untimed, layer by layer). Returns (layer-steps, seconds)."""
+    from oracle import rtp_oracle as O
+    spent = 0.0
+    for l in range(w.layers):
+        q, kp, vv = _layer_inputs_f64(w, l, [(b, g) for b in range(w.B) for g in range(w.Hkv)])
+        t0 = time.perf_counter()
+        O.decode_layer(q, w.w_qidx(l), w.w_kidx(l), lambda b, g: kp[(b, g)],
+                       lambda b, g: vv[(b, g)], w.ret_mask[l], w.seq_lens, w.p, w.sinks, w.window,
+                       w.rope_base)
+        spent += time.perf_counter() - t0
+        del q, kp, vv
+    return w.layers, spent
+
+
+def oracle_group_sample(w):
+    """Bounded oracle sample for long contexts: the G query heads of one retrieval KV head
+    and of one local KV head of sequence 0, each timed once; a step is scaled from them by
+    the workload's mix of retrieval and local (sequence, KV head) pairs over all layers.
+    Returns (layer-steps/s, seconds spent, description)."""
+    from oracle import rtp_oracle as O
+    l = next(i for i in range(w.layers) if w.ret_mask[i].any() and not w.ret_mask[i].all())
+    g_r = int(np.nonzero(w.ret_mask[l])[0][0])
+    g_l = int(np.nonzero(~w.ret_mask[l])[0][0])
+    t = {}
+    for g in (g_r, g_l):
+        q, kp, vv = _layer_inputs_f64(w, l, [(0, g)])
+        heads = [(0, g * w.G + i) for i in range(w.G)]
+        t0 = time.perf_counter()
+        O.decode_layer(q, w.w_qidx(l), w.w_kidx(l), lambda b, gg: kp[(b, gg)],
+                       lambda b, gg: vv[(b, gg)], w.ret_mask[l], w.seq_lens, w.p, w.sinks,
+                       w.window, w.rope_base, heads=heads)
+        t[g] = time.perf_counter() - t0
+        del q, kp, vv
+    n_ret = int(w.ret_mask.sum()) * w.B
+    n_loc = int((~w.ret_mask).sum()) * w.B
+    step_s = n_ret * t[g_r] + n_loc * t[g_l]
+    desc = (f"{w.name}: the {w.G} query heads of retrieval KV head {g_r} and of local KV head "
+            f"{g_l} of layer {l}, sequence 0, timed once each ({t[g_r]:.2f} s, {t[g_l]:.3f} s of "
+            f"float64 NumPy); a {w.layers}-layer step scaled as {n_ret} retrieval + {n_loc} local "
+            f"(sequence, KV head) pairs")
+    return w.layers / step_s, t[g_r] + t[g_l], desc
+
+
 def sample_layers(w):
     """A retrieval-head layer and a local-only (or the next) layer: the two kinds of layer-step."""
     ret = [l for l in range(w.layers) if w.ret_mask[l].any()]
@@ -233,9 +292,9 @@ def _bits_to_dev(bits, dev):
     return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).to(dev)
 
 
-def _traffic(kernel: str):
-    """DRAM bytes per launch of ``kernel`` from a committed ncu summary, if it was taken on the
-    current source (its sha256 recorded beside it); else None."""
+def _traffic(kernel: str, workload: str):
+    """DRAM bytes per launch of ``kernel`` on ``workload`` from a committed ncu summary, if it
+    was taken on the current source (its sha256 recorded beside it); else None."""
     import hashlib
     p = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(p):
@@ -247,19 +306,261 @@ def _traffic(kernel: str):
     for name in sorted(os.listdir(src)):
         with open(os.path.join(src, name), "rb") as f:
             h.update(f.read())
-    e = d.get(kernel)
+    e = d.get(f"{kernel}/{workload}")
     if not e or e.get("source_sha256") != h.hexdigest():
         return None
     return e
+
+
+class GpuWorkload:
+    """Every layer of a workload on one GPU: caches filled by the counter-stream fill kernel
+    up to position N - 1, the decode token's k / v and the query packed per layer (the step's
+    input), outputs per layer. measure(p) times one step per CUDA-graph replay."""
+
+    def __init__(self, w, dev, fused):
+        import torch
+        from long_context_sparse_rtpurbo_b200.layer import DecodeLayer
+        from synth.gpu import LayerFiller
+        self.w, self.dev, self.fused = w, dev, fused
+        N = np.asarray(w.seq_lens, np.int64)
+        self.N = N
+        B, Hq, Hkv, Lyr = w.B, w.Hq, w.Hkv, w.layers
+        nq, nk = B * Hq * 128, B * Hkv * 128
+        per_layer_in = nq + 2 * nk
+        self.inp = torch.empty(Lyr * per_layer_in, dtype=torch.bfloat16, device=dev)
+        self.out_all = torch.empty((Lyr, B, Hq, 128), dtype=torch.bfloat16, device=dev)
+        self.cnt_all = torch.empty((Lyr, B, Hq), dtype=torch.int32, device=dev)
+        self.layers = []
+        t_fill = time.perf_counter()
+        chunk = max(1024, min(16384, (1 << 27) // max(1, B * Hkv * 128 * 2)))
+        for l in range(Lyr):
+            lay = DecodeLayer(B, Hq, Hkv, w.sinks, w.window, int(N.max()), w.ret_mask[l], N, dev,
+                              w.rope_base)
+            wq = torch.from_numpy(np.array(w.w_qidx(l))).to(dev)
+            wk = torch.from_numpy(np.array(w.w_kidx(l))).to(dev)
+            filler = LayerFiller(w, l, dev)
+            top = int(N.max()) - 1
+            for t0 in range(0, top, chunk):
+                n = min(chunk, top - t0)
+                nv = np.clip(N - 1 - t0, 0, n).astype(np.int32)
+                k, v = filler.fill(np.full(B, t0), n, nv)
+                lay.append(k, v, wk, torch.full((B,), t0, dtype=torch.int32, device=dev),
+                           torch.from_numpy(nv).to(dev))
+            base = l * per_layer_in
+            q = self.inp[base:base + nq].view(B, Hq, 128)
+            knew = self.inp[base + nq:base + nq + nk].view(B, 1, Hkv, 128)
+            vnew = self.inp[base + nq + nk:base + per_layer_in].view(B, 1, Hkv, 128)
+            q.copy_(_bits_to_dev(w.q_pre_bits(l), dev))
+            kk, vv = filler.fill(N - 1, 1)
+            knew.copy_(kk)
+            vnew.copy_(vv)
+            self.layers.append(dict(lay=lay, q=q, wq=wq, wk=wk, knew=knew, vnew=vnew,
+                                    start=torch.tensor(N - 1, dtype=torch.int32, device=dev),
+                                    seq=torch.tensor(N, dtype=torch.int32, device=dev),
+                                    out=self.out_all[l], cnt=self.cnt_all[l]))
+            del filler
+        torch.cuda.synchronize()
+        self.setup_s = time.perf_counter() - t_fill
+
+    def step(self, p, with_append=True, launches=None):
+        from long_context_sparse_rtpurbo_b200 import rtp
+        w = self.w
+        B, Hkv = w.B, w.Hkv
+        for L in self.layers:
+            if with_append and self.fused:     # append + decode in one launch
+                L["lay"].decode_append(L["knew"].view(B, Hkv, 128), L["vnew"].view(B, Hkv, 128),
+                                       L["wk"], L["q"], L["wq"], L["seq"], p, L["out"], L["cnt"])
+                if launches is not None:
+                    launches[0] += rtp.rtp_last_launch_count()
+                continue
+            if with_append:
+                L["lay"].append(L["knew"], L["vnew"], L["wk"], L["start"])
+                if launches is not None:
+                    launches[0] += rtp.rtp_last_launch_count()
+            L["lay"].decode(L["q"], L["wq"], L["seq"], p, L["out"], L["cnt"])
+            if launches is not None:
+                launches[0] += rtp.rtp_last_launch_count()
+
+    def selections(self, p):
+        """Union sizes of the selected sets per retrieval (sequence, KV head) and the
+        per-head counts (untimed, through sel_idx), for the algorithmic byte count."""
+        import torch
+        w, N, dev = self.w, self.N, self.dev
+        B, Hq, Hkv = w.B, w.Hq, w.Hkv
+        unions, conc, diff, allc = [], [], [], []
+        for l, L in enumerate(self.layers):
+            u = {}
+            if w.ret_mask[l].any():
+                sel = torch.full((B, Hq, int(N.max())), -1, dtype=torch.int32, device=dev)
+                cnt = torch.empty((B, Hq), dtype=torch.int32, device=dev)
+                out = torch.empty((B, Hq, 128), dtype=torch.bfloat16, device=dev)
+                L["lay"].decode(L["q"], L["wq"], L["seq"], p, out, cnt, sel)
+                c = cnt.cpu().numpy()
+                for b in range(B):
+                    for g in range(Hkv):
+                        if not w.ret_mask[l, g]:
+                            continue
+                        hs = range(g * w.G, (g + 1) * w.G)
+                        parts = [sel[b, h, :int(c[b, h])] for h in hs]
+                        u[(b, g)] = int(torch.unique(torch.cat(parts)).numel())
+                        for h in hs:
+                            kind = w.group_layout(l, b, g).targets[h % w.G][0]
+                            (conc if kind == "conc" else diff).append(int(c[b, h]))
+                            allc.append(int(c[b, h]))
+                del sel
+            unions.append(u)
+            st = L["lay"].status()
+            if st != 0:
+                raise RuntimeError(f"device status {st} in layer {l}")
+        return unions, conc, diff, allc
+
+    def measure(self, p, args, world, e2e=False):
+        import torch
+        import torch.distributed as dist
+        w, dev, fused = self.w, self.dev, self.fused
+        Lyr = w.layers
+        launches = [0]
+        self.step(p, launches=launches)        # eager (kernel attributes set outside capture)
+        per_step_launches = launches[0]
+        unions, conc, diff, allc = self.selections(p)
+        step_bytes = algorithmic_bytes(w, unions, include_append=True)
+        dec_bytes = algorithmic_bytes(w, unions, include_append=False)
+        side = torch.cuda.Stream(device=dev)
+        side.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(side):
+            self.step(p)
+            g_full = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g_full, stream=side):
+                self.step(p)
+            g_dec = torch.cuda.CUDAGraph()                  # the decode kernel alone
+            with torch.cuda.graph(g_dec, stream=side):
+                self.step(p, with_append=fused)
+        torch.cuda.current_stream().wait_stream(side)
+        torch.cuda.synchronize()
+
+        def barrier():
+            if world > 1:
+                dist.barrier()
+
+        def timed(fn, k):
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            torch.cuda.synchronize()
+            barrier()
+            torch.cuda.synchronize()
+            e0.record()
+            for _ in range(k):
+                fn()
+            e1.record()
+            torch.cuda.synchronize()
+            barrier()
+            return e0.elapsed_time(e1)
+
+        for _ in range(args.warmup):
+            g_full.replay()
+        torch.cuda.synchronize()
+        local = dev.index if dev.index is not None else 0
+        with ClockSampler(local) as clk:
+            t_end = time.perf_counter() + args.preroll      # untimed pre-roll under load
+            while time.perf_counter() < t_end:
+                g_full.replay()
+                torch.cuda.synchronize()
+            torch.cuda.nvtx.range_push("rtp_timed")
+            ms = timed(g_full.replay, args.steps)
+            torch.cuda.nvtx.range_pop()
+            dec_ms = timed(g_dec.replay, args.steps)
+        clocks = clk.summary()
+        ms_step = max_over_ranks(ms / args.steps, world, dev)
+        dec_step = max_over_ranks(dec_ms / args.steps, world, dev)
+        res = {}
+        if e2e:
+            # H2D of the step's inputs from pinned memory, the step, D2H of the outputs
+            inp_host = self.inp.cpu().pin_memory()
+            out_host = torch.empty(self.out_all.shape, dtype=self.out_all.dtype).pin_memory()
+            cnt_host = torch.empty(self.cnt_all.shape, dtype=self.cnt_all.dtype).pin_memory()
+
+            def e2e_step():
+                self.inp.copy_(inp_host, non_blocking=True)
+                g_full.replay()
+                out_host.copy_(self.out_all, non_blocking=True)
+                cnt_host.copy_(self.cnt_all, non_blocking=True)
+
+            for _ in range(max(3, args.warmup)):
+                e2e_step()
+            e2e_ms = max_over_ranks(timed(e2e_step, args.steps) / args.steps, world, dev)
+            h2d = self.inp.numel() * self.inp.element_size()
+            d2h = (self.out_all.numel() * self.out_all.element_size() +
+                   self.cnt_all.numel() * self.cnt_all.element_size())
+            res["e2e"] = {"value": aggregate(Lyr, 1, world, e2e_ms), "unit": "layer-steps/s",
+                          "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                          "ms_per_step": e2e_ms}
+        del g_full, g_dec
+        peak, peak_kind = load_peaks()
+        kern_bytes = step_bytes if fused else dec_bytes   # the fused kernel also appends
+        achieved = kern_bytes / (dec_step * 1e-3) / 1e9
+        tr = _traffic("rtp_decode_step", w.name)
+        N = self.N
+        attended = float(sum(allc)) + sum(min(int(n), w.sinks + w.window) * w.G
+                                          for l in range(Lyr) for n in N
+                                          for g in range(w.Hkv) if not w.ret_mask[l, g])
+        scored = float(sum(int(n) * w.G for l in range(Lyr) for n in N
+                           for g in range(w.Hkv) if w.ret_mask[l, g]))
+        res.update({
+            "value": aggregate(Lyr, 1, world, ms_step), "unit": "layer-steps/s",
+            "ms_per_step": ms_step, "p": p,
+            "config": workload_config(w, "inputs larger than L2 (%.2f GB read per step vs "
+                                         "126 MB L2)" % (step_bytes / 1e9)),
+            "achieved_step_gbs": step_bytes / (ms_step * 1e-3) / 1e9,
+            "step_bytes": step_bytes,
+            "token_heads_per_s": {"attended": attended * world / (ms_step * 1e-3),
+                                  "scored": scored * world / (ms_step * 1e-3)},
+            "roofline": {"kernel": "rtp_decode_step", "bound": "hbm", "achieved": achieved,
+                         "peak": peak, "unit": "GB/s", "frac": achieved / peak,
+                         "peak_kind": peak_kind + " hbm_gbs (copy bandwidth, burst)",
+                         "traffic": None if tr is None else tr["dram_bytes_per_launch"],
+                         "bytes_per_launch": kern_bytes / Lyr,
+                         "launch_us": dec_step * 1e3 / Lyr, "fused_append": fused,
+                         "frac_of_nominal_8tbs": achieved / 8000.0},
+            "gpu_launches": per_step_launches * args.steps,
+            "clocks": clocks,
+            "selected_tokens": {"concentrated_mean": float(np.mean(conc)) if conc else None,
+                                "diffuse_mean": float(np.mean(diff)) if diff else None,
+                                "min": int(min(allc)) if allc else None,
+                                "max": int(max(allc)) if allc else None,
+                                "union_mean": float(np.mean([x for u in unions for x in u.values()]))
+                                if allc else None},
+            "setup_s": self.setup_s,
+        })
+        return res
+
+    def close(self):
+        import torch
+        del self.layers, self.inp, self.out_all, self.cnt_all
+        torch.cuda.empty_cache()
+
+
+def _cpu_baseline(w, budget_s):
+    """The oracle on the host cores: whole layer-steps (alternating a layer with retrieval
+    heads and one without) up to budget_s seconds, or, for contexts beyond 64K tokens, the
+    scaled per-head-group sample."""
+    if int(w.seq_lens.max()) > 65536:
+        v, spent, desc = oracle_group_sample(w)
+        return {"value": v, "unit": "layer-steps/s", "cores": cpu_threads(), "kind": "oracle",
+                "sample": desc}
+    prepared = prepare_oracle_layers(w, sample_layers(w))
+    n_done, spent = oracle_layer_steps(w, prepared, budget_s)
+    return {"value": n_done / spent, "unit": "layer-steps/s", "cores": cpu_threads(),
+            "kind": "oracle",
+            "sample": f"{n_done} whole layer-steps of {w.name} (all heads, alternating layers "
+                      f"{[p[0] for p in prepared]}: one with retrieval heads, one without), "
+                      f"{spent:.1f} s of float64 NumPy"}
 
 
 def run_ours(args, w):
     import datetime
     import torch
     import torch.distributed as dist
-    from long_context_sparse_rtpurbo_b200 import rtp
-    from long_context_sparse_rtpurbo_b200.layer import DecodeLayer
-    from synth.gpu import LayerFiller
+    from synth import workloads
 
     rank, world, local = dist_env()
     if world > 1:
@@ -267,220 +568,53 @@ def run_ours(args, w):
                                 device_id=torch.device("cuda", local))
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
-    N = np.asarray(w.seq_lens, np.int64)
-    B, Hq, Hkv, Lyr = w.B, w.Hq, w.Hkv, w.layers
-    # packed per-step inputs (q of all layers, current-token k/v) and outputs
-    nq, nk = B * Hq * 128, B * Hkv * 128
-    per_layer_in = nq + 2 * nk
-    inp = torch.empty(Lyr * per_layer_in, dtype=torch.bfloat16, device=dev)
-    out_all = torch.empty((Lyr, B, Hq, 128), dtype=torch.bfloat16, device=dev)
-    cnt_all = torch.empty((Lyr, B, Hq), dtype=torch.int32, device=dev)
-    layers = []
-    t_fill = time.perf_counter()
-    chunk = max(1024, min(16384, (1 << 27) // max(1, B * Hkv * 128 * 2)))
-    for l in range(Lyr):
-        lay = DecodeLayer(B, Hq, Hkv, w.sinks, w.window, int(N.max()), w.ret_mask[l], N, dev,
-                          w.rope_base)
-        wq = torch.from_numpy(np.array(w.w_qidx(l))).to(dev)
-        wk = torch.from_numpy(np.array(w.w_kidx(l))).to(dev)
-        filler = LayerFiller(w, l, dev)
-        top = int(N.max()) - 1
-        for t0 in range(0, top, chunk):
-            n = min(chunk, top - t0)
-            nv = np.clip(N - 1 - t0, 0, n).astype(np.int32)
-            k, v = filler.fill(np.full(B, t0), n, nv)
-            lay.append(k, v, wk, torch.full((B,), t0, dtype=torch.int32, device=dev),
-                       torch.from_numpy(nv).to(dev))
-        base = l * per_layer_in
-        q = inp[base:base + nq].view(B, Hq, 128)
-        knew = inp[base + nq:base + nq + nk].view(B, 1, Hkv, 128)
-        vnew = inp[base + nq + nk:base + per_layer_in].view(B, 1, Hkv, 128)
-        q.copy_(_bits_to_dev(w.q_pre_bits(l), dev))
-        kk, vv = filler.fill(N - 1, 1)
-        knew.copy_(kk)
-        vnew.copy_(vv)
-        layers.append(dict(lay=lay, q=q, wq=wq, wk=wk, knew=knew, vnew=vnew,
-                           start=torch.tensor(N - 1, dtype=torch.int32, device=dev),
-                           seq=torch.tensor(N, dtype=torch.int32, device=dev),
-                           out=out_all[l], cnt=cnt_all[l]))
-        del filler
-    torch.cuda.synchronize()
-    t_fill = time.perf_counter() - t_fill
-
-    launches = {"n": 0}
-
     fused = not args.separate_append
 
-    def step(with_append=True, count=False):
-        for L in layers:
-            if with_append and fused:          # append + decode in one launch
-                L["lay"].decode_append(L["knew"].view(B, Hkv, 128), L["vnew"].view(B, Hkv, 128),
-                                       L["wk"], L["q"], L["wq"], L["seq"], w.p, L["out"],
-                                       L["cnt"])
-                if count:
-                    launches["n"] += rtp.rtp_last_launch_count()
-                continue
-            if with_append:
-                L["lay"].append(L["knew"], L["vnew"], L["wk"], L["start"])
-                if count:
-                    launches["n"] += rtp.rtp_last_launch_count()
-            L["lay"].decode(L["q"], L["wq"], L["seq"], w.p, L["out"], L["cnt"])
-            if count:
-                launches["n"] += rtp.rtp_last_launch_count()
-
-    # one eager step (sets kernel attributes outside capture), then the unions of the
-    # selected sets (untimed, with sel_idx) for the algorithmic byte count
-    step(count=True)
-    per_step_launches = launches["n"]
-    unions, conc, diff, allc = [], [], [], []
-    for l, L in enumerate(layers):
-        u = {}
-        if w.ret_mask[l].any():
-            sel = torch.full((B, Hq, int(N.max())), -1, dtype=torch.int32, device=dev)
-            cnt = torch.empty((B, Hq), dtype=torch.int32, device=dev)
-            out = torch.empty((B, Hq, 128), dtype=torch.bfloat16, device=dev)
-            L["lay"].decode(L["q"], L["wq"], L["seq"], w.p, out, cnt, sel)
-            c = cnt.cpu().numpy()
-            for b in range(B):
-                for g in range(Hkv):
-                    if not w.ret_mask[l, g]:
-                        continue
-                    hs = range(g * w.G, (g + 1) * w.G)
-                    parts = [sel[b, h, :int(c[b, h])] for h in hs]
-                    u[(b, g)] = int(torch.unique(torch.cat(parts)).numel())
-                    for h in hs:
-                        kind = w.group_layout(l, b, g).targets[h % w.G][0]
-                        (conc if kind == "conc" else diff).append(int(c[b, h]))
-                        allc.append(int(c[b, h]))
-            del sel
-        unions.append(u)
-        st = L["lay"].status()
-        if st != 0:
-            raise RuntimeError(f"device status {st} in layer {l}")
-    step_bytes = algorithmic_bytes(w, unions, include_append=True)
-    dec_bytes = algorithmic_bytes(w, unions, include_append=False)
-
-    side = torch.cuda.Stream(device=dev)
-    side.wait_stream(torch.cuda.current_stream())
-    with torch.cuda.stream(side):
-        step()
-        g_full = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g_full, stream=side):
-            step()
-        g_dec = torch.cuda.CUDAGraph()                      # the decode kernel alone
-        with torch.cuda.graph(g_dec, stream=side):
-            step(with_append=fused)
-    torch.cuda.current_stream().wait_stream(side)
-    torch.cuda.synchronize()
-
-    def barrier():
-        if world > 1:
-            dist.barrier()
-
-    def timed(fn, k):
-        e0 = torch.cuda.Event(enable_timing=True)
-        e1 = torch.cuda.Event(enable_timing=True)
-        torch.cuda.synchronize()
-        barrier()
-        torch.cuda.synchronize()
-        e0.record()
-        for _ in range(k):
-            fn()
-        e1.record()
-        torch.cuda.synchronize()
-        barrier()
-        return e0.elapsed_time(e1)
-
-    for _ in range(args.warmup):
-        g_full.replay()
-    torch.cuda.synchronize()
-    with ClockSampler(local) as clk:
-        t_end = time.perf_counter() + args.preroll          # untimed pre-roll under load
-        while time.perf_counter() < t_end:
-            g_full.replay()
-            torch.cuda.synchronize()
-        torch.cuda.nvtx.range_push("rtp_timed")
-        ms = timed(g_full.replay, args.steps)
-        torch.cuda.nvtx.range_pop()
-        dec_ms = timed(g_dec.replay, args.steps)
-    clocks = clk.summary()
-    ms_step = max_over_ranks(ms / args.steps, world, dev)
-    dec_step = max_over_ranks(dec_ms / args.steps, world, dev)
-
-    # end to end: H2D of the step's inputs from pinned memory, the step, D2H of the outputs
-    inp_host = inp.cpu().pin_memory()
-    out_host = torch.empty(out_all.shape, dtype=out_all.dtype).pin_memory()
-    cnt_host = torch.empty(cnt_all.shape, dtype=cnt_all.dtype).pin_memory()
-
-    def e2e_step():
-        inp.copy_(inp_host, non_blocking=True)
-        g_full.replay()
-        out_host.copy_(out_all, non_blocking=True)
-        cnt_host.copy_(cnt_all, non_blocking=True)
-
+    gw = GpuWorkload(w, dev, fused)
+    m = gw.measure(w.p, args, world, e2e=not args.no_e2e)
+    gw.close()
+    del gw
     if args.no_e2e:
-        e2e_ms = float("nan")
-    else:
-        for _ in range(max(3, args.warmup)):
-            e2e_step()
-        e2e_ms = max_over_ranks(timed(e2e_step, args.steps) / args.steps, world, dev)
-    h2d = inp.numel() * inp.element_size()
-    d2h = out_all.numel() * out_all.element_size() + cnt_all.numel() * cnt_all.element_size()
-
-    value = aggregate(Lyr, 1, world, ms_step)
-    peak, peak_kind = load_peaks()
-    kern_bytes = step_bytes if fused else dec_bytes       # the fused kernel also appends
-    achieved = kern_bytes / (dec_step * 1e-3) / 1e9
-    tr = _traffic("rtp_decode_step")
-    attended = float(sum(allc)) + sum(min(int(n), w.sinks + w.window) * w.G
-                                      for l in range(Lyr) for n in N
-                                      for g in range(Hkv) if not w.ret_mask[l, g])
-    scored = float(sum(int(n) * w.G for l in range(Lyr) for n in N
-                       for g in range(Hkv) if w.ret_mask[l, g]))
-    line = {
-        "metric": METRIC, "value": value, "unit": "layer-steps/s", "n_gpus": world,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
-        "data": "synthetic",
-        "config": workload_config(w, "inputs larger than L2 (%.2f GB read per step vs 126 MB L2)"
-                                  % (step_bytes / 1e9)),
-        "achieved_step_gbs": step_bytes / (ms_step * 1e-3) / 1e9 * 1.0,
-        "step_bytes": step_bytes,
-        "token_heads_per_s": {"attended": attended * world / (ms_step * 1e-3),
-                              "scored": scored * world / (ms_step * 1e-3)},
-        "roofline": {"kernel": "rtp_decode_step", "bound": "hbm", "achieved": achieved,
-                     "peak": peak, "unit": "GB/s", "frac": achieved / peak,
-                     "peak_kind": peak_kind + " hbm_gbs (copy bandwidth)",
-                     "traffic": None if tr is None else tr["dram_bytes_per_launch"],
-                     "bytes_per_launch": kern_bytes / Lyr, "launch_us": dec_step * 1e3 / Lyr,
-                     "fused_append": fused, "frac_of_nominal_8tbs": achieved / 8000.0},
-        "e2e": {"value": aggregate(Lyr, 1, world, e2e_ms), "unit": "layer-steps/s",
-                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
-        "gpu_launches": per_step_launches * args.steps,
-        "clocks": clocks,
-        "selected_tokens": {"concentrated_mean": float(np.mean(conc)) if conc else None,
-                            "diffuse_mean": float(np.mean(diff)) if diff else None,
-                            "min": int(min(allc)) if allc else None,
-                            "max": int(max(allc)) if allc else None,
-                            "union_mean": float(np.mean([x for u in unions for x in u.values()]))
-                            if allc else None},
-        "setup_s": t_fill,
-    }
+        m["e2e"] = {"value": float("nan"), "unit": "layer-steps/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0, "ms_per_step": float("nan")}
+    line = {"metric": METRIC, "value": m.pop("value"), "unit": m.pop("unit"), "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": m.pop("ms_per_step"),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic"}
+    line.update(m)
+    extra = {}
+    for spec in [x for x in (args.extra or "").split(",") if x.strip()]:
+        wi = int(spec)
+        if wi == args.workload:
+            continue
+        we = workloads.workload(wi)
+        if args.layers:
+            we.layers = min(we.layers, args.layers)
+        ps = [0.8, 0.9, 0.95] if wi == 5 else [we.p]
+        gw = GpuWorkload(we, dev, fused)
+        for p in ps:
+            me = gw.measure(p, args, world)
+            key = we.name if len(ps) == 1 else f"{we.name}@p={p}"
+            extra[key] = me
+        gw.close()
+        del gw
+    if extra:
+        line["extra"] = extra
     if rank == 0 and world == 1 and not args.no_cpu:
-        del layers
-        torch.cuda.empty_cache()
-        prepared = prepare_oracle_layers(w, sample_layers(w))
-        n_done, spent = oracle_layer_steps(w, prepared, args.cpu_budget)
-        line["cpu_baseline"] = {"value": n_done / spent, "unit": "layer-steps/s",
-                                "cores": cpu_threads(), "kind": "oracle",
-                                "sample": f"{n_done} whole layer-steps of {w.name} (all heads, "
-                                          f"alternating layers {[p[0] for p in prepared]}: one "
-                                          f"with retrieval heads, one without), {spent:.1f} s of "
-                                          f"float64 NumPy"}
+        line["cpu_baseline"] = _cpu_baseline(w, args.cpu_budget)
+        for key, me in extra.items():
+            if me["config"]["workload"] == "qwen3-8b-32k-b1":   # one whole 36-layer step
+                we = workloads.workload(2)
+                if args.layers:
+                    we.layers = min(we.layers, args.layers)
+                n, spent = oracle_full_step(we)
+                me["cpu_baseline"] = {"value": n / spent, "unit": "layer-steps/s",
+                                      "cores": cpu_threads(), "kind": "oracle",
+                                      "sample": f"one whole step of {we.name}: all {n} layers, "
+                                                f"every head, {spent:.1f} s of float64 NumPy"}
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:
-        del g_full, g_dec
         dist.barrier()
         dist.destroy_process_group()
 
@@ -490,7 +624,9 @@ def main(argv=None):
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--workload", type=int, default=2)
+    ap.add_argument("--workload", type=int, default=4)
+    ap.add_argument("--extra", default="2,3,5",
+                    help="workloads measured in the same run and reported under 'extra'")
     ap.add_argument("--p", type=float, default=None)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--cpu-budget", type=float, default=12.0)

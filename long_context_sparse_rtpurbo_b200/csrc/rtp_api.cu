@@ -152,11 +152,14 @@ int dev_info(DevInfo& di) {
 }
 
 // Ring rows per local item (RL, a multiple of the 16-row tile, at least 64) and items per
-// local group (PL): about 256 rows per item; in a layer without retrieval heads the items
-// are the whole launch, so they are cut to about one per CTA.
+// local group (PL): about as many items as CTAs (an item's fixed costs, the query, the merge
+// of the warps and of the items, are paid per item, its rows stream at the tile loop's
+// rate), but at least 256 rows each; a layer without retrieval heads has only local items,
+// so they are cut to about one per CTA.
 void local_split(const LayerShape& L, int n_lgroups, int n_ret, int P, int& PL, int& RL) {
   const int64_t rows = std::min<int64_t>(L.maxN, L.ring);
-  int64_t pl = (rows + 255) / 256;
+  int64_t pl = n_lgroups > 0 ? (P + n_lgroups - 1) / n_lgroups : 1;
+  pl = std::min<int64_t>(pl, (rows + 255) / 256);
   if (n_ret == 0 && n_lgroups > 0) pl = std::max<int64_t>(pl, P / n_lgroups);
   pl = std::max<int64_t>(pl, 1);
   int64_t rl = (rows + pl - 1) / pl;

@@ -125,26 +125,30 @@ __device__ __forceinline__ void warp_attn_init(WarpAttn& W, const unsigned char*
   W.qb = smem_u32(qbuf);
 }
 
-// Copies up to 16 rows into a tile: lane l handles row l / 2 (both K and V, the 16-byte
-// chunks of parity l & 1, XOR-swizzled by the row). Rows with ok = false get zero V (their
-// logits are masked; a zero V keeps stale shared memory out of the P V product).
+// Copies up to 16 rows into a tile. Lane 2 r holds row r's pointers and flag (the caller's
+// lane -> row l / 2 mapping); they are broadcast so that each copy instruction moves two
+// whole rows (lane l: row 2 u + l / 16, 16-byte chunk l % 16 of its K and of its V), every
+// 128-byte line requested once and whole. Chunks are XOR-swizzled by the row. Rows with
+// ok = false get zero V (their logits are masked; a zero V keeps stale shared memory out of
+// the P V product).
 __device__ __forceinline__ void tile_copy(unsigned char* tile, const uint16_t* krow,
                                           const uint16_t* vrow, bool ok) {
-  const int lane = threadIdx.x & 31, i = lane >> 1, part = lane & 1;
-  unsigned char* kd = tile + i * 256;
-  unsigned char* vd = tile + 4096 + i * 256;
-  if (ok) {
+  const int lane = threadIdx.x & 31, c = lane & 15;
+  const unsigned long long kq = reinterpret_cast<unsigned long long>(krow);
+  const unsigned long long vq = reinterpret_cast<unsigned long long>(vrow);
+  const uint32_t okb = __ballot_sync(0xffffffffu, ok);
 #pragma unroll
-    for (int u = 0; u < 8; ++u) {
-      const int c = 2 * u + part;
-      cp_async16(kd + ((c ^ (i & 7)) << 4), krow + c * 8);
-      cp_async16(vd + ((c ^ (i & 7)) << 4), vrow + c * 8);
-    }
-  } else {
-#pragma unroll
-    for (int u = 0; u < 8; ++u) {
-      const int c = 2 * u + part;
-      *reinterpret_cast<uint4*>(vd + ((c ^ (i & 7)) << 4)) = make_uint4(0, 0, 0, 0);
+  for (int u = 0; u < 8; ++u) {
+    const int r = 2 * u + (lane >> 4);
+    const unsigned long long kr = __shfl_sync(0xffffffffu, kq, 2 * r);
+    const unsigned long long vr = __shfl_sync(0xffffffffu, vq, 2 * r);
+    unsigned char* kd = tile + r * 256 + ((c ^ (r & 7)) << 4);
+    unsigned char* vd = tile + 4096 + r * 256 + ((c ^ (r & 7)) << 4);
+    if ((okb >> (2 * r)) & 1u) {
+      cp_async16(kd, reinterpret_cast<const uint16_t*>(kr) + c * 8);
+      cp_async16(vd, reinterpret_cast<const uint16_t*>(vr) + c * 8);
+    } else {
+      *reinterpret_cast<uint4*>(vd) = make_uint4(0, 0, 0, 0);
     }
   }
 }

@@ -428,13 +428,18 @@ struct DecodeCta {
     const long long Tr = (long long)block_sum_int(sumN, sm.ints()) * P.L.n_ret;
     const long long loc_rows = (long long)block_sum_int(sumL, sm.ints()) * P.L.n_loc;
     // CTAs [0, P_ret) take the chunks, the others start on local items at once; the split
-    // follows the bytes of each side (index read twice as a proxy for index and gather)
+    // follows the bytes of each side (index read twice as a proxy for index and gather), but
+    // the chunk CTAs are at least as many as hold the retrieval rows at one tensor-memory
+    // capacity each: a CTA's chunks run their phases one after another (and wait on the other
+    // CTAs' chunks of the same groups), while local items are taken from a queue by whichever
+    // CTA is free, so the retrieval chain is the one to keep short
     C = 1024;
     P_ret = 0;
     if (Tr > 0) {
       const double ret_b = 64.0 * (double)Tr, loc_b = 512.0 * (double)loc_rows;
       const int pr = (int)((double)P.P * ret_b / (ret_b + loc_b) + 0.5);
-      P_ret = max(1, min(P.P, pr));
+      const long long pcap = (Tr + P.C_cap - 1) / P.C_cap;
+      P_ret = max(1, min(P.P, max(pr, (int)min(pcap, (long long)P.P))));
       // chunk size: the fewest steps (chunks per CTA) whose chunks fit the score slot, at
       // most kMaxSteps; C >= C_min keeps the chunks per group within the workspace arrays
       long long steps = (Tr + (long long)P_ret * P.C_cap - 1) / ((long long)P_ret * P.C_cap);
