@@ -233,6 +233,41 @@ def oracle_group_sample(w):
     return w.layers / step_s, t[g_r] + t[g_l], desc
 
 
+def oracle_retained_mass(w, p=None, k=None):
+    """Retained mass of the selected sets, from the oracle, for every retrieval query head of
+    the workload's first layer with two or more retrieval KV heads, sequence 0: the top-p sets
+    (p), or the fixed-budget top-k sets (k). Two shares: of the dense softmax weights over all
+    cached tokens (full attention; DeepRead "Key Results", "Full Attention Strikes Back"
+    §2.3), and of the index-space mass exp(s - max s) the selector works on."""
+    from oracle import rtp_oracle as O
+    from synth import gen
+    layer = next((l for l in range(w.layers) if w.ret_mask[l].sum() >= 2),
+                 next(l for l in range(w.layers) if w.ret_mask[l].any()))
+    N = int(w.seq_lens[0])
+    qb = w.q_pre_bits(layer)
+    masses, imass, sizes = [], [], []
+    for g in np.nonzero(w.ret_mask[layer])[0]:
+        kp = gen.bf16_bits_to_f32(w.kpre_bits(layer, 0, int(g), 0, N)).astype(np.float64)
+        kidx = O.index_keys(kp, w.w_kidx(layer)[g])
+        for h in range(g * w.G, (g + 1) * w.G):
+            q = gen.bf16_bits_to_f32(qb[0, h]).astype(np.float64)
+            s = O.index_scores(O.index_query(q, w.w_qidx(layer)[h]), kidx)
+            sel = O.topk_histogram(s, k) if k else O.topp_histogram(s, p)
+            pos = np.nonzero(sel.mask)[0]
+            masses.append(O.full_attention_mass(q, kp, pos, w.rope_base))
+            e = np.exp(s - s.max())
+            imass.append(float(e[pos].sum() / e.sum()))
+            sizes.append(len(pos))
+    return {"mean": float(np.mean(masses)), "min": float(np.min(masses)),
+            "max": float(np.max(masses)),
+            "index_mass": {"mean": float(np.mean(imass)), "min": float(np.min(imass)),
+                           "max": float(np.max(imass))},
+            "tokens_mean": float(np.mean(sizes)),
+            "tokens_total": int(np.sum(sizes)), "heads": len(masses),
+            "sample": f"every retrieval query head of layer {layer}, sequence 0, of {w.name} "
+                      f"({'top-k k=%d' % k if k else 'top-p p=%g' % p}), float64 oracle"}
+
+
 def sample_layers(w):
     """A retrieval-head layer and a local-only (or the next) layer: the two kinds of layer-step."""
     ret = [l for l in range(w.layers) if w.ret_mask[l].any()]
@@ -362,11 +397,20 @@ class GpuWorkload:
         torch.cuda.synchronize()
         self.setup_s = time.perf_counter() - t_fill
 
-    def step(self, p, with_append=True, launches=None):
+    def step(self, p, with_append=True, launches=None, topk=0):
         from long_context_sparse_rtpurbo_b200 import rtp
         w = self.w
         B, Hkv = w.B, w.Hkv
         for L in self.layers:
+            if topk:                           # fixed-budget top-k: append, then decode
+                if with_append:
+                    L["lay"].append(L["knew"], L["vnew"], L["wk"], L["start"])
+                    if launches is not None:
+                        launches[0] += rtp.rtp_last_launch_count()
+                L["lay"].decode_topk(L["q"], L["wq"], L["seq"], topk, L["out"], L["cnt"])
+                if launches is not None:
+                    launches[0] += rtp.rtp_last_launch_count()
+                continue
             if with_append and self.fused:     # append + decode in one launch
                 L["lay"].decode_append(L["knew"].view(B, Hkv, 128), L["vnew"].view(B, Hkv, 128),
                                        L["wk"], L["q"], L["wq"], L["seq"], p, L["out"], L["cnt"])
@@ -381,7 +425,7 @@ class GpuWorkload:
             if launches is not None:
                 launches[0] += rtp.rtp_last_launch_count()
 
-    def selections(self, p):
+    def selections(self, p, topk=0):
         """Union sizes of the selected sets per retrieval (sequence, KV head) and the
         per-head counts (untimed, through sel_idx), for the algorithmic byte count."""
         import torch
@@ -394,7 +438,10 @@ class GpuWorkload:
                 sel = torch.full((B, Hq, int(N.max())), -1, dtype=torch.int32, device=dev)
                 cnt = torch.empty((B, Hq), dtype=torch.int32, device=dev)
                 out = torch.empty((B, Hq, 128), dtype=torch.bfloat16, device=dev)
-                L["lay"].decode(L["q"], L["wq"], L["seq"], p, out, cnt, sel)
+                if topk:
+                    L["lay"].decode_topk(L["q"], L["wq"], L["seq"], topk, out, cnt, sel)
+                else:
+                    L["lay"].decode(L["q"], L["wq"], L["seq"], p, out, cnt, sel)
                 c = cnt.cpu().numpy()
                 for b in range(B):
                     for g in range(Hkv):
@@ -414,27 +461,28 @@ class GpuWorkload:
                 raise RuntimeError(f"device status {st} in layer {l}")
         return unions, conc, diff, allc
 
-    def measure(self, p, args, world, e2e=False):
+    def measure(self, p, args, world, e2e=False, topk=0):
         import torch
         import torch.distributed as dist
-        w, dev, fused = self.w, self.dev, self.fused
+        w, dev = self.w, self.dev
+        fused = self.fused and not topk        # the top-k entry point has no fused append
         Lyr = w.layers
         launches = [0]
-        self.step(p, launches=launches)        # eager (kernel attributes set outside capture)
+        self.step(p, launches=launches, topk=topk)   # eager (attributes set outside capture)
         per_step_launches = launches[0]
-        unions, conc, diff, allc = self.selections(p)
+        unions, conc, diff, allc = self.selections(p, topk)
         step_bytes = algorithmic_bytes(w, unions, include_append=True)
         dec_bytes = algorithmic_bytes(w, unions, include_append=False)
         side = torch.cuda.Stream(device=dev)
         side.wait_stream(torch.cuda.current_stream())
         with torch.cuda.stream(side):
-            self.step(p)
+            self.step(p, topk=topk)
             g_full = torch.cuda.CUDAGraph()
             with torch.cuda.graph(g_full, stream=side):
-                self.step(p)
+                self.step(p, topk=topk)
             g_dec = torch.cuda.CUDAGraph()                  # the decode kernel alone
             with torch.cuda.graph(g_dec, stream=side):
-                self.step(p, with_append=fused)
+                self.step(p, with_append=fused, topk=topk)
         torch.cuda.current_stream().wait_stream(side)
         torch.cuda.synchronize()
 
@@ -507,7 +555,7 @@ class GpuWorkload:
                            for g in range(w.Hkv) if w.ret_mask[l, g]))
         res.update({
             "value": aggregate(Lyr, 1, world, ms_step), "unit": "layer-steps/s",
-            "ms_per_step": ms_step, "p": p,
+            "ms_per_step": ms_step, "p": None if topk else p, "topk": topk or None,
             "config": workload_config(w, "inputs larger than L2 (%.2f GB read per step vs "
                                          "126 MB L2)" % (step_bytes / 1e9)),
             "achieved_step_gbs": step_bytes / (ms_step * 1e-3) / 1e9,
@@ -596,6 +644,8 @@ def run_ours(args, w):
             me = gw.measure(p, args, world)
             key = we.name if len(ps) == 1 else f"{we.name}@p={p}"
             extra[key] = me
+        if wi == 2 and args.topk > 0:          # the fixed-budget top-k variant at 32K
+            extra[f"{we.name}@topk={args.topk}"] = gw.measure(we.p, args, world, topk=args.topk)
         gw.close()
         del gw
     if extra:
@@ -603,15 +653,20 @@ def run_ours(args, w):
     if rank == 0 and world == 1 and not args.no_cpu:
         line["cpu_baseline"] = _cpu_baseline(w, args.cpu_budget)
         for key, me in extra.items():
-            if me["config"]["workload"] == "qwen3-8b-32k-b1":   # one whole 36-layer step
-                we = workloads.workload(2)
-                if args.layers:
-                    we.layers = min(we.layers, args.layers)
-                n, spent = oracle_full_step(we)
-                me["cpu_baseline"] = {"value": n / spent, "unit": "layer-steps/s",
-                                      "cores": cpu_threads(), "kind": "oracle",
-                                      "sample": f"one whole step of {we.name}: all {n} layers, "
-                                                f"every head, {spent:.1f} s of float64 NumPy"}
+            if me["config"]["workload"] != "qwen3-8b-32k-b1":
+                continue
+            we = workloads.workload(2)
+            if args.layers:
+                we.layers = min(we.layers, args.layers)
+            if me.get("topk"):                  # the budget-vs-mass comparison of the pages
+                me["retained_full_attention_mass"] = oracle_retained_mass(we, k=me["topk"])
+                continue
+            me["retained_full_attention_mass"] = oracle_retained_mass(we, p=me["p"])
+            n, spent = oracle_full_step(we)      # one whole 36-layer step
+            me["cpu_baseline"] = {"value": n / spent, "unit": "layer-steps/s",
+                                  "cores": cpu_threads(), "kind": "oracle",
+                                  "sample": f"one whole step of {we.name}: all {n} layers, "
+                                            f"every head, {spent:.1f} s of float64 NumPy"}
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:
@@ -627,6 +682,9 @@ def main(argv=None):
     ap.add_argument("--workload", type=int, default=4)
     ap.add_argument("--extra", default="2,3,5",
                     help="workloads measured in the same run and reported under 'extra'")
+    ap.add_argument("--topk", type=int, default=2048,
+                    help="k of the fixed-budget top-k variant measured on the 32K workload "
+                         "(0: skip)")
     ap.add_argument("--p", type=float, default=None)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--cpu-budget", type=float, default=12.0)

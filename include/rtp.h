@@ -143,8 +143,8 @@ int rtp_decode_step(const rtp_layer_desc* desc, const rtp_cache* cache, const ui
  * rtp_append_kv writes it, and the outputs equal those of the two calls in sequence.
  *   k_new, v_new: bf16 [B][Hkv][128], the decode token's pre-RoPE key and value.
  *   w_kidx      : fp32 [Hkv][128][16] (may be NULL when the layer has no retrieval head).
- * Other arguments as rtp_decode_step. Inside the launch, the CTA that scores a retrieval
- * group's last chunk, and the local item whose ring slice holds the new row, write the token
+ * Other arguments as rtp_decode_step. Inside the launch, the CTA whose chunk holds the new
+ * row of a retrieval group, and the local item whose ring slice holds it, write the token
  * before reading those rows; every other reader comes after a device-wide arrival. The pages
  * describe the two steps separately; one launch saves the second launch of every layer.
  * Errors as rtp_decode_step; RTP_EINVAL when k_new or v_new is NULL, or w_kidx is NULL in a
@@ -155,6 +155,19 @@ int rtp_decode_step_append(const rtp_layer_desc* desc, const rtp_cache* cache,
                            const uint16_t* q_pre, const float* w_qidx, const int32_t* seq_lens,
                            double p, uint16_t* out, int32_t* sel_counts, int32_t* sel_idx,
                            int64_t sel_stride, void* ws, size_t ws_bytes, rtp_stream_t stream);
+
+/*
+ * Decode step with a fixed-budget top-k selector in place of top-p (the budget the paper's
+ * Table 1 compares top-p against; the same 256-bin histogram, with a count threshold):
+ * b* = highest bin whose token count from the top reaches k; S = tokens with bin >= b*, so S
+ * holds the k highest scores plus, at most, other tokens of bin b*. All tokens are kept when
+ * k >= N or hi == lo. Local heads as in rtp_decode_step.
+ *   k: >= 1 (RTP_EINVAL otherwise). Other arguments and errors as rtp_decode_step.
+ */
+int rtp_decode_step_topk(const rtp_layer_desc* desc, const rtp_cache* cache,
+                         const uint16_t* q_pre, const float* w_qidx, const int32_t* seq_lens,
+                         int64_t k, uint16_t* out, int32_t* sel_counts, int32_t* sel_idx,
+                         int64_t sel_stride, void* ws, size_t ws_bytes, rtp_stream_t stream);
 
 /* Size of the library-owned scratch of rtp_decode_step_static (bytes). */
 #define RTP_STATIC_SCRATCH_BYTES (16u << 20)

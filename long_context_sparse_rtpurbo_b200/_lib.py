@@ -14,7 +14,7 @@ RTP_OK, RTP_EINVAL, RTP_ESHAPE, RTP_EWORKSPACE, RTP_ECUDA, RTP_ETIMEOUT, RTP_EDE
 EXPORTS = (
     "rtp_status_str", "rtp_build_slot_map", "rtp_workspace_bytes", "rtp_workspace_init",
     "rtp_append_kv", "rtp_decode_step", "rtp_read_device_status", "rtp_last_launch_count",
-    "rtp_decode_step_static", "rtp_decode_step_append", "rtp_debug_set_wait_limit",
+    "rtp_decode_step_static", "rtp_decode_step_append", "rtp_decode_step_topk", "rtp_debug_set_wait_limit",
     "rtp_debug_fail_next_call",
 )
 RTP_STATIC_SCRATCH_BYTES = 16 << 20
@@ -68,6 +68,8 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.rtp_decode_step_append.restype = ctypes.c_int
     lib.rtp_decode_step_append.argtypes = [D, C, vp, vp, vp, vp, vp, vp, ctypes.c_double, vp, vp,
                                            vp, i64, vp, sz, vp]
+    lib.rtp_decode_step_topk.restype = ctypes.c_int
+    lib.rtp_decode_step_topk.argtypes = [D, C, vp, vp, vp, i64, vp, vp, vp, i64, vp, sz, vp]
     lib.rtp_decode_step_static.restype = ctypes.c_int
     lib.rtp_decode_step_static.argtypes = [D, C, vp, vp, vp, ctypes.c_double, vp, vp, vp]
     lib.rtp_read_device_status.restype = ctypes.c_int

@@ -9,6 +9,7 @@
 #include <mutex>
 
 #include "../../include/rtp.h"
+#include "rtp_attr_cache.h"
 #include "rtp_decode.cuh"
 
 using namespace rtp;
@@ -209,27 +210,18 @@ int smem_layout(DecodeParams& P, const Plan& pl, int smem_optin) {
 }
 
 // The shared-memory opt-in of decode_kernel<G> is a per-device function attribute: set it
-// once per (device, instance), under a lock.
-std::mutex g_attr_mu;
-int g_attr_smem[4][64];
-bool g_attr_init = false;
+// once per (device, instance) (rtp_attr_cache.h).
+AttrCache<4, 64> g_attr;
 
 template <int G>
 int ensure_smem_attr(int dev, int smem) {
   constexpr int gi = G == 1 ? 0 : (G == 2 ? 1 : (G == 4 ? 2 : 3));
-  if (dev < 0 || dev >= 64) return RTP_ECUDA;
-  std::lock_guard<std::mutex> lock(g_attr_mu);
-  if (!g_attr_init) {
-    for (auto& row : g_attr_smem) for (int& v : row) v = -1;
-    g_attr_init = true;
-  }
-  if (g_attr_smem[gi][dev] < smem) {
-    if (cudaFuncSetAttribute(decode_kernel<G>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             smem) != cudaSuccess)
-      return RTP_ECUDA;
-    g_attr_smem[gi][dev] = smem;
-  }
-  return RTP_OK;
+  const int rc = g_attr.ensure(gi, dev, smem, [](int, int bytes) {
+    // the current device is `dev` (the caller's cudaGetDevice)
+    return cudaFuncSetAttribute(decode_kernel<G>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                bytes) == cudaSuccess ? 0 : 1;
+  });
+  return rc == 0 ? RTP_OK : RTP_ECUDA;
 }
 
 template <int G>
@@ -269,7 +261,7 @@ int decode_impl(const rtp_layer_desc* desc, const rtp_cache* cache, const uint16
                 const float* w_qidx, const int32_t* seq_lens, double p, uint16_t* out,
                 int32_t* sel_counts, int32_t* sel_idx, int64_t sel_stride, void* ws,
                 size_t ws_bytes, rtp_stream_t stream, const uint16_t* k_new,
-                const uint16_t* v_new, const float* w_kidx);
+                const uint16_t* v_new, const float* w_kidx, int64_t topk = 0);
 
 }  // namespace
 
@@ -357,6 +349,19 @@ int rtp_decode_step_append(const rtp_layer_desc* desc, const rtp_cache* cache,
                      sel_stride, ws, ws_bytes, stream, k_new, v_new, w_kidx);
 }
 
+int rtp_decode_step_topk(const rtp_layer_desc* desc, const rtp_cache* cache,
+                         const uint16_t* q_pre, const float* w_qidx, const int32_t* seq_lens,
+                         int64_t k, uint16_t* out, int32_t* sel_counts, int32_t* sel_idx,
+                         int64_t sel_stride, void* ws, size_t ws_bytes, rtp_stream_t stream) {
+  if (k < 1) {
+    g_launches = 0;
+    if (const int inj = take_injected()) return inj;
+    return RTP_EINVAL;
+  }
+  return decode_impl(desc, cache, q_pre, w_qidx, seq_lens, 0.5, out, sel_counts, sel_idx,
+                     sel_stride, ws, ws_bytes, stream, nullptr, nullptr, nullptr, k);
+}
+
 }  // extern "C"
 
 namespace {
@@ -365,7 +370,7 @@ int decode_impl(const rtp_layer_desc* desc, const rtp_cache* cache, const uint16
                 const float* w_qidx, const int32_t* seq_lens, double p, uint16_t* out,
                 int32_t* sel_counts, int32_t* sel_idx, int64_t sel_stride, void* ws,
                 size_t ws_bytes, rtp_stream_t stream, const uint16_t* k_new,
-                const uint16_t* v_new, const float* w_kidx) {
+                const uint16_t* v_new, const float* w_kidx, int64_t topk) {
   g_launches = 0;
   if (const int inj = take_injected()) return inj;
   Plan pl;
@@ -392,8 +397,9 @@ int decode_impl(const rtp_layer_desc* desc, const rtp_cache* cache, const uint16
   P.n_groups = pl.n_groups; P.n_lgroups = pl.n_lgroups;
   local_split(L, pl.n_lgroups, L.n_ret, std::min(di.sms, kPlanCTAs), P.PL, P.RL);
   P.n_loc_items = pl.n_lgroups * P.PL;          // <= pl.n_loc_items (RL >= 64)
-  P.select_all = p >= 1.0 ? 1 : 0;
+  P.select_all = (topk == 0 && p >= 1.0) ? 1 : 0;
   P.p = p;
+  P.topk = topk;
   P.spin_limit = g_spin_limit.load();
   P.cand_stride = pl.cand_stride;
   P.q_pre = q_pre; P.w_qidx = w_qidx; P.seq_lens = seq_lens;

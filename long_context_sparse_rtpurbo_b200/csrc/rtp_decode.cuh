@@ -78,8 +78,9 @@ struct DecodeParams {
   int PL;            // local items per local group
   int RL;            // ring rows per local item
   int n_loc_items;
-  int select_all;    // p >= 1
+  int select_all;    // p >= 1 (top-p mode)
   double p;
+  long long topk;    // > 0: fixed-budget top-k (count threshold) instead of top-p
   long long spin_limit;
   int64_t cand_stride;   // list entries per group (>= max_seq_len)
   // shared-memory layout (byte offsets into the dynamic buffer)
@@ -507,11 +508,13 @@ struct DecodeCta {
 #pragma unroll
       for (int u = 0; u < 2; ++u) {
         const int p = lane + 32 * u, r = p >> 1, hh = p & 1;
-        if (rb + r < N)
+        if (rb + r < N) {
           cp_async16_s(slot + idx_half_off(r, hh), src + (int64_t)(rb + r) * 32 + hh * 16);
-        else      // zero rows: a stale inf or NaN times a zero query column would poison the
+        }
+        else {    // zero rows: a stale inf or NaN times a zero query column would poison the
                   // other half-tile's scores
           st_shared_zero16(slot + idx_half_off(r, hh));
+        }
       }
     }
     cp_async_commit();
@@ -620,12 +623,14 @@ struct DecodeCta {
     float thr[2];                  // per slot: cutoff edge (+inf for a padding column)
     int hd[2];
     int N, qn, qoff, hp_off, hist_off;
+    bool count_only;               // top-k: each score adds 1 (counts, not masses)
     __device__ __forceinline__ void add(float y, int h) const {
       const float4 p = smem_at<float4>(hp_off)[h];           // lo, inv, hi
       const int b = p.y > 0.f ? bin_of(y, p.x, p.y) : 0;
       const float ex = y - p.z;
-      if (ex > -42.f) {                     // below 2^-41 the fixed-point mass rounds to 0
-        const unsigned long long q = __float2ull_rn(exp2f(ex) * kMassScale);
+      if (count_only || ex > -42.f) {       // below 2^-41 the fixed-point mass rounds to 0
+        const unsigned long long q =
+            count_only ? 1ull : __float2ull_rn(exp2f(ex) * kMassScale);
         uint32_t* hlo = smem_at<uint32_t>(hist_off);
         uint32_t* hhi = hlo + G * kHistStride;
         const int bi = h * kHistStride + b;
@@ -905,9 +910,10 @@ struct DecodeCta {
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) T += __shfl_xor_sync(0xffffffffu, T, o);
       const float inv = (hi > lo && !P.select_all) ? (float)kBins / (hi - lo) : 0.f;
-      // cutoff bin, its score edge; per-head parameters of the binning
+      // cutoff bin, its score edge; per-head parameters of the binning (top-k counts every
+      // token: no cutoff)
       int bch = 0;
-      if (P.p < 1.0 && inv > 0.f) {
+      if (P.topk == 0 && P.p < 1.0 && inv > 0.f) {
         const float arg = (float)((1.0 - P.p) * T * (1.0 - 1e-3) / (double)N);
         const float c = hi + log2f(arg);
         bch = c > lo ? bin_of(c, lo, inv) : 0;
@@ -942,6 +948,7 @@ struct DecodeCta {
     hc.qoff = tail(kTailHq) + warp * kHQueueMax * 8;
     hc.hp_off = P.sm_int + kIntHp * 4;
     hc.hist_off = P.sm_hist;
+    hc.count_only = P.topk > 0;
     if (tcol >= 0) {
       ScoreTile<G> T;                      // lane layout only (no query needed)
       T.init(sm.qidx());
@@ -993,7 +1000,8 @@ struct DecodeCta {
     T.init(sm.qidx());                     // lane layout; its query part is not used here
     if (!wait_for(P.bar + (int64_t)g * 4 + 1, (uint32_t)S)) { abort_ = true; return; }
     trace(kEvW0);
-    // b* per head (warp h: head h): the highest bin whose mass from the top reaches p T
+    // b* per head (warp h: head h): the highest bin whose mass from the top reaches p T (top-k:
+    // whose count from the top reaches k)
     if (warp < G) {
       int best = 0;
       if (!P.select_all) {
@@ -1008,7 +1016,8 @@ struct DecodeCta {
           const unsigned long long y = __shfl_down_sync(0xffffffffu, x, o);
           if (lane + o < 32) x += y;
         }
-        const double thr = P.p * sm.tcache()[step * G + warp] * (double)kMassScale;
+        const double thr = P.topk > 0 ? (double)P.topk
+                                      : P.p * sm.tcache()[step * G + warp] * (double)kMassScale;
         best = -1;
         unsigned long long cum = x - lt;
 #pragma unroll

@@ -50,6 +50,13 @@ class DecodeLayer:
         return rtp.rtp_decode_step(self.desc, self.cache, q_pre, w_qidx, seq_lens, p, out,
                                    sel_counts, sel_idx, stride, self.ws, self.ws_bytes, stream)
 
+    def decode_topk(self, q_pre, w_qidx, seq_lens, k, out, sel_counts, sel_idx=None, stream=None):
+        """Decode step with the fixed-budget top-k selector."""
+        stride = 0 if sel_idx is None else sel_idx.shape[-1]
+        return rtp.rtp_decode_step_topk(self.desc, self.cache, q_pre, w_qidx, seq_lens, k, out,
+                                        sel_counts, sel_idx, stride, self.ws, self.ws_bytes,
+                                        stream)
+
     def decode_append(self, k_new, v_new, w_kidx, q_pre, w_qidx, seq_lens, p, out, sel_counts,
                       sel_idx=None, stream=None):
         """Append of the decode token (k_new, v_new: bf16 [B][Hkv][128] at seq_lens - 1) and

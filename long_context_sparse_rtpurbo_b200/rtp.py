@@ -117,6 +117,18 @@ def rtp_decode_step_append(desc: LayerDesc, cache: RtpCache, k_new, v_new, w_kid
         int(sel_stride), _ptr(ws), int(ws_bytes), _stream(stream)))
 
 
+def rtp_decode_step_topk(desc: LayerDesc, cache: RtpCache, q_pre, w_qidx, seq_lens, k, out,
+                         sel_counts, sel_idx=None, sel_stride=0, ws=None, ws_bytes=None,
+                         stream=None):
+    """Decode step with the fixed-budget top-k selector (see include/rtp.h)."""
+    if ws_bytes is None:
+        ws_bytes = 0 if ws is None else ws.numel() * ws.element_size()
+    return _check("rtp_decode_step_topk", _lib.load().rtp_decode_step_topk(
+        desc.ref, ctypes.byref(cache), _ptr(q_pre), _ptr(w_qidx), _ptr(seq_lens), int(k),
+        _ptr(out), _ptr(sel_counts), _ptr(sel_idx), int(sel_stride), _ptr(ws), int(ws_bytes),
+        _stream(stream)))
+
+
 def rtp_decode_step_static(desc: LayerDesc, cache: RtpCache, q_pre, w_qidx, seq_lens, p, out,
                            sel_counts, stream=None):
     """rtp_decode_step on the library's own fixed scratch (no workspace argument): for callers

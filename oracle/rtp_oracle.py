@@ -185,6 +185,48 @@ def topp_exact(s, p: float) -> np.ndarray:
     return mask
 
 
+# --------------------------------------------------------------------------- fixed top-k variant
+def topk_histogram(s, k: int) -> Selection:
+    """Fixed-budget top-k through the same 256-bin histogram, with a count threshold in place
+    of the mass threshold: the top-k selector the pages compare Top-P against ([P] Table 1,
+    top-k budgets vs top-p; [DR] "Method": the 256-bin threshold).
+
+    count_b = number of tokens in bin b; K_b = sum_{b' >= b} count_b'; b* = max{b : K_b >= k};
+    S = {n : bin(s_n) >= b*}. k >= N, or all-equal scores, selects every token. The fields M
+    and C of the result hold the counts and their suffix sums; T = N.
+
+    b* is the bin of the k-th highest score: the k highest scores all have bins >= it, and if
+    k tokens had bins above it the k-th highest score would too. So S holds the exact top-k
+    plus, at most, tokens of that one bin.
+    """
+    s = np.asarray(s, np.float64)
+    N = s.shape[0]
+    if N < 1:
+        raise ValueError("top-k needs at least one token")
+    if k < 1:
+        raise ValueError("top-k needs k >= 1")
+    lo, hi = float(s.min()), float(s.max())
+    if k >= N or hi == lo:
+        cnt = np.zeros(N_BINS)
+        cnt[0] = N
+        return Selection(np.ones(N, bool), 0, lo, hi, np.zeros(N, np.int64), cnt, cnt.copy(),
+                         float(N), True)
+    bins = score_bins(s, lo, hi)
+    cnt = np.bincount(bins, minlength=N_BINS).astype(np.float64)
+    C = np.cumsum(cnt[::-1])[::-1]
+    bstar = int(np.nonzero(C >= k)[0].max())
+    return Selection(bins >= bstar, bstar, lo, hi, bins, cnt, C, float(N), False)
+
+
+def topk_exact(s, k: int) -> np.ndarray:
+    """The k highest scores (equal scores by lower index first), by sort. Returns a bool mask."""
+    s = np.asarray(s, np.float64)
+    order = np.lexsort((np.arange(s.shape[0]), -s))
+    mask = np.zeros(s.shape[0], bool)
+    mask[order[:min(int(k), s.shape[0])]] = True
+    return mask
+
+
 # --------------------------------------------------------------------------- eq. (5): attention
 def attend(q, K, V, scale: float | None = None) -> np.ndarray:
     """sum_n softmax_n(q^T k_n / sqrt(d)) v_n over the rows given ([P] §3.2 eq. (5); R9)."""

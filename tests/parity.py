@@ -75,14 +75,17 @@ def make_layer(w, layer, device="cuda", seq_lens=None, caps=None):
                        caps, device, w.rope_base)
 
 
-def decode(lay: DecodeLayer, q, wq, seq_lens, p, device="cuda", with_sel=True):
+def decode(lay: DecodeLayer, q, wq, seq_lens, p, device="cuda", with_sel=True, k=None):
     B, Hq = lay.B, lay.Hq
     out = torch.zeros((B, Hq, 128), dtype=torch.bfloat16, device=device)
     cnt = torch.zeros((B, Hq), dtype=torch.int32, device=device)
     stride = int(lay.desc.c.max_seq_len)
     sel = torch.full((B, Hq, stride), -1, dtype=torch.int32, device=device) if with_sel else None
     sl = torch.as_tensor(np.asarray(seq_lens, np.int32), device=device)
-    lay.decode(q, wq, sl, p, out, cnt, sel)
+    if k is not None:
+        lay.decode_topk(q, wq, sl, k, out, cnt, sel)
+    else:
+        lay.decode(q, wq, sl, p, out, cnt, sel)
     torch.cuda.synchronize()
     return out, cnt, sel
 
@@ -103,25 +106,41 @@ def check_selection(s, p, gpu_set: np.ndarray) -> dict:
                 mass=float(mass), ok=bool(ok_mass and near.all()), bstar=sel.bstar)
 
 
+def check_selection_topk(s, k, gpu_set: np.ndarray) -> dict:
+    """Selection rule check for one retrieval head under the fixed-budget top-k selector:
+    the same one-bin-width rule, and at least min(k, N) tokens."""
+    sel = O.topk_histogram(s, k)
+    ref = np.nonzero(sel.mask)[0]
+    diff = np.setxor1d(ref, gpu_set)
+    if sel.select_all:
+        near = np.zeros(len(diff), bool)
+    else:
+        near = np.abs(s[diff] - sel.edge()) <= sel.width
+    ok_count = len(gpu_set) >= min(int(k), len(s))
+    return dict(n_ref=len(ref), n_gpu=len(gpu_set), n_diff=len(diff), n_far=int((~near).sum()),
+                ok=bool(ok_count and near.all()), bstar=sel.bstar)
+
+
 def run_layer_parity(workload_index=1, layer=0, p=None, check_sets=True, heads=None,
-                     source="numpy", device="cuda", w=None, seq_lens=None) -> dict:
-    """Builds one layer, appends all tokens, decodes once and compares with the oracle.
-    Returns a report; raises AssertionError on a parity failure."""
+                     source="numpy", device="cuda", w=None, seq_lens=None, k=None) -> dict:
+    """Builds one layer, appends all tokens, decodes once (top-p, or top-k when k is given)
+    and compares with the oracle. Returns a report; raises AssertionError on a parity
+    failure."""
     w = w if w is not None else workloads.workload(workload_index)
     p = w.p if p is None else p
     seq_lens = np.asarray(w.seq_lens if seq_lens is None else seq_lens, np.int64)
     q, wq, wk = layer_inputs(w, layer, device)
     lay = make_layer(w, layer, device, seq_lens)
     fill_layer(w, layer, lay, wk, seq_lens, source=source, device=device)
-    out, cnt, sel = decode(lay, q, wq, seq_lens, p, device, with_sel=check_sets)
+    out, cnt, sel = decode(lay, q, wq, seq_lens, p, device, with_sel=check_sets, k=k)
     st = lay.status()
     assert st == 0, f"device status {st}"
-    report = check_outputs(w, layer, seq_lens, p, out, cnt, sel, heads)
+    report = check_outputs(w, layer, seq_lens, p, out, cnt, sel, heads, k=k)
     report["layer"] = lay
     return report
 
 
-def check_outputs(w, layer, seq_lens, p, out, cnt, sel=None, heads=None) -> dict:
+def check_outputs(w, layer, seq_lens, p, out, cnt, sel=None, heads=None, k=None) -> dict:
     """Compares one decode's outputs (device tensors) with the oracle under the rules above,
     for the (b, h) pairs in ``heads`` (every head when None). Raises AssertionError."""
     seq_lens = np.asarray(seq_lens, np.int64)
@@ -150,8 +169,9 @@ def check_outputs(w, layer, seq_lens, p, out, cnt, sel=None, heads=None) -> dict
                 assert np.all(np.diff(gset) > 0), "sel_idx not ascending"
                 assert gset.size == 0 or (gset[0] >= 0 and gset[-1] < N)
             else:
-                gset = np.nonzero(O.topp_histogram(s, p).mask)[0]
-            chk = check_selection(s, p, gset)
+                gset = np.nonzero((O.topp_histogram(s, p) if k is None
+                                   else O.topk_histogram(s, k)).mask)[0]
+            chk = check_selection(s, p, gset) if k is None else check_selection_topk(s, k, gset)
             entry.update(chk)
             assert chk["ok"], f"selection parity failed at (b={b}, h={h}): {chk}"
             assert cnt[b, h] == len(gset)

@@ -143,6 +143,29 @@ def test_two_wave_schedule(G, N):
     assert all(e["retrieval"] and e["count"] > 0 for e in rep["heads"])
 
 
+@pytest.mark.parametrize("k", [1, 64, 2048, 4096, 5000])
+def test_topk_tiny_layer_parity(k):
+    """The fixed-budget top-k selector (count threshold on the same histogram), N = 4096:
+    k = 1, small, mid, k = N and k > N (every token)."""
+    rep = _parity().run_layer_parity(workload_index=1, layer=0, k=k)
+    for e in rep["heads"]:
+        if e["retrieval"]:
+            assert e["count"] >= min(k, 4096)
+
+
+@pytest.mark.parametrize("G", [1, 8])
+def test_topk_group_sizes(G):
+    _parity().run_layer_parity(w=_small(G=G, seq=(3000,)), layer=0, k=300)
+
+
+def test_topk_qwen_layer_32k():
+    """A full Qwen3-8B-shaped layer at N = 32768 with k = 2048 (every head)."""
+    w = workloads.workload(2)
+    layer = int(np.nonzero(w.ret_mask.sum(1) >= 2)[0][0])
+    rep = _parity().run_layer_parity(w=w, layer=layer, source="gpu", k=2048)
+    assert all(e["count"] >= 2048 for e in rep["heads"] if e["retrieval"])
+
+
 # Full benchmark sizes, in the launch configuration the bench times (one layer of the 36, all
 # caches filled on the GPU); the oracle checks sampled heads one by one.
 def _layer_with(w, n_ret):

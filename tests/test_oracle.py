@@ -233,6 +233,79 @@ def test_topp_special_cases():
         O.topp_histogram(np.array([]), 0.9)
 
 
+def test_topk_hand_worked_example():
+    """Scores {0, 1, 2, 3}: bins 0, 85, 170, 255 (256 / 3 = 85.33); counts from the top 1, 2,
+    3, 4, so k = 1 -> b* = 255 {3}; k = 2 -> 170 {2, 3}; k = 3 -> 85 {1, 2, 3}. Scores
+    {0, 10, 10.01, 10.02}: the three high scores share bin 255 (256 * 10 / 10.02 = 255.49),
+    so k = 2 keeps all three (the extra token sits in the threshold bin)."""
+    s = np.array([0.0, 1.0, 2.0, 3.0])
+    for k, bstar, want in ((1, 255, [3]), (2, 170, [2, 3]), (3, 85, [1, 2, 3])):
+        sel = O.topk_histogram(s, k)
+        assert list(sel.bins) == [0, 85, 170, 255]
+        assert sel.bstar == bstar and list(np.nonzero(sel.mask)[0]) == want
+        assert list(np.nonzero(O.topk_exact(s, k))[0]) == want
+    s = np.array([0.0, 10.0, 10.01, 10.02])
+    sel = O.topk_histogram(s, 2)
+    assert sel.bstar == 255 and list(np.nonzero(sel.mask)[0]) == [1, 2, 3]
+    assert list(np.nonzero(O.topk_exact(s, 2))[0]) == [2, 3]
+
+
+@pytest.mark.parametrize("seed", range(12))
+def test_topk_contains_a_top_k_set_by_enumeration(seed):
+    """Every k-subset whose scores are all >= the scores outside it is a valid top-k; the
+    histogram set contains one of them and its other tokens lie in bin b*."""
+    rng = np.random.default_rng(300 + seed)
+    N = int(rng.integers(2, 11))
+    s = rng.standard_normal(N) * rng.uniform(0.1, 4.0)
+    if seed % 3 == 0:
+        s = np.round(s, 1)                                  # ties
+    k = int(rng.integers(1, N))
+    sel = O.topk_histogram(s, k)
+    valid = [set(c) for c in itertools.combinations(range(N), k)
+             if min(s[list(c)]) >= max(np.delete(s, list(c)), default=-np.inf)]
+    got = set(np.nonzero(sel.mask)[0])
+    assert valid and any(c <= got for c in valid)
+    c = next(c for c in valid if c <= got)
+    assert all(sel.bins[n] == sel.bstar for n in got - c)
+    assert set(np.nonzero(O.topk_exact(s, k))[0]) in valid
+
+
+@pytest.mark.parametrize("seed", range(30))
+def test_topk_histogram_invariants(seed):
+    """|S| >= k; bins above b* hold fewer than k tokens (b* maximal); b* is the bin of the
+    k-th highest score; the sorted top-k is a subset and the extras sit in bin b*."""
+    rng = np.random.default_rng(400 + seed)
+    N = int(rng.integers(2, 5000 if seed % 3 == 0 else 80))
+    s = rng.standard_normal(N) * rng.uniform(0.2, 6.0)
+    if seed % 5 == 1:
+        s[: max(1, N // 20)] += rng.uniform(2, 8)
+    if seed % 7 == 2:
+        s = np.round(s)
+    k = int(rng.integers(1, N + 1))
+    sel = O.topk_histogram(s, k)
+    ex = O.topk_exact(s, k)
+    assert sel.mask.sum() >= k
+    assert np.all(sel.mask[ex])
+    if not sel.select_all:
+        assert (sel.bins > sel.bstar).sum() < k
+        kth = np.sort(s)[::-1][k - 1]
+        assert sel.bstar == O.score_bins(np.array([kth]), sel.lo, sel.hi)[0]
+        assert np.all(sel.bins[sel.mask & ~ex] == sel.bstar)
+
+
+def test_topk_special_cases():
+    rng = np.random.default_rng(9)
+    s = rng.standard_normal(50)
+    assert O.topk_histogram(s, 50).mask.all()              # k = N -> all
+    assert O.topk_histogram(s, 80).mask.all()              # k > N -> all
+    assert O.topk_histogram(np.full(10, 1.5), 3).mask.all()   # all scores equal -> all
+    assert O.topk_histogram(np.array([2.0]), 1).mask.all()     # N = 1
+    with pytest.raises(ValueError):
+        O.topk_histogram(s, 0)
+    with pytest.raises(ValueError):
+        O.topk_histogram(np.array([]), 1)
+
+
 def test_bins_linear_over_min_max():
     s = np.linspace(-3.0, 5.0, 257)                        # exactly on the 256 bin edges
     b = O.score_bins(s, -3.0, 5.0)

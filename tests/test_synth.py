@@ -71,3 +71,33 @@ def test_workload_shapes():
             assert w.ret_mask.sum() == 43 and w.ret_mask.shape == (36, 8)
     w5 = workloads.workload(5)
     assert w5.seq_lens.min() >= 8192 and w5.seq_lens.max() <= 65536 and len(w5.seq_lens) == 64
+
+
+def test_topk_vs_topp_budget_on_the_32k_workload():
+    """The comparison the pages draw between a fixed top-k budget and top-p (oracle only, one
+    32K layer with two retrieval groups, every query head): with k equal to the mean top-p
+    budget, the concentrated heads keep more than p of their mass and at least one diffuse
+    head keeps less; giving every head at least p needs k = the largest top-p set, which
+    spends more tokens in total than top-p does."""
+    from oracle import rtp_oracle as O
+    w = workloads.workload(2)
+    layer = int(np.nonzero(w.ret_mask.sum(1) >= 2)[0][0])
+    N = int(w.seq_lens[0])
+    qb = w.q_pre_bits(layer)
+    rows = []
+    for g in np.nonzero(w.ret_mask[layer])[0]:
+        kp = gen.bf16_bits_to_f32(w.kpre_bits(layer, 0, int(g), 0, N)).astype(np.float64)
+        kidx = O.index_keys(kp, w.w_kidx(layer)[g])
+        for h in range(g * w.G, (g + 1) * w.G):
+            q = gen.bf16_bits_to_f32(qb[0, h]).astype(np.float64)
+            s = O.index_scores(O.index_query(q, w.w_qidx(layer)[h]), kidx)
+            kind = w.group_layout(layer, 0, int(g)).targets[h % w.G][0]
+            rows.append((kind, s, int(O.topp_histogram(s, w.p).mask.sum())))
+    mean_budget = int(round(np.mean([r[2] for r in rows])))
+    mass = lambda s, m: float(np.exp(s - s.max())[m].sum() / np.exp(s - s.max()).sum())
+    conc = [mass(s, O.topk_exact(s, mean_budget)) for kind, s, _ in rows if kind == "conc"]
+    diff = [mass(s, O.topk_exact(s, mean_budget)) for kind, s, _ in rows if kind == "diff"]
+    assert conc and diff
+    assert min(conc) > w.p and min(diff) < w.p
+    k_all = max(r[2] for r in rows)
+    assert len(rows) * k_all > sum(r[2] for r in rows)
