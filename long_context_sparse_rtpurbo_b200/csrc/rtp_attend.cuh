@@ -33,6 +33,18 @@ __device__ __forceinline__ void cp_async16(void* smem, const void* gmem) {
 __device__ __forceinline__ void cp_async16_s(uint32_t saddr, const void* gmem) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(saddr), "l"(gmem) : "memory");
 }
+// L2 policy for data read once per launch (the index rows, gathered K/V rows, local rings):
+// evict first, so the stream does not push the kernel's code and the launch's small shared
+// arrays (histograms, statistics, partials) out of L2.
+__device__ __forceinline__ uint64_t l2_evict_first() {
+  uint64_t pol;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
+  return pol;
+}
+__device__ __forceinline__ void cp_async16_s_ef(uint32_t saddr, const void* gmem, uint64_t pol) {
+  asm volatile("cp.async.cg.shared.global.L2::cache_hint [%0], [%1], 16, %2;"
+               ::"r"(saddr), "l"(gmem), "l"(pol) : "memory");
+}
 __device__ __forceinline__ void st_shared_zero16(uint32_t saddr) {
   asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(saddr), "r"(0u) : "memory");
 }
@@ -137,6 +149,7 @@ __device__ __forceinline__ void tile_copy(unsigned char* tile, const uint16_t* k
   const unsigned long long kq = reinterpret_cast<unsigned long long>(krow);
   const unsigned long long vq = reinterpret_cast<unsigned long long>(vrow);
   const uint32_t okb = __ballot_sync(0xffffffffu, ok);
+  const uint64_t pol = l2_evict_first();
 #pragma unroll
   for (int u = 0; u < 8; ++u) {
     const int r = 2 * u + (lane >> 4);
@@ -145,8 +158,8 @@ __device__ __forceinline__ void tile_copy(unsigned char* tile, const uint16_t* k
     unsigned char* kd = tile + r * 256 + ((c ^ (r & 7)) << 4);
     unsigned char* vd = tile + 4096 + r * 256 + ((c ^ (r & 7)) << 4);
     if ((okb >> (2 * r)) & 1u) {
-      cp_async16(kd, reinterpret_cast<const uint16_t*>(kr) + c * 8);
-      cp_async16(vd, reinterpret_cast<const uint16_t*>(vr) + c * 8);
+      cp_async16_s_ef(smem_u32(kd), reinterpret_cast<const uint16_t*>(kr) + c * 8, pol);
+      cp_async16_s_ef(smem_u32(vd), reinterpret_cast<const uint16_t*>(vr) + c * 8, pol);
     } else {
       *reinterpret_cast<uint4*>(vd) = make_uint4(0, 0, 0, 0);
     }

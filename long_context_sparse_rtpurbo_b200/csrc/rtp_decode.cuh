@@ -500,16 +500,19 @@ struct DecodeCta {
   // scores (rb: group row of the tile's row 0, N when the warp has no tile this stage; rows
   // at or past N score 0 and are masked by the callers).
   __device__ __forceinline__ void slot_issue(uint32_t ring, const unsigned char* src, int st,
-                                             int nst, int N, int nc, int j, int ntl) {
+                                             int nst, int N, int nc, int j, int ntl, bool last) {
     if (st < nst) {
       const int lane = threadIdx.x & 31;
       const int rb = tile_row(N, nc, j, ntl, st, threadIdx.x >> 5);
       const uint32_t slot = ring + (st % kSStages) * kStageBytes;
+      const uint64_t pol = l2_evict_first();
 #pragma unroll
       for (int u = 0; u < 2; ++u) {
         const int p = lane + 32 * u, r = p >> 1, hh = p & 1;
         if (rb + r < N) {
-          cp_async16_s(slot + idx_half_off(r, hh), src + (int64_t)(rb + r) * 32 + hh * 16);
+          const unsigned char* g = src + (int64_t)(rb + r) * 32 + hh * 16;
+          if (last) cp_async16_s_ef(slot + idx_half_off(r, hh), g, pol);
+          else      cp_async16_s(slot + idx_half_off(r, hh), g);
         }
         else {    // zero rows: a stale inf or NaN times a zero query column would poison the
                   // other half-tile's scores
@@ -519,8 +522,10 @@ struct DecodeCta {
     }
     cp_async_commit();
   }
+  // last: this is the launch's last read of these rows (L2 evict-first); chunks whose scores
+  // are recomputed later keep the default policy on their earlier reads
   template <class Fn>
-  __device__ __forceinline__ void stream_chunk(int g, int j, bool patch, Fn& fn) {
+  __device__ __forceinline__ void stream_chunk(int g, int j, bool patch, bool last, Fn& fn) {
     const int b = g / P.L.n_ret, r = g % P.L.n_ret, kvh = P.L.ret_kv[r];
     const int N = gN(g), nc = nch(g);
     const int ntl = chunk_tiles(N, nc, j), nst = chunk_stages(N, nc, j);
@@ -530,7 +535,7 @@ struct DecodeCta {
     const uint32_t ring = smem_u32(sm.stage()) + warp * kSlotBytes;
     __syncthreads();                       // the staging region may still be in use
 #pragma unroll
-    for (int st = 0; st < kSStages - 1; ++st) slot_issue(ring, src, st, nst, N, nc, j, ntl);
+    for (int st = 0; st < kSStages - 1; ++st) slot_issue(ring, src, st, nst, N, nc, j, ntl, last);
     index_query<G>(P, b, kvh, sm.qidx(), reinterpret_cast<float*>(sm.tmp()));
     // The chunk holding the decode token writes it while the first stages are in flight; a
     // copy of its index row may be stale, so the warp holding it patches its slot.
@@ -544,7 +549,7 @@ struct DecodeCta {
     const int prow = patch ? N - 1 : -1;
 #pragma unroll 1
     for (int st = 0; st < nst; ++st) {
-      slot_issue(ring, src, st + kSStages - 1, nst, N, nc, j, ntl);
+      slot_issue(ring, src, st + kSStages - 1, nst, N, nc, j, ntl, last);
       cp_async_wait<kSStages - 1>();
       __syncwarp();
       const uint32_t slot = ring + (st % kSStages) * kStageBytes;
@@ -786,7 +791,7 @@ struct DecodeCta {
     const bool patch = P.k_new && ((N - 1) / kWRows) % nch(g) == j;   // holds row N - 1
     SStats sst(tcol >= 0 ? chunk_taddr(tcol) : 0u, tcol >= 0, N);
     trace(kEvS0);
-    stream_chunk(g, j, patch, sst);
+    stream_chunk(g, j, patch, tcol >= 0, sst);
     if (tcol >= 0) tmem_wait_st();
     trace(kEvS1);
     // chunk statistics per head: lanes of one tig hold the same heads (reduce over gid),
@@ -962,7 +967,7 @@ struct DecodeCta {
         hc(st, tile_row(N, nc, j, ntl, st, warp), c, T);
       }
     } else {
-      stream_chunk(g, j, false, hc);
+      stream_chunk(g, j, false, false, hc);
     }
     hc.finish();
     __syncthreads();
@@ -1086,7 +1091,7 @@ struct DecodeCta {
       wsel.rm_off = rm_off;
       wsel.nw = 0;
       wsel.gl = gl;
-      stream_chunk(g, j, false, wsel);
+      stream_chunk(g, j, false, true, wsel);
       hc[0] = wsel.hc[0]; hc[1] = wsel.hc[1];
       __threadfence_block();
       const int total = list_prefix(wsel.nw);
