@@ -204,33 +204,50 @@ def oracle_full_step(w):
     return w.layers, spent
 
 
+class OracleGroupSample:
+    """Bounded oracle sample for long contexts: the G query heads of one retrieval KV head and
+    of one local KV head of sequence 0 (inputs generated once, untimed); a step is scaled from
+    their times by the workload's mix of retrieval and local (sequence, KV head) pairs over
+    all layers."""
+
+    def __init__(self, w):
+        self.w = w
+        self.l = next(i for i in range(w.layers) if w.ret_mask[i].any() and not w.ret_mask[i].all())
+        self.g_r = int(np.nonzero(w.ret_mask[self.l])[0][0])
+        self.g_l = int(np.nonzero(~w.ret_mask[self.l])[0][0])
+        self.inputs = {g: _layer_inputs_f64(w, self.l, [(0, g)]) for g in (self.g_r, self.g_l)}
+        self.n_ret = int(w.ret_mask.sum()) * w.B
+        self.n_loc = int((~w.ret_mask).sum()) * w.B
+
+    def time_groups(self):
+        from oracle import rtp_oracle as O
+        w, t = self.w, {}
+        for g, (q, kp, vv) in self.inputs.items():
+            heads = [(0, g * w.G + i) for i in range(w.G)]
+            t0 = time.perf_counter()
+            O.decode_layer(q, w.w_qidx(self.l), w.w_kidx(self.l), lambda b, gg: kp[(b, gg)],
+                           lambda b, gg: vv[(b, gg)], w.ret_mask[self.l], w.seq_lens, w.p,
+                           w.sinks, w.window, w.rope_base, heads=heads)
+            t[g] = time.perf_counter() - t0
+        return t
+
+    def step_seconds(self, t):
+        """Seconds of one whole step (all layers) scaled from the two group times."""
+        return self.n_ret * t[self.g_r] + self.n_loc * t[self.g_l]
+
+    def describe(self, t):
+        w = self.w
+        return (f"{w.name}: the {w.G} query heads of retrieval KV head {self.g_r} and of local KV "
+                f"head {self.g_l} of layer {self.l}, sequence 0 ({t[self.g_r]:.2f} s, "
+                f"{t[self.g_l]:.3f} s of float64 NumPy); a {w.layers}-layer step scaled as "
+                f"{self.n_ret} retrieval + {self.n_loc} local (sequence, KV head) pairs")
+
+
 def oracle_group_sample(w):
-    """Bounded oracle sample for long contexts: the G query heads of one retrieval KV head
-    and of one local KV head of sequence 0, each timed once; a step is scaled from them by
-    the workload's mix of retrieval and local (sequence, KV head) pairs over all layers.
-    Returns (layer-steps/s, seconds spent, description)."""
-    from oracle import rtp_oracle as O
-    l = next(i for i in range(w.layers) if w.ret_mask[i].any() and not w.ret_mask[i].all())
-    g_r = int(np.nonzero(w.ret_mask[l])[0][0])
-    g_l = int(np.nonzero(~w.ret_mask[l])[0][0])
-    t = {}
-    for g in (g_r, g_l):
-        q, kp, vv = _layer_inputs_f64(w, l, [(0, g)])
-        heads = [(0, g * w.G + i) for i in range(w.G)]
-        t0 = time.perf_counter()
-        O.decode_layer(q, w.w_qidx(l), w.w_kidx(l), lambda b, gg: kp[(b, gg)],
-                       lambda b, gg: vv[(b, gg)], w.ret_mask[l], w.seq_lens, w.p, w.sinks,
-                       w.window, w.rope_base, heads=heads)
-        t[g] = time.perf_counter() - t0
-        del q, kp, vv
-    n_ret = int(w.ret_mask.sum()) * w.B
-    n_loc = int((~w.ret_mask).sum()) * w.B
-    step_s = n_ret * t[g_r] + n_loc * t[g_l]
-    desc = (f"{w.name}: the {w.G} query heads of retrieval KV head {g_r} and of local KV head "
-            f"{g_l} of layer {l}, sequence 0, timed once each ({t[g_r]:.2f} s, {t[g_l]:.3f} s of "
-            f"float64 NumPy); a {w.layers}-layer step scaled as {n_ret} retrieval + {n_loc} local "
-            f"(sequence, KV head) pairs")
-    return w.layers / step_s, t[g_r] + t[g_l], desc
+    """One timing of OracleGroupSample. Returns (layer-steps/s, seconds spent, description)."""
+    smp = OracleGroupSample(w)
+    t = smp.time_groups()
+    return w.layers / smp.step_seconds(t), sum(t.values()), smp.describe(t)
 
 
 def oracle_retained_mass(w, p=None, k=None):
@@ -291,16 +308,27 @@ def run_reference(args, w):
     rank, world, _ = dist_env()
     if rank != 0:
         return
-    prepared = prepare_oracle_layers(w, sample_layers(w))
     steps_s = []
-    for i in range(args.warmup + args.steps):
-        n, s = oracle_layer_steps(w, prepared[i % len(prepared):] + prepared[:i % len(prepared)],
-                                  0.0, max_steps=1)
-        if i >= args.warmup:
-            steps_s.append(s / n)
+    if int(w.seq_lens.max()) > 65536:
+        # long contexts: per step, the scaled per-head-group sample (a whole layer-step at 1M
+        # is minutes of float64 work and tens of GB of float64 inputs)
+        smp = OracleGroupSample(w)
+        for i in range(args.warmup + args.steps):
+            t = smp.time_groups()
+            if i >= args.warmup:
+                steps_s.append(smp.step_seconds(t) / w.layers)
+        sample = "per step, " + smp.describe(t)
+    else:
+        prepared = prepare_oracle_layers(w, sample_layers(w))
+        for i in range(args.warmup + args.steps):
+            n, s = oracle_layer_steps(w, prepared[i % len(prepared):] + prepared[:i % len(prepared)],
+                                      0.0, max_steps=1)
+            if i >= args.warmup:
+                steps_s.append(s / n)
+        sample = (f"one whole layer-step (all heads, all sequences) of {w.name} per step, "
+                  f"alternating layers {[p[0] for p in prepared]} (one with retrieval heads, one "
+                  f"without)")
     v = 1.0 / float(np.mean(steps_s))
-    sample = (f"one whole layer-step (all heads, all sequences) of {w.name} per step, alternating "
-              f"layers {[p[0] for p in prepared]} (one with retrieval heads, one without)")
     line = {"impl": "reference", "metric": METRIC, "value": v, "unit": "layer-steps/s",
             "n_gpus": 0, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": float(np.mean(steps_s)) * 1e3, "higher_is_better": True,
