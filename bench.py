@@ -355,9 +355,16 @@ def _bits_to_dev(bits, dev):
     return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).to(dev)
 
 
+# The device sources the decode kernel is compiled from: a recorded ncu traffic figure holds
+# while their hash is the one recorded beside it.
+DECODE_KERNEL_SOURCES = ("rtp_common.cuh", "rtp_append.cuh", "rtp_attend.cuh", "rtp_score.cuh",
+                         "rtp_tmem.cuh", "rtp_decode.cuh")
+
+
 def _traffic(kernel: str, workload: str):
     """DRAM bytes per launch of ``kernel`` on ``workload`` from a committed ncu summary, if it
-    was taken on the current source (its sha256 recorded beside it); else None."""
+    was taken on the current kernel source (the sha256 of its device sources recorded beside
+    it); else None."""
     import hashlib
     p = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(p):
@@ -366,7 +373,7 @@ def _traffic(kernel: str, workload: str):
         d = json.load(f)
     src = os.path.join(ROOT, "long_context_sparse_rtpurbo_b200", "csrc")
     h = hashlib.sha256()
-    for name in sorted(os.listdir(src)):
+    for name in DECODE_KERNEL_SOURCES:
         with open(os.path.join(src, name), "rb") as f:
             h.update(f.read())
     e = d.get(f"{kernel}/{workload}")

@@ -601,7 +601,10 @@ struct DecodeCta {
     }
     __device__ __forceinline__ void operator()(int st, int rb, const float (&c)[V],
                                                const ScoreTile<G>& T) {
-      if (keep) Tmem<V>::st(taddr + st * V, c);          // whole warp
+      if (keep) {                          // warp-collective: converged first
+        __syncwarp();
+        Tmem<V>::st(taddr + st * V, c);
+      }
 #pragma unroll
       for (int v = 0; v < V; ++v) {
         const int e = v & 1;
@@ -792,7 +795,10 @@ struct DecodeCta {
     SStats sst(tcol >= 0 ? chunk_taddr(tcol) : 0u, tcol >= 0, N);
     trace(kEvS0);
     stream_chunk(g, j, patch, tcol >= 0, sst);
-    if (tcol >= 0) tmem_wait_st();
+    if (tcol >= 0) {
+      __syncwarp();
+      tmem_wait_st();
+    }
     trace(kEvS1);
     // chunk statistics per head: lanes of one tig hold the same heads (reduce over gid),
     // then a fixed-order pass over (warp, tig, slot)
@@ -962,7 +968,8 @@ struct DecodeCta {
 #pragma unroll 1
       for (int st = 0; st < nst; ++st) {
         float c[V];
-        Tmem<V>::ld(ta + st * V, c);       // whole warp
+        __syncwarp();                      // tcgen05.ld is warp-collective
+        Tmem<V>::ld(ta + st * V, c);
         tmem_wait_ld();
         hc(st, tile_row(N, nc, j, ntl, st, warp), c, T);
       }
@@ -1069,7 +1076,8 @@ struct DecodeCta {
 #pragma unroll 1
         for (int st = s0; st < s1; ++st) {
           float c[V];
-          Tmem<V>::ld(ta + st * V, c);     // whole warp
+          __syncwarp();                    // tcgen05.ld is warp-collective
+          Tmem<V>::ld(ta + st * V, c);
           tmem_wait_ld();
           const int rb = tile_row(N, S, j, ntl, st, warp);
           const uint32_t mask = tile_select(c, rb, N, ts, T, rm_off, hc);
