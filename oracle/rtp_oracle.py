@@ -328,6 +328,34 @@ def decode_layer(q_pre, w_qidx, w_kidx, k_pre, v, ret_mask, seq_lens, p: float, 
     return res
 
 
+# --------------------------------------------------------------------------- prefill (f1)
+def prefill_head(q_pre, k_pre, v, local: bool, sinks: int, window: int,
+                 base: float = 1e6) -> np.ndarray:
+    """Causal prefill of one query head over a prompt of n tokens at positions 0..n-1
+    ([P] §3.2: retrieval heads use dense attention in prefill, local heads attention sinks
+    plus a sliding window in prefill and decode). Query m attends to the positions n <= m
+    (retrieval) or to local_positions(m + 1, sinks, window) (local); keys are stored RoPE'd in
+    bf16 (as the append writes them), q = R(m) q_pre, scale 1 / sqrt(d).
+
+    q_pre, k_pre, v: [n][d] (bf16 values as float64). Returns float64 [n][d].
+    """
+    q_pre = np.asarray(q_pre, np.float64)
+    k_pre = np.asarray(k_pre, np.float64)
+    v = np.asarray(v, np.float64)
+    n, d = q_pre.shape
+    pos = np.arange(n)
+    K = bf16_round(rope_rotate(k_pre, pos, base))
+    Q = rope_rotate(q_pre, pos, base)
+    z = (Q @ K.T) / np.sqrt(d)
+    m_idx, n_idx = np.meshgrid(pos, pos, indexing="ij")
+    allowed = n_idx <= m_idx
+    if local:
+        allowed &= (n_idx < sinks) | (n_idx > m_idx - window)
+    z = np.where(allowed, z, -np.inf)
+    w = np.exp(z - z.max(axis=1, keepdims=True))
+    return (w @ v) / w.sum(axis=1, keepdims=True)
+
+
 def append_rows(k_pre, v, w_kidx_g, positions, base: float = 1e6):
     """Rows the append step stores for one KV head: bf16(R(n) k_pre_n), v_n and the index key
     bf16(W^K k_pre_n) ([P] §2.2 eq. (1), §3.2 eq. (4); R2, R7)."""

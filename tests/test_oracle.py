@@ -510,3 +510,62 @@ def test_full_attention_mass_bruteforce_tiny(N):
     w = [math.exp(x - zmax) for x in z]
     ref = sum(w[n] for n in sub) / sum(w)
     assert abs(O.full_attention_mass(q, kp, np.array(sub)) - ref) < 1e-12
+
+
+# ----------------------------------------------------------------------------- prefill (f1)
+def test_prefill_retrieval_matches_torch_causal_sdpa():
+    """Dense causal prefill against torch SDPA (is_causal) on the same RoPE'd inputs."""
+    rng = np.random.default_rng(11)
+    n = 48
+    q = rng.standard_normal((n, 128))
+    k = rng.standard_normal((n, 128))
+    v = rng.standard_normal((n, 128))
+    got = O.prefill_head(q, k, v, False, 4, 16)
+    pos = np.arange(n)
+    Q = torch.from_numpy(_rope_complex(q, pos))
+    K = torch.from_numpy(O.bf16_round(_rope_complex(k, pos)))
+    ref = torch.nn.functional.scaled_dot_product_attention(
+        Q[None, None], K[None, None], torch.from_numpy(v)[None, None], is_causal=True)[0, 0]
+    np.testing.assert_allclose(got, ref.numpy(), rtol=1e-10, atol=1e-12)
+
+
+def test_prefill_local_matches_sdpa_with_a_position_mask():
+    """Sinks + window prefill against torch SDPA with a boolean mask built row by row from
+    the pinned decode-time position sets (query m sees local_positions(m + 1))."""
+    rng = np.random.default_rng(12)
+    n, sinks, window = 40, 3, 7
+    q = rng.standard_normal((n, 128))
+    k = rng.standard_normal((n, 128))
+    v = rng.standard_normal((n, 128))
+    got = O.prefill_head(q, k, v, True, sinks, window)
+    mask = np.zeros((n, n), bool)
+    for m in range(n):
+        mask[m, O.local_positions(m + 1, sinks, window)] = True
+    pos = np.arange(n)
+    Q = torch.from_numpy(_rope_complex(q, pos))
+    K = torch.from_numpy(O.bf16_round(_rope_complex(k, pos)))
+    ref = torch.nn.functional.scaled_dot_product_attention(
+        Q[None, None], K[None, None], torch.from_numpy(v)[None, None],
+        attn_mask=torch.from_numpy(mask)[None, None])[0, 0]
+    np.testing.assert_allclose(got, ref.numpy(), rtol=1e-10, atol=1e-12)
+
+
+@pytest.mark.parametrize("local", [False, True])
+def test_prefill_rows_equal_the_decode_step(local):
+    """Row m of a prefill equals the decode-step attention with N = m + 1 (dense attention
+    for a retrieval head at p = 1, the sinks + window head for a local one): two oracle
+    paths for the same quantity."""
+    rng = np.random.default_rng(13 + int(local))
+    n, sinks, window = 30, 2, 5
+    q = rng.standard_normal((n, 128))
+    k = rng.standard_normal((n, 128))
+    v = rng.standard_normal((n, 128))
+    got = O.prefill_head(q, k, v, local, sinks, window)
+    for m in range(n):
+        if local:
+            ref = O.local_head(q[m], k[: m + 1], v[: m + 1], sinks, window).out
+        else:
+            pos = np.arange(m + 1)
+            ref = O.attend(O.rope_rotate(q[m], m), O.bf16_round(O.rope_rotate(k[: m + 1], pos)),
+                           v[: m + 1])
+        np.testing.assert_allclose(got[m], ref, rtol=1e-10, atol=1e-12)
