@@ -169,6 +169,29 @@ int rtp_decode_step_topk(const rtp_layer_desc* desc, const rtp_cache* cache,
                          int64_t k, uint16_t* out, int32_t* sel_counts, int32_t* sel_idx,
                          int64_t sel_stride, void* ws, size_t ws_bytes, rtp_stream_t stream);
 
+/*
+ * Causal prefill of one layer over a prompt at positions 0 .. n_b[b] - 1 (paper §3.2:
+ * retrieval heads attend densely in prefill, local heads to the attention sinks plus the
+ * sliding window in prefill as in decode). Query row m of head h attends to the positions
+ * j <= m (retrieval KV head of h) or to j < sinks and m - window < j <= m (local KV head);
+ * keys are R(j) k_pre rounded to bf16 as rtp_append_kv stores them, q = R(m) q_pre in
+ * single precision, weights softmax(q . k / sqrt(128)), out = sum of weights times v.
+ *   q_pre : bf16 [B][n_max][Hq][128], pre-RoPE queries.
+ *   k_pre, v : bf16 [B][n_max][Hkv][128], pre-RoPE keys and values (the same buffers an
+ *           rtp_append_kv of the prompt takes; this call does not write the cache).
+ *   n_b   : device int32 [B], prompt lengths; clamped to [0, n_max] on the device.
+ *   out   : bf16 [B][n_max][Hq][128]; rows m >= n_b[b] are not written.
+ *   ws    : at least rtp_prefill_workspace_bytes(desc, n_max) bytes, 256-byte aligned; it
+ *           holds the rotated keys and its contents are undefined afterwards (a decode
+ *           workspace reused here needs rtp_workspace_init before the next decode step).
+ * n_max == 0 does nothing. Errors: RTP_EINVAL (null pointer, n_max < 0), RTP_ESHAPE (bad
+ * description, n_max > max_seq_len), RTP_EWORKSPACE, RTP_ECUDA. Two launches.
+ */
+size_t rtp_prefill_workspace_bytes(const rtp_layer_desc* desc, int32_t n_max);
+int rtp_prefill(const rtp_layer_desc* desc, const uint16_t* q_pre, const uint16_t* k_pre,
+                const uint16_t* v, const int32_t* n_b, int32_t n_max, uint16_t* out, void* ws,
+                size_t ws_bytes, rtp_stream_t stream);
+
 /* Size of the library-owned scratch of rtp_decode_step_static (bytes). */
 #define RTP_STATIC_SCRATCH_BYTES (16u << 20)
 

@@ -5,4 +5,4 @@ one layer's caches and workspace with PyTorch and drives the library.
 """
 from . import rtp  # noqa: F401
 from .rtp import (rtp_append_kv, rtp_build_slot_map, rtp_decode_step,  # noqa: F401
-                  rtp_read_device_status, rtp_status_str, rtp_workspace_bytes, rtp_workspace_init)
+                  rtp_prefill, rtp_prefill_workspace_bytes, rtp_read_device_status, rtp_status_str, rtp_workspace_bytes, rtp_workspace_init)

@@ -15,7 +15,7 @@ EXPORTS = (
     "rtp_status_str", "rtp_build_slot_map", "rtp_workspace_bytes", "rtp_workspace_init",
     "rtp_append_kv", "rtp_decode_step", "rtp_read_device_status", "rtp_last_launch_count",
     "rtp_decode_step_static", "rtp_decode_step_append", "rtp_decode_step_topk", "rtp_debug_set_wait_limit",
-    "rtp_debug_fail_next_call",
+    "rtp_debug_fail_next_call", "rtp_prefill_workspace_bytes", "rtp_prefill",
 )
 RTP_STATIC_SCRATCH_BYTES = 16 << 20
 
@@ -72,6 +72,10 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.rtp_decode_step_topk.argtypes = [D, C, vp, vp, vp, i64, vp, vp, vp, i64, vp, sz, vp]
     lib.rtp_decode_step_static.restype = ctypes.c_int
     lib.rtp_decode_step_static.argtypes = [D, C, vp, vp, vp, ctypes.c_double, vp, vp, vp]
+    lib.rtp_prefill_workspace_bytes.restype = sz
+    lib.rtp_prefill_workspace_bytes.argtypes = [D, i32]
+    lib.rtp_prefill.restype = ctypes.c_int
+    lib.rtp_prefill.argtypes = [D, vp, vp, vp, vp, i32, vp, vp, sz, vp]
     lib.rtp_read_device_status.restype = ctypes.c_int
     lib.rtp_read_device_status.argtypes = [vp, vp]
     lib.rtp_last_launch_count.restype = i32

@@ -11,6 +11,7 @@
 #include "../../include/rtp.h"
 #include "rtp_attr_cache.h"
 #include "rtp_decode.cuh"
+#include "rtp_prefill.cuh"
 
 using namespace rtp;
 
@@ -212,6 +213,7 @@ int smem_layout(DecodeParams& P, const Plan& pl, int smem_optin) {
 // The shared-memory opt-in of decode_kernel<G> is a per-device function attribute: set it
 // once per (device, instance) (rtp_attr_cache.h).
 AttrCache<4, 64> g_attr;
+AttrCache<1, 64> g_attr_pf;     // prefill_kernel
 
 template <int G>
 int ensure_smem_attr(int dev, int smem) {
@@ -480,6 +482,42 @@ int rtp_decode_step_static(const rtp_layer_desc* desc, const rtp_cache* cache,
   if (cudaMemsetAsync(ws, 0, 256, (cudaStream_t)stream) != cudaSuccess) return RTP_ECUDA;
   return rtp_decode_step(desc, cache, q_pre, w_qidx, seq_lens, p, out, sel_counts, nullptr, 0,
                          ws, (size_t)RTP_STATIC_SCRATCH_BYTES, stream);
+}
+
+size_t rtp_prefill_workspace_bytes(const rtp_layer_desc* desc, int32_t n_max) {
+  LayerShape L;
+  if (check_desc(desc, L) != RTP_OK || n_max < 1 || n_max > desc->max_seq_len) return 0;
+  return align256((size_t)L.B * L.Hkv * (size_t)n_max * kD * sizeof(uint16_t));
+}
+
+int rtp_prefill(const rtp_layer_desc* desc, const uint16_t* q_pre, const uint16_t* k_pre,
+                const uint16_t* v, const int32_t* n_b, int32_t n_max, uint16_t* out, void* ws,
+                size_t ws_bytes, rtp_stream_t stream) {
+  g_launches = 0;
+  if (const int inj = take_injected()) return inj;
+  LayerShape L;
+  const int rc = check_desc(desc, L);
+  if (rc != RTP_OK) return rc;
+  if (!q_pre || !k_pre || !v || !n_b || !out || n_max < 0) return RTP_EINVAL;
+  if (n_max > desc->max_seq_len) return RTP_ESHAPE;
+  if (n_max == 0) return RTP_OK;
+  if (!ws || ws_bytes < rtp_prefill_workspace_bytes(desc, n_max)) return RTP_EWORKSPACE;
+  if ((reinterpret_cast<uintptr_t>(ws) & 255) != 0) return RTP_EWORKSPACE;
+  DevInfo di;
+  if (dev_info(di) != RTP_OK) return RTP_ECUDA;
+  const int rc2 = g_attr_pf.ensure(0, di.dev, kPfSmem, [](int, int bytes) {
+    return cudaFuncSetAttribute(prefill_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                bytes) == cudaSuccess ? 0 : 1;
+  });
+  if (rc2 != 0) return RTP_ECUDA;
+  cudaStream_t st = (cudaStream_t)stream;
+  uint16_t* k_rope = static_cast<uint16_t*>(ws);
+  const dim3 g1((n_max + kAppendTok - 1) / kAppendTok, L.B, L.Hkv);
+  prefill_rope_keys<<<g1, 128, 0, st>>>(L, k_pre, n_b, n_max, k_rope);
+  const dim3 g2((n_max + kPfQ - 1) / kPfQ, L.Hq, L.B);
+  prefill_kernel<<<g2, kPfThreads, kPfSmem, st>>>(L, q_pre, k_rope, v, n_b, n_max, out);
+  g_launches = 2;
+  return cudaGetLastError() == cudaSuccess ? RTP_OK : RTP_ECUDA;
 }
 
 int rtp_read_device_status(void* ws, rtp_stream_t stream) {

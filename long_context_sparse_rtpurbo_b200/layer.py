@@ -66,5 +66,25 @@ class DecodeLayer:
                                           w_qidx, seq_lens, p, out, sel_counts, sel_idx, stride,
                                           self.ws, self.ws_bytes, stream)
 
+    def prefill(self, q_pre, k_pre, v, w_kidx, n_b, out, stream=None):
+        """Prompt of n_b[b] tokens at positions 0..n_b[b]-1 (q_pre: bf16 [B][n_max][Hq][128];
+        k_pre, v: bf16 [B][n_max][Hkv][128]; n_b: device int32 [B]): appends its K/V and index
+        keys to the caches, then writes the causal prefill attention to out
+        ([B][n_max][Hq][128]). The prefill scratch is allocated on first use and grown with
+        the prompt."""
+        n_max = q_pre.shape[1]
+        start = torch.zeros(self.B, dtype=torch.int32, device=n_b.device)
+        rtp.rtp_append_kv(self.desc, self.cache, k_pre, v, w_kidx, start, n_b, n_max, self.ws,
+                          stream)
+        need = rtp.rtp_prefill_workspace_bytes(self.desc, n_max)
+        if need == 0:
+            raise ValueError("librtp rejected the prompt length")
+        if getattr(self, "pf_ws", None) is None or self.pf_ws.numel() < need:
+            buf = torch.empty(need + 256, dtype=torch.uint8, device=q_pre.device)
+            off = (-buf.data_ptr()) % 256
+            self.pf_ws = buf[off:off + need]
+        return rtp.rtp_prefill(self.desc, q_pre, k_pre, v, n_b, n_max, out, self.pf_ws,
+                               self.pf_ws.numel(), stream)
+
     def status(self, stream=None) -> int:
         return rtp.rtp_read_device_status(self.ws, stream)

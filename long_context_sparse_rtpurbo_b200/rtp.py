@@ -129,6 +129,20 @@ def rtp_decode_step_topk(desc: LayerDesc, cache: RtpCache, q_pre, w_qidx, seq_le
         _stream(stream)))
 
 
+def rtp_prefill_workspace_bytes(desc: LayerDesc, n_max: int) -> int:
+    return int(_lib.load().rtp_prefill_workspace_bytes(desc.ref, int(n_max)))
+
+
+def rtp_prefill(desc: LayerDesc, q_pre, k_pre, v, n_b, n_max, out, ws=None, ws_bytes=None,
+                stream=None):
+    """Causal prefill attention of one layer over a prompt (see include/rtp.h)."""
+    if ws_bytes is None:
+        ws_bytes = 0 if ws is None else ws.numel() * ws.element_size()
+    return _check("rtp_prefill", _lib.load().rtp_prefill(
+        desc.ref, _ptr(q_pre), _ptr(k_pre), _ptr(v), _ptr(n_b), int(n_max), _ptr(out), _ptr(ws),
+        int(ws_bytes), _stream(stream)))
+
+
 def rtp_decode_step_static(desc: LayerDesc, cache: RtpCache, q_pre, w_qidx, seq_lens, p, out,
                            sel_counts, stream=None):
     """rtp_decode_step on the library's own fixed scratch (no workspace argument): for callers

@@ -33,7 +33,7 @@ INV_STD = np.float32(1.0 / np.sqrt((65536.0 ** 2 - 1.0) / 3.0))
 IH_CENTRE = 2 * 65535
 
 # Tensor ids of the streams.
-T_KPRE, T_V, T_QPRE, T_WQIDX, T_WKIDX = 1, 2, 3, 4, 5
+T_KPRE, T_V, T_QPRE, T_WQIDX, T_WKIDX, T_QPROMPT = 1, 2, 3, 4, 5, 6
 
 
 def mix64(z):

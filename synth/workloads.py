@@ -110,6 +110,17 @@ class Workload:
         key = gen.stream_key(self.seed, gen.T_V, layer, b, kvh)
         return gen.token_rows_bits(key, t0, t1, self.head_dim)
 
+    def prompt_q_bits(self, layer: int, b: int, h: int, t0: int, t1: int,
+                      scale: float = 1.0) -> np.ndarray:
+        """bf16 bits [t1 - t0][128] of the pre-RoPE queries of query head h at prompt
+        positions t0..t1-1 (prefill inputs): rows of their own counter stream, each value
+        times ``scale`` (one float32 multiplication) before rounding; scale sets how peaked
+        the prompt's attention rows are."""
+        key = gen.stream_key(self.seed, gen.T_QPROMPT, layer, b, h)
+        c = np.arange(t0 * self.head_dim, t1 * self.head_dim, dtype=np.uint64)
+        x = gen.normal_f32(key, c.reshape(t1 - t0, self.head_dim)) * np.float32(scale)
+        return gen.f32_to_bf16_bits(x)
+
     def q_target(self, layer: int, b: int, h: int):
         """Target 16-dim projected query of a retrieval query head (float64), else None."""
         kvh = h // self.G

@@ -190,3 +190,78 @@ def check_outputs(w, layer, seq_lens, p, out, cnt, sel=None, heads=None, k=None)
         assert entry["max_abs"] <= MAX_ABS and entry["mean_abs"] <= MEAN_ABS, entry
         report["heads"].append(entry)
     return report
+
+
+# ------------------------------------------------------------------------------ prefill
+def prefill_inputs(w, layer, n_max, q_scale=1.0):
+    """bf16 bits of a prompt at positions 0..n_max-1 of every sequence: q_pre
+    [B][n_max][Hq][128] from the prompt-query streams, k_pre and v [B][n_max][Hkv][128] from
+    the same streams the decode workloads use."""
+    qb = np.zeros((w.B, n_max, w.Hq, 128), np.uint16)
+    kb = np.zeros((w.B, n_max, w.Hkv, 128), np.uint16)
+    vb = np.zeros_like(kb)
+    for b in range(w.B):
+        for h in range(w.Hq):
+            qb[b, :, h] = w.prompt_q_bits(layer, b, h, 0, n_max, q_scale)
+        for g in range(w.Hkv):
+            kb[b, :, g] = w.kpre_bits(layer, b, g, 0, n_max)
+            vb[b, :, g] = w.v_bits(layer, b, g, 0, n_max)
+    return qb, kb, vb
+
+
+def prefill(lay: DecodeLayer, qb, kb, vb, n_b, wk, device="cuda", sentinel=-7.0):
+    """rtp_prefill through the layer (append of the prompt, then the prefill attention); out
+    is pre-filled with ``sentinel`` so rows the call must not write can be checked."""
+    B, n_max = qb.shape[0], qb.shape[1]
+    q, k, v = (bits_to_torch(x, device) for x in (qb, kb, vb))
+    out = torch.full((B, n_max, lay.Hq, 128), sentinel, dtype=torch.bfloat16, device=device)
+    nb = torch.as_tensor(np.asarray(n_b, np.int32), device=device)
+    lay.prefill(q, k, v, wk, nb, out)
+    torch.cuda.synchronize()
+    return out
+
+
+def check_prefill(w, layer, n_b, qb, kb, vb, out, rows=None, heads=None,
+                  sentinel=-7.0) -> dict:
+    """Compares prefill outputs (device tensor [B][n_max][Hq][128]) with the oracle: every row
+    m < n_b[b] (oracle prefill_head) or the sampled ``rows`` (the row's own oracle: dense
+    attention over positions 0..m for a retrieval head, the sinks + window head with N = m + 1
+    for a local one), in the bf16 output format under the decode rule (max-abs <= 1e-2,
+    mean-abs <= 1e-3 per head); rows m >= n_b[b] must still hold the sentinel."""
+    out = out.float().cpu().numpy()
+    pairs = heads if heads is not None else [(b, h) for b in range(w.B) for h in range(w.Hq)]
+    report = dict(max_abs=0.0, mean_abs=0.0, rows=0)
+    krot = {}                # (b, g) -> the stored keys bf16(R(j) k_j) of a retrieval head
+    for (b, h) in pairs:
+        g = h // w.G
+        N = int(n_b[b])
+        local = not bool(w.ret_mask[layer, g])
+        assert np.all(out[b, N:, h] == sentinel), f"rows >= n_b written at (b={b}, h={h})"
+        if N == 0:
+            continue
+        q = bits_to_f64(qb[b, :N, h])
+        k = bits_to_f64(kb[b, :N, g])
+        v = bits_to_f64(vb[b, :N, g])
+        if rows is None:
+            ms = np.arange(N)
+            ref = O.prefill_head(q, k, v, local, w.sinks, w.window, w.rope_base)
+        else:
+            ms = np.unique(np.clip(np.asarray(rows, np.int64), 0, N - 1))
+            ref = np.zeros((ms.size, 128))
+            for i, m in enumerate(ms):
+                if local:
+                    ref[i] = O.local_head(q[m], k[:m + 1], v[:m + 1], w.sinks, w.window,
+                                          w.rope_base).out
+                else:
+                    if (b, g) not in krot:
+                        krot[(b, g)] = O.bf16_round(O.rope_rotate(k, np.arange(N), w.rope_base))
+                    K = krot[(b, g)][:m + 1]
+                    ref[i] = O.attend(O.rope_rotate(q[m], m, w.rope_base), K, v[:m + 1])
+        err = np.abs(out[b, ms, h] - O.bf16_round(ref))
+        mx, mn = float(err.max()), float(err.mean())
+        report["max_abs"] = max(report["max_abs"], mx)
+        report["mean_abs"] = max(report["mean_abs"], mn)
+        report["rows"] += int(ms.size)
+        assert mx <= MAX_ABS and mn <= MEAN_ABS, dict(b=b, h=h, local=local, max_abs=mx,
+                                                      mean_abs=mn)
+    return report
