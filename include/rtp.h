@@ -181,11 +181,18 @@ int rtp_decode_step_topk(const rtp_layer_desc* desc, const rtp_cache* cache,
  *           rtp_append_kv of the prompt takes; this call does not write the cache).
  *   n_b   : device int32 [B], prompt lengths; clamped to [0, n_max] on the device.
  *   out   : bf16 [B][n_max][Hq][128]; rows m >= n_b[b] are not written.
- *   ws    : at least rtp_prefill_workspace_bytes(desc, n_max) bytes, 256-byte aligned; it
- *           holds the rotated keys and its contents are undefined afterwards (a decode
- *           workspace reused here needs rtp_workspace_init before the next decode step).
+ *   ws    : at least rtp_prefill_workspace_bytes(desc, n_max) bytes, 256-byte aligned: a
+ *           status word (cleared by each call; rtp_read_device_status reads it) and the rotated
+ *           keys. A decode workspace reused here needs rtp_workspace_init before the next
+ *           decode step.
+ * S = Q K^T and P V run on the tensor cores (tcgen05) with fp32 accumulation; the query and
+ * the probabilities enter as two bf16 terms each (value and rounded remainder), so the result
+ * carries fp32-level error before the bf16 output rounding. A device wait for the tensor cores
+ * that runs out (rtp_debug_set_wait_limit) records RTP_ETIMEOUT in the status word and leaves
+ * the rows of that CTA unwritten.
  * n_max == 0 does nothing. Errors: RTP_EINVAL (null pointer, n_max < 0), RTP_ESHAPE (bad
- * description, n_max > max_seq_len), RTP_EWORKSPACE, RTP_ECUDA. Two launches.
+ * description, n_max > max_seq_len), RTP_EWORKSPACE, RTP_ECUDA. Two launches (and a 256-byte
+ * memset of the status word).
  */
 size_t rtp_prefill_workspace_bytes(const rtp_layer_desc* desc, int32_t n_max);
 int rtp_prefill(const rtp_layer_desc* desc, const uint16_t* q_pre, const uint16_t* k_pre,
@@ -233,7 +240,7 @@ int32_t rtp_last_launch_count(void);
  * Test hooks for the failure paths. The pages describe no failure handling; these exist so
  * the error paths can be exercised without faulting a GPU.
  *   rtp_debug_set_wait_limit: the limit, in SM clock cycles, of every device-side wait of
- *     later decode launches (0 restores the default of about one second; negative values are
+ *     later decode and prefill launches (0 restores the default of about one second; negative values are
  *     RTP_EINVAL). A wait that runs out records RTP_ETIMEOUT in the workspace status word and
  *     raises an abort flag that ends the launch's other waits; the outputs of that call are
  *     undefined and its workspace must be re-initialised with rtp_workspace_init. Process-wide.

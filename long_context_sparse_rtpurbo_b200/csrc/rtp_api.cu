@@ -484,10 +484,11 @@ int rtp_decode_step_static(const rtp_layer_desc* desc, const rtp_cache* cache,
                          ws, (size_t)RTP_STATIC_SCRATCH_BYTES, stream);
 }
 
+// prefill workspace: the status word (256 bytes), then the rotated keys [B][Hkv][n_max][128]
 size_t rtp_prefill_workspace_bytes(const rtp_layer_desc* desc, int32_t n_max) {
   LayerShape L;
   if (check_desc(desc, L) != RTP_OK || n_max < 1 || n_max > desc->max_seq_len) return 0;
-  return align256((size_t)L.B * L.Hkv * (size_t)n_max * kD * sizeof(uint16_t));
+  return 256 + align256((size_t)L.B * L.Hkv * (size_t)n_max * kD * sizeof(uint16_t));
 }
 
 int rtp_prefill(const rtp_layer_desc* desc, const uint16_t* q_pre, const uint16_t* k_pre,
@@ -511,11 +512,19 @@ int rtp_prefill(const rtp_layer_desc* desc, const uint16_t* q_pre, const uint16_
   });
   if (rc2 != 0) return RTP_ECUDA;
   cudaStream_t st = (cudaStream_t)stream;
-  uint16_t* k_rope = static_cast<uint16_t*>(ws);
+  if (cudaMemsetAsync(ws, 0, 256, st) != cudaSuccess) return RTP_ECUDA;
+  uint16_t* k_rope = at<uint16_t>(ws, 256);
   const dim3 g1((n_max + kAppendTok - 1) / kAppendTok, L.B, L.Hkv);
   prefill_rope_keys<<<g1, 128, 0, st>>>(L, k_pre, n_b, n_max, k_rope);
+  PrefillParams PP;
+  memset(&PP, 0, sizeof(PP));
+  PP.L = L;
+  PP.q_pre = q_pre; PP.k_rope = k_rope; PP.v = v; PP.n_b = n_b; PP.out = out;
+  PP.status = static_cast<int*>(ws);
+  PP.spin_limit = g_spin_limit.load();
+  PP.n_max = n_max;
   const dim3 g2((n_max + kPfQ - 1) / kPfQ, L.Hq, L.B);
-  prefill_kernel<<<g2, kPfThreads, kPfSmem, st>>>(L, q_pre, k_rope, v, n_b, n_max, out);
+  prefill_kernel<<<g2, kPfThreads, kPfSmem, st>>>(PP);
   g_launches = 2;
   return cudaGetLastError() == cudaSuccess ? RTP_OK : RTP_ECUDA;
 }

@@ -5,26 +5,38 @@
 // prefill_rope_keys: the prompt's keys rotated by R(j) with the append's arithmetic (double
 // angles and rotation, one rounding to bf16), so they equal the cache rows the append writes;
 // local heads need them because their ring keeps only the last window.
-// prefill_kernel: one CTA of 4 warps per (64 query rows, query head, sequence); K/V tiles of
-// 64 rows, double-buffered with cp.async (16-byte chunks XOR-swizzled by the row), over the
-// tiles the head can see (causal; local heads skip the tiles between the sinks and the
-// window). Per warp 16 query rows: S = Q K^T and O += P V on the tensor cores (mma.sync
-// m16n8k16, bf16 x bf16 -> fp32), the query and the probabilities each as two bf16 terms (the
-// rounded value and its rounded remainder) so logits and outputs keep fp32-level accuracy;
-// online softmax in the log2 domain (the query carries log2(e) / sqrt(128)).
+// prefill_kernel: one CTA of 4 warps per (128 query rows, query head, sequence), two CTAs per
+// SM; thread t owns query row t. Over the 64-key tiles the rows can see (causal; local heads
+// skip the tiles between the sinks and the window), with K and V tiles staged by cp.async in
+// the 128-byte-swizzled operand layout:
+//   S = Q K^T on the fifth-generation tensor cores (tcgen05.mma, 128 x 64, fp32 in tensor
+//   memory), the query as two bf16 terms (the rounded value and its rounded remainder) so the
+//   logits keep fp32-level accuracy;
+//   masked online softmax in the log2 domain (the query carries log2(e) / sqrt(128)), the
+//   probabilities written back to tensor memory as two bf16 terms;
+//   the tile's P V from tensor memory (TS form, 128 x 128), added to the thread's fp32 output
+//   row in registers after the running-maximum rescale.
+// The next K tile loads while the softmax runs, the next V tile while the next S is computed.
 #pragma once
 
 #include "rtp_append.cuh"
 #include "rtp_attend.cuh"
+#include "rtp_tmem.cuh"
+#include "rtp_umma.cuh"
 
 namespace rtp {
 
-constexpr int kPfThreads = 128;      // 4 warps
-constexpr int kPfQ = 64;             // query rows per CTA (16 per warp)
-constexpr int kPfK = 64;             // key rows per tile
-constexpr int kPfQBytes = 2 * kPfQ * 256;            // q hi, q lo: [64 rows][256 B] each
-constexpr int kPfTileBytes = 2 * kPfK * 256;         // K then V
-constexpr int kPfSmem = kPfQBytes + 2 * kPfTileBytes;   // 96 KB
+constexpr int kPfThreads = 128;      // 4 warps: thread t owns query row t (tensor-memory lane t)
+constexpr int kPfQ = 128;            // query rows per CTA (the MMA's M)
+constexpr int kPfK = 64;             // keys per tile
+constexpr uint32_t kPfQBlock = kPfQ * 128;                // one 64-dim block of the query tile
+constexpr uint32_t kPfBlock = kPfK * 128;                 // one 64-dim block of a K or V tile
+constexpr uint32_t kPfQHi = 0, kPfQLo = 2 * kPfQBlock;    // query terms: 2 blocks each
+constexpr uint32_t kPfKt = 4 * kPfQBlock, kPfVt = kPfKt + 2 * kPfBlock;
+constexpr uint32_t kPfBar = kPfVt + 2 * kPfBlock;         // two mbarriers, the tensor-memory word
+constexpr int kPfSmem = (int)kPfBar + 64 + 1024;          // + slack to align the base to 1024
+constexpr uint32_t kPfTmemCols = 256;  // S, then P hi / lo, in [0, 64); the PV tile in [128, 256)
+constexpr uint32_t kPfColO = 128;
 
 __global__ void __launch_bounds__(128)
 prefill_rope_keys(LayerShape L, const uint16_t* __restrict__ k_pre, const int32_t* __restrict__ n_b,
@@ -46,207 +58,253 @@ prefill_rope_keys(LayerShape L, const uint16_t* __restrict__ k_pre, const int32_
   }
 }
 
-// byte offset of channel c (bf16) of row r in a 256-byte-row tile with swizzled chunks
-__device__ __forceinline__ int pf_off(int r, int c) {
-  return r * 256 + ((((c >> 3) ^ (r & 7))) << 4) + (c & 7) * 2;
-}
-
 // next key tile at or after kt that a query tile [q0, q1] can see (-1: none); local heads see
 // keys [0, sinks) and (q0 - window, q1]
 __device__ __forceinline__ int pf_next_tile(int kt, int q0, int q1, bool local, int sinks,
                                             int window) {
   const int last = q1 / kPfK;
-  for (; kt <= last; ++kt) {
-    if (!local) return kt;
-    const int k0 = kt * kPfK, k1 = k0 + kPfK - 1;
-    if (k0 < sinks || k1 > q0 - window) return kt;
-  }
-  return -1;
+  if (kt > last) return -1;
+  if (!local || kt * kPfK < sinks) return kt;
+  const int first_win = max(q0 - window + 1, 0) / kPfK;   // tile of the lowest window key
+  const int n = max(kt, first_win);
+  return n <= last ? n : -1;
 }
 
-__global__ void __launch_bounds__(kPfThreads)
-prefill_kernel(LayerShape L, const uint16_t* __restrict__ q_pre, const uint16_t* __restrict__ k_rope,
-               const uint16_t* __restrict__ v, const int32_t* __restrict__ n_b, int n_max,
-               uint16_t* __restrict__ out) {
-  extern __shared__ __align__(16) unsigned char pf_smem[];
-  // the longest causal rows first, so the short tiles fill the tail of the grid
+struct PrefillParams {
+  LayerShape L;
+  const uint16_t* q_pre;     // [B][n_max][Hq][128]
+  const uint16_t* k_rope;    // [B][Hkv][n_max][128]
+  const uint16_t* v;         // [B][n_max][Hkv][128]
+  const int32_t* n_b;
+  uint16_t* out;             // [B][n_max][Hq][128]
+  int* status;
+  long long spin_limit;
+  int n_max;
+};
+
+__device__ __forceinline__ float pf_ex2(float x) {
+  float r;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
+  return r;
+}
+
+// Load one 64-row K or V tile into its 128-byte-swizzled blocks (dims 0-63, then 64-127);
+// rows past the prompt are zeros (their probabilities are 0 and must meet finite values).
+__device__ __forceinline__ void pf_load_tile(uint32_t dst, const uint16_t* src, int64_t stride,
+                                             int kt, int nb) {
+  const int t = threadIdx.x;
+#pragma unroll
+  for (int u = 0; u < (kPfK * 16) / kPfThreads; ++u) {
+    const int e = t + u * kPfThreads, r = e >> 4, c16 = e & 15;
+    const int key = kt * kPfK + r;
+    const uint32_t off = dst + (uint32_t)(c16 >> 3) * kPfBlock + sw128_off(r, c16 & 7);
+    if (key < nb) cp_async16_s(off, src + key * stride + c16 * 8);
+    else st_shared_zero16(off);
+  }
+}
+
+__global__ void __launch_bounds__(kPfThreads, 2) prefill_kernel(PrefillParams P) {
+  extern __shared__ __align__(1024) unsigned char pf_raw[];
+  const LayerShape& L = P.L;
   const int qt = gridDim.x - 1 - blockIdx.x, h = blockIdx.y, b = blockIdx.z;
-  const int nb = min(max(n_b[b], 0), n_max);
+  const int nb = min(max(P.n_b[b], 0), P.n_max);
   const int q0 = qt * kPfQ;
   if (q0 >= nb) return;
   const int q1 = min(q0 + kPfQ, nb) - 1;                 // last query row of the CTA
   const int g = h / L.G;
   const bool local = L.slot[g] < 0;
-  const int t = threadIdx.x, lane = t & 31, warp = t >> 5, gid = lane >> 2, tig = lane & 3;
-  unsigned char* qs = pf_smem;                            // hi, then lo at + kPfQ * 256
-  unsigned char* tiles = pf_smem + kPfQBytes;
-  const uint16_t* kbase = k_rope + ((int64_t)b * L.Hkv + g) * n_max * kD;
-
-  auto issue = [&](int kt, int stage) {
-    unsigned char* kd = tiles + stage * kPfTileBytes;
-    unsigned char* vd = kd + kPfK * 256;
-#pragma unroll
-    for (int u = 0; u < (kPfK * 16) / kPfThreads; ++u) {
-      const int e = t + u * kPfThreads, r = e >> 4, c = e & 15;
-      const int key = kt * kPfK + r;
-      const int off = r * 256 + ((c ^ (r & 7)) << 4);
-      if (key < nb) {
-        cp_async16(kd + off, kbase + (int64_t)key * kD + c * 8);
-        cp_async16(vd + off, v + (((int64_t)b * n_max + key) * L.Hkv + g) * kD + c * 8);
-      } else {                                            // zero V: masked keys must add 0
-        *reinterpret_cast<uint4*>(vd + off) = make_uint4(0u, 0u, 0u, 0u);
-      }
-    }
-    cp_async_commit();
-  };
+  const int t = threadIdx.x, warp = t >> 5;
+  const uint32_t raw = smem_u32(pf_raw);
+  const uint32_t base = (raw + 1023u) & ~1023u;          // swizzle atoms need 1024-byte alignment
+  unsigned char* sm = pf_raw + (base - raw);
+  const uint32_t sQh = base + kPfQHi, sQl = base + kPfQLo, sK = base + kPfKt, sV = base + kPfVt;
+  const uint32_t barS = base + kPfBar, barO = barS + 8, tword = barS + 16;
+  const uint16_t* kbase = P.k_rope + ((int64_t)b * L.Hkv + g) * P.n_max * kD;
+  const uint16_t* vbase = P.v + (int64_t)b * P.n_max * L.Hkv * kD + (int64_t)g * kD;
+  const int64_t vstride = (int64_t)L.Hkv * kD;
 
   int kt = pf_next_tile(0, q0, q1, local, L.sinks, L.window);
-  issue(kt, 0);
-  // the rotated, scaled query rows, split into two bf16 terms
+  pf_load_tile(sK, kbase, kD, kt, nb);
+  cp_async_commit();
+  pf_load_tile(sV, vbase, vstride, kt, nb);
+  cp_async_commit();
+  // the rotated, scaled query rows as two bf16 terms (hi, lo), K-major 128-byte-swizzled
   const float scale = kLog2e * 0.08838834764831845f;    // log2(e) / sqrt(128)
-  for (int e = t; e < kPfQ * 64; e += kPfThreads) {
-    const int r = e >> 6, i = e & 63, m = q0 + r;
-    float x0 = 0.f, x1 = 0.f;
+#pragma unroll 1
+  for (int u = 0; u < (kPfQ * 8) / kPfThreads; ++u) {
+    const int e = t + u * kPfThreads, r = e >> 3, c = e & 7;   // row r, dims 8c.. and 64 + 8c..
+    const int m = q0 + r;
+    uint32_t h0[4] = {0, 0, 0, 0}, l0[4] = {0, 0, 0, 0}, h1[4] = {0, 0, 0, 0}, l1[4] = {0, 0, 0, 0};
     if (m < nb) {
-      const uint16_t* q = q_pre + (((int64_t)b * n_max + m) * L.Hq + h) * kD;
-      float sn, cs;
-      rope_sincosf((double)m, L.theta[i], &sn, &cs);
-      const float qa = bf1(q[i]), qb = bf1(q[i + 64]);
-      x0 = (qa * cs - qb * sn) * scale;
-      x1 = (qa * sn + qb * cs) * scale;
+      const uint16_t* q = P.q_pre + (((int64_t)b * P.n_max + m) * L.Hq + h) * kD;
+      const uint4 wa = *reinterpret_cast<const uint4*>(q + 8 * c);
+      const uint4 wb = *reinterpret_cast<const uint4*>(q + 64 + 8 * c);
+      float qa[8], qb[8];
+      unpack8(wa, qa);
+      unpack8(wb, qb);
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        float x[2], y[2];
+#pragma unroll
+        for (int z = 0; z < 2; ++z) {
+          const int j = 2 * k + z;
+          float sn, cs;
+          rope_sincosf((double)m, L.theta[8 * c + j], &sn, &cs);
+          x[z] = (qa[j] * cs - qb[j] * sn) * scale;
+          y[z] = (qa[j] * sn + qb[j] * cs) * scale;
+        }
+        split_bf2(x[0], x[1], h0[k], l0[k]);
+        split_bf2(y[0], y[1], h1[k], l1[k]);
+      }
     }
-    uint32_t h0, l0, h1, l1;
-    split_bf2(x0, 0.f, h0, l0);
-    split_bf2(x1, 0.f, h1, l1);
-    *reinterpret_cast<uint16_t*>(qs + pf_off(r, i)) = (uint16_t)h0;
-    *reinterpret_cast<uint16_t*>(qs + kPfQ * 256 + pf_off(r, i)) = (uint16_t)l0;
-    *reinterpret_cast<uint16_t*>(qs + pf_off(r, i + 64)) = (uint16_t)h1;
-    *reinterpret_cast<uint16_t*>(qs + kPfQ * 256 + pf_off(r, i + 64)) = (uint16_t)l1;
+    const uint32_t o0 = sw128_off(r, c);
+    *reinterpret_cast<uint4*>(sm + kPfQHi + o0) = make_uint4(h0[0], h0[1], h0[2], h0[3]);
+    *reinterpret_cast<uint4*>(sm + kPfQHi + kPfQBlock + o0) = make_uint4(h1[0], h1[1], h1[2], h1[3]);
+    *reinterpret_cast<uint4*>(sm + kPfQLo + o0) = make_uint4(l0[0], l0[1], l0[2], l0[3]);
+    *reinterpret_cast<uint4*>(sm + kPfQLo + kPfQBlock + o0) = make_uint4(l1[0], l1[1], l1[2], l1[3]);
   }
+  fence_async_smem();
+  if (t == 0) {
+    mbar_init(barS, 1);
+    mbar_init(barO, 1);
+    mbar_init_fence();
+  }
+  if (warp == 0) tmem_alloc_cols(tword, kPfTmemCols);
+  tmem_fence_before_sync();
+  __syncthreads();
+  tmem_fence_after_sync();
+  const uint32_t tm = *reinterpret_cast<volatile uint32_t*>(sm + kPfBar + 16);
+  const uint32_t tl = tm + ((uint32_t)(warp * 32) << 16);     // this thread's lane (row t)
+  constexpr uint32_t idS = umma_idesc_bf16(kPfQ, kPfK, 0);   // S = Q K^T: 128 x 64, K-major B
+  constexpr uint32_t idO = umma_idesc_bf16(kPfQ, kD, 1);     // O = P V: 128 x 128, MN-major B
 
-  float o[16][4];
+  float o[kD];
 #pragma unroll
-  for (int d = 0; d < 16; ++d)
-#pragma unroll
-    for (int e = 0; e < 4; ++e) o[d][e] = 0.f;
-  float mrow[2] = {-INFINITY, -INFINITY}, lrow[2] = {0.f, 0.f};
-  const int row0 = q0 + warp * 16 + gid;                  // this thread's rows: row0, row0 + 8
-  const uint32_t qaddr = smem_u32(qs);
-  int stage = 0;
+  for (int d = 0; d < kD; ++d) o[d] = 0.f;
+  float m_run = -INFINITY, l_run = 0.f;
+  const int row = q0 + t;
+  int j = 0, pend = 0;                                      // pend: 1 S, 2 PV in flight at an abort
 #pragma unroll 1
   while (kt >= 0) {
     const int kn = pf_next_tile(kt + 1, q0, q1, local, L.sinks, L.window);
-    cp_async_wait<0>();
-    __syncthreads();                                      // tile kt landed; the other stage is free
-    if (kn >= 0) issue(kn, stage ^ 1);
-    const uint32_t kaddr = smem_u32(tiles + stage * kPfTileBytes);
-    const uint32_t vaddr = kaddr + kPfK * 256;
-    // S = Q K^T: 16 rows x 64 keys (8 key tiles of 8)
-    float s[8][4];
+    cp_async_wait<1>();                                     // K tile kt landed (V may be pending)
+    fence_async_smem();
+    tmem_fence_before_sync();
+    __syncthreads();
+    if (t == 0) {
+      tmem_fence_after_sync();
 #pragma unroll
-    for (int n = 0; n < 8; ++n)
-#pragma unroll
-      for (int e = 0; e < 4; ++e) s[n][e] = 0.f;
-#pragma unroll
-    for (int kk = 0; kk < 8; ++kk) {
-      uint32_t ah[4], al[4];
-      {
-        const int r = warp * 16 + (lane & 7) + ((lane >> 3) & 1) * 8, c = 2 * kk + (lane >> 4);
-        const uint32_t off = r * 256 + ((c ^ (r & 7)) << 4);
-        ldsm_x4(qaddr + off, ah);
-        ldsm_x4(qaddr + kPfQ * 256 + off, al);
+      for (int ks = 0; ks < kD / 16; ++ks) {
+        const uint32_t ko = (uint32_t)(ks >> 2) * kPfBlock + (uint32_t)(ks & 3) * 32;
+        const uint32_t qo = (uint32_t)(ks >> 2) * kPfQBlock + (uint32_t)(ks & 3) * 32;
+        const uint64_t bk = umma_desc_sw128(sK + ko, 16, 1024);
+        umma_ss(tm, umma_desc_sw128(sQh + qo, 16, 1024), bk, idS, ks > 0);
+        umma_ss(tm, umma_desc_sw128(sQl + qo, 16, 1024), bk, idS, 1);
       }
+      umma_commit(barS);
+    }
+    __syncwarp();
+    if (__syncthreads_or(!mbar_wait(barS, j & 1, P.spin_limit))) { pend = 1; break; }
+    tmem_fence_after_sync();
+    if (kn >= 0) pf_load_tile(sK, kbase, kD, kn, nb);       // the K buffer is free again
+    cp_async_commit();
+    // masked online softmax of row `row` over the tile's 64 keys, 32 columns at a time: the
+    // maximum first, then the probabilities, each half's two bf16 terms written over its own
+    // scores (hi, then lo: columns 32 half + [0, 16) and + [16, 32))
+    const int k0 = kt * kPfK;
+    const int lo_ok = local ? row - L.window : -1;          // local: keys > lo_ok or < sinks
+    float mx = -INFINITY;
 #pragma unroll
-      for (int np = 0; np < 4; ++np) {                     // key tiles 2 np, 2 np + 1
-        uint32_t bk[4];
-        const int r = (2 * np + (lane >> 4)) * 8 + (lane & 7), c = 2 * kk + ((lane >> 3) & 1);
-        ldsm_x4(kaddr + r * 256 + ((c ^ (r & 7)) << 4), bk);
-        mma_bf16(s[2 * np], ah, bk[0], bk[1]);
-        mma_bf16(s[2 * np], al, bk[0], bk[1]);
-        mma_bf16(s[2 * np + 1], ah, bk[2], bk[3]);
-        mma_bf16(s[2 * np + 1], al, bk[2], bk[3]);
+    for (int half = 0; half < 2; ++half) {
+      uint32_t sr[32];
+      tmem_ld32(tl + 32 * half, sr);
+      tmem_wait_ld();
+#pragma unroll
+      for (int i = 0; i < 32; ++i) {
+        const int key = k0 + 32 * half + i;
+        const bool ok = key <= row && key < nb && (key > lo_ok || key < L.sinks);
+        mx = ok ? fmaxf(mx, __uint_as_float(sr[i])) : mx;
       }
     }
-    // masks and the online softmax (rows row0 and row0 + 8; a quad of lanes shares a row)
-    float mx[2] = {-INFINITY, -INFINITY};
+    const float mn = fmaxf(m_run, mx);
+    const float alpha = mn == -INFINITY ? 1.f : pf_ex2(m_run - mn);
+    m_run = mn;
+    float lsum = 0.f;
 #pragma unroll
-    for (int n = 0; n < 8; ++n) {
+    for (int half = 0; half < 2; ++half) {
+      uint32_t sr[32], ph[16], pl[16];
+      tmem_ld32(tl + 32 * half, sr);
+      tmem_wait_ld();
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const int row = row0 + (e >> 1) * 8;
-        const int key = kt * kPfK + n * 8 + 2 * tig + (e & 1);
-        bool ok = key <= row && key < nb;
-        if (local) ok = ok && (key < L.sinks || key > row - L.window);
-        s[n][e] = ok ? s[n][e] : -INFINITY;
-        mx[e >> 1] = fmaxf(mx[e >> 1], s[n][e]);
+      for (int c = 0; c < 16; ++c) {
+        const int key = k0 + 32 * half + 2 * c;
+        const bool ok0 = key <= row && key < nb && (key > lo_ok || key < L.sinks);
+        const bool ok1 = key + 1 <= row && key + 1 < nb && (key + 1 > lo_ok || key + 1 < L.sinks);
+        const float p0 = ok0 ? pf_ex2(__uint_as_float(sr[2 * c]) - mn) : 0.f;
+        const float p1 = ok1 ? pf_ex2(__uint_as_float(sr[2 * c + 1]) - mn) : 0.f;
+        lsum += p0 + p1;
+        split_bf2(p0, p1, ph[c], pl[c]);
       }
+      tmem_st16(tl + 32 * half, ph);
+      tmem_st16(tl + 32 * half + 16, pl);
     }
-    float al2[2];
+    l_run = l_run * alpha + lsum;
+    tmem_wait_st();
+    cp_async_wait<1>();                                     // V tile kt landed
+    fence_async_smem();
+    tmem_fence_before_sync();
+    __syncthreads();
+    if (t == 0) {
+      tmem_fence_after_sync();
 #pragma unroll
-    for (int u = 0; u < 2; ++u) {
-      mx[u] = fmaxf(mx[u], __shfl_xor_sync(0xffffffffu, mx[u], 1));
-      mx[u] = fmaxf(mx[u], __shfl_xor_sync(0xffffffffu, mx[u], 2));
-      const float mn = fmaxf(mrow[u], mx[u]);
-      al2[u] = mn == -INFINITY ? 1.f : exp2f(mrow[u] - mn);
-      mrow[u] = mn;
-      lrow[u] *= al2[u];
-    }
-#pragma unroll
-    for (int d = 0; d < 16; ++d) {
-      o[d][0] *= al2[0]; o[d][1] *= al2[0];
-      o[d][2] *= al2[1]; o[d][3] *= al2[1];
-    }
-#pragma unroll
-    for (int n = 0; n < 8; ++n)
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const float m = mrow[e >> 1];
-        const float pv = s[n][e] == -INFINITY ? 0.f : exp2f(s[n][e] - m);
-        s[n][e] = pv;
-        lrow[e >> 1] += pv;
+      for (int ks = 0; ks < kPfK / 16; ++ks) {
+        const uint64_t bv = umma_desc_sw128(sV + (uint32_t)ks * 2048, kPfBlock, 1024);
+        const uint32_t pa = tm + 32 * (ks >> 1) + 8 * (ks & 1);   // P hi of keys 16 ks..
+        umma_ts(tm + kPfColO, pa, bv, idO, ks > 0);
+        umma_ts(tm + kPfColO, pa + 16, bv, idO, 1);                // P lo
       }
-    // O += P V: P (16 x 64) as the A operand, 4 key steps of 16; V^T fragments by ldmatrix.trans
+      umma_commit(barO);
+    }
+    __syncwarp();
+    if (__syncthreads_or(!mbar_wait(barO, j & 1, P.spin_limit))) { pend = 2; break; }
+    tmem_fence_after_sync();
+    if (kn >= 0) pf_load_tile(sV, vbase, vstride, kn, nb);  // the V buffer is free again
+    cp_async_commit();
 #pragma unroll
-    for (int kk = 0; kk < 4; ++kk) {
-      uint32_t ph[4], pl[4];
-      split_bf2(s[2 * kk][0], s[2 * kk][1], ph[0], pl[0]);
-      split_bf2(s[2 * kk][2], s[2 * kk][3], ph[1], pl[1]);
-      split_bf2(s[2 * kk + 1][0], s[2 * kk + 1][1], ph[2], pl[2]);
-      split_bf2(s[2 * kk + 1][2], s[2 * kk + 1][3], ph[3], pl[3]);
+    for (int c = 0; c < kD / 32; ++c) {
+      uint32_t r[32];
+      tmem_ld32(tl + kPfColO + 32 * c, r);
+      tmem_wait_ld();
 #pragma unroll
-      for (int dp = 0; dp < 8; ++dp) {                     // dim tiles 2 dp, 2 dp + 1
-        uint32_t bv[4];
-        const int r = kk * 16 + (lane & 7) + ((lane >> 3) & 1) * 8, c = 2 * dp + (lane >> 4);
-        ldsm_x4_t(vaddr + r * 256 + ((c ^ (r & 7)) << 4), bv);
-        mma_bf16(o[2 * dp], ph, bv[0], bv[1]);
-        mma_bf16(o[2 * dp], pl, bv[0], bv[1]);
-        mma_bf16(o[2 * dp + 1], ph, bv[2], bv[3]);
-        mma_bf16(o[2 * dp + 1], pl, bv[2], bv[3]);
-      }
+      for (int i = 0; i < 32; ++i) o[32 * c + i] = fmaf(o[32 * c + i], alpha, __uint_as_float(r[i]));
     }
     kt = kn;
-    stage ^= 1;
+    ++j;
+  }
+  if (pend) {
+    // a wait ran out: record it, let the MMA in flight finish (bounded) before the columns are
+    // freed, and leave this CTA's rows unwritten
+    if (t == 0) set_status(P.status, -5);
+    mbar_wait(pend == 1 ? barS : barO, j & 1, 2000000000LL);
+  } else if (row <= q1) {
+    uint16_t* dst = P.out + (((int64_t)b * P.n_max + row) * L.Hq + h) * kD;
+    const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
+#pragma unroll
+    for (int c = 0; c < kD / 8; ++c) {
+      uint4 w;
+      w.x = pack_bf2(o[8 * c] * inv, o[8 * c + 1] * inv);
+      w.y = pack_bf2(o[8 * c + 2] * inv, o[8 * c + 3] * inv);
+      w.z = pack_bf2(o[8 * c + 4] * inv, o[8 * c + 5] * inv);
+      w.w = pack_bf2(o[8 * c + 6] * inv, o[8 * c + 7] * inv);
+      *reinterpret_cast<uint4*>(dst + 8 * c) = w;
+    }
   }
   cp_async_wait<0>();
-  // the row sums over the quad, then O / l in bf16
-#pragma unroll
-  for (int u = 0; u < 2; ++u) {
-    lrow[u] += __shfl_xor_sync(0xffffffffu, lrow[u], 1);
-    lrow[u] += __shfl_xor_sync(0xffffffffu, lrow[u], 2);
-  }
-#pragma unroll
-  for (int u = 0; u < 2; ++u) {
-    const int row = row0 + u * 8;
-    if (row > q1) continue;
-    uint16_t* dst = out + (((int64_t)b * n_max + row) * L.Hq + h) * kD;
-    const float inv = lrow[u] > 0.f ? 1.f / lrow[u] : 0.f;
-#pragma unroll
-    for (int d = 0; d < 16; ++d) {
-      const int c = d * 8 + 2 * tig;
-      const uint32_t pk = (uint32_t)f2bf_rn(o[d][2 * u] * inv) |
-                          ((uint32_t)f2bf_rn(o[d][2 * u + 1] * inv) << 16);
-      *reinterpret_cast<uint32_t*>(dst + c) = pk;
-    }
+  tmem_fence_before_sync();
+  __syncthreads();
+  if (warp == 0) {
+    __syncwarp();
+    tmem_dealloc_cols(tm, kPfTmemCols);
   }
 }
 

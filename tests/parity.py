@@ -34,8 +34,8 @@ def bits_to_torch(bits: np.ndarray, device) -> torch.Tensor:
 def layer_inputs(w, layer, device):
     """q_pre (bf16, device), W_qidx / W_kidx (fp32, device) of one layer."""
     q = bits_to_torch(w.q_pre_bits(layer), device)
-    wq = torch.from_numpy(np.ascontiguousarray(w.w_qidx(layer))).to(device)
-    wk = torch.from_numpy(np.ascontiguousarray(w.w_kidx(layer))).to(device)
+    wq = torch.from_numpy(np.array(w.w_qidx(layer), np.float32)).to(device)
+    wk = torch.from_numpy(np.array(w.w_kidx(layer), np.float32)).to(device)
     return q, wq, wk
 
 

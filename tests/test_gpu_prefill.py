@@ -123,7 +123,7 @@ def test_prefill_argument_errors():
     nb = torch.full((1,), 64, dtype=torch.int32, device=DEV)
     out = torch.zeros_like(q)
     need = rtp.rtp_prefill_workspace_bytes(lay.desc, 64)
-    assert need == 64 * w.Hkv * 256
+    assert need == 256 + 64 * w.Hkv * 256
     ws = torch.zeros(need, dtype=torch.uint8, device=DEV)
     for args, code in (((lay.desc, q, kv, kv, nb, -1, out, ws), RTP_EINVAL),
                        ((lay.desc, q, kv, kv, nb, 65, out, ws), RTP_ESHAPE),
@@ -133,3 +133,27 @@ def test_prefill_argument_errors():
             rtp.rtp_prefill(*args)
         assert e.value.code == code
     assert rtp.rtp_prefill(lay.desc, q, kv, kv, nb, 0, out, None) == 0   # nothing to do
+
+
+def test_prefill_wait_timeout_then_recovery():
+    """With the device-wait limit at one SM cycle the prefill's first wait for its MMAs runs
+    out: the call returns, the status word holds RTP_ETIMEOUT and the rows stay unwritten;
+    with the default limit the same prompt then meets parity."""
+    from long_context_sparse_rtpurbo_b200 import rtp
+    from long_context_sparse_rtpurbo_b200._lib import RTP_ETIMEOUT
+    P = _parity()
+    w = _small(B=1)
+    n = 200
+    lay = P.make_layer(w, 0, DEV, seq_lens=[n], caps=[n])
+    qb, kb, vb = P.prefill_inputs(w, 0, n, 2.0)
+    try:
+        rtp.rtp_debug_set_wait_limit(1)
+        out = P.prefill(lay, qb, kb, vb, [n], _wk(w, 0), DEV)
+        st = rtp.rtp_read_device_status(lay.pf_ws)
+    finally:
+        rtp.rtp_debug_set_wait_limit(0)
+    assert st == RTP_ETIMEOUT
+    assert bool((out.float() == -7.0).all())
+    out = P.prefill(lay, qb, kb, vb, [n], _wk(w, 0), DEV)
+    assert rtp.rtp_read_device_status(lay.pf_ws) == 0
+    P.check_prefill(w, 0, [n], qb, kb, vb, out)
