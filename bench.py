@@ -622,6 +622,185 @@ class GpuWorkload:
         torch.cuda.empty_cache()
 
 
+def load_tensor_peak():
+    """Dense bf16 tensor-core peak (TFLOP/s): the sustained cuBLAS figure (a prefill step runs
+    for a fraction of a second under the power cap)."""
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["bf16_tflops_sustained"]), "measured bf16_tflops_sustained"
+    return 1400.0, "fallback (sustained)"
+
+
+def prefill_flops(w, n):
+    """Algorithmic FLOPs of the attention of a prefill of n tokens over every layer: 4 * 128
+    per (query head, row m, attended key), attended = m + 1 for a retrieval head and
+    min(m + 1, sinks + window) for a local one."""
+    m = np.arange(n, dtype=np.float64)
+    dense = float((m + 1).sum())
+    local = float(np.minimum(m + 1, w.sinks + w.window).sum())
+    per = [(dense if w.ret_mask[l, g] else local) * w.G for l in range(w.layers)
+           for g in range(w.Hkv)]
+    return 4.0 * 128 * float(sum(per)) * w.B
+
+
+class PrefillWorkload:
+    """A causal prefill of an n-token prompt through every layer of a workload's head layout:
+    per layer rtp_append_kv of the prompt into that layer's caches, then rtp_prefill (the
+    RoPE'd-key pre-pass and the attention). One prompt (the layer-0 streams: q_pre from the
+    prompt-query streams at scale 2, k_pre and v from the fill kernel) feeds every layer."""
+
+    def __init__(self, w, n, dev):
+        import torch
+        from long_context_sparse_rtpurbo_b200 import rtp
+        from long_context_sparse_rtpurbo_b200.layer import DecodeLayer
+        from synth.gpu import LayerFiller
+        self.w, self.n, self.dev = w, n, dev
+        t0 = time.perf_counter()
+        B, Hq, Hkv = w.B, w.Hq, w.Hkv
+        qb = np.zeros((B, n, Hq, 128), np.uint16)
+        for b in range(B):
+            for h in range(Hq):
+                qb[b, :, h] = w.prompt_q_bits(0, b, h, 0, n, 2.0)
+        self.q = _bits_to_dev(qb, dev)
+        del qb
+        self.k, self.v = LayerFiller(w, 0, dev).fill(np.zeros(B, np.int64), n)
+        self.out = torch.empty((B, n, Hq, 128), dtype=torch.bfloat16, device=dev)
+        self.nb = torch.full((B,), n, dtype=torch.int32, device=dev)
+        self.start = torch.zeros(B, dtype=torch.int32, device=dev)
+        caps = np.full(B, n, np.int64)
+        self.layers = []
+        for l in range(w.layers):
+            lay = DecodeLayer(B, Hq, Hkv, w.sinks, w.window, n, w.ret_mask[l], caps, dev,
+                              w.rope_base)
+            wk = torch.from_numpy(np.array(w.w_kidx(l), np.float32)).to(dev)
+            self.layers.append((lay, wk))
+        need = rtp.rtp_prefill_workspace_bytes(self.layers[0][0].desc, n)
+        self.ws = torch.empty(need, dtype=torch.uint8, device=dev)
+        torch.cuda.synchronize()
+        self.setup_s = time.perf_counter() - t0
+
+    def step(self, attention_only=False):
+        from long_context_sparse_rtpurbo_b200 import rtp
+        for lay, wk in self.layers:
+            if not attention_only:
+                rtp.rtp_append_kv(lay.desc, lay.cache, self.k, self.v, wk, self.start, self.nb,
+                                  self.n, lay.ws)
+            rtp.rtp_prefill(lay.desc, self.q, self.k, self.v, self.nb, self.n, self.out,
+                            self.ws, self.ws.numel())
+
+    def measure(self, args, world):
+        import torch
+        from long_context_sparse_rtpurbo_b200 import rtp
+        w, n, dev = self.w, self.n, self.dev
+        self.step()
+        per_step_launches = 0
+        for lay, wk in self.layers:
+            rtp.rtp_append_kv(lay.desc, lay.cache, self.k, self.v, wk, self.start, self.nb, n,
+                              lay.ws)
+            per_step_launches += rtp.rtp_last_launch_count()
+            rtp.rtp_prefill(lay.desc, self.q, self.k, self.v, self.nb, n, self.out, self.ws,
+                            self.ws.numel())
+            per_step_launches += rtp.rtp_last_launch_count()
+        torch.cuda.synchronize()
+        assert rtp.rtp_read_device_status(self.ws) == 0
+
+        def timed(fn, k):
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            torch.cuda.synchronize()
+            if world > 1:
+                torch.distributed.barrier()
+            torch.cuda.synchronize()
+            e0.record()
+            for _ in range(k):
+                fn()
+            e1.record()
+            torch.cuda.synchronize()
+            if world > 1:
+                torch.distributed.barrier()
+            return e0.elapsed_time(e1)
+
+        for _ in range(max(3, args.warmup)):
+            self.step()
+        steps = max(1, args.prefill_steps)
+        local = dev.index if dev.index is not None else 0
+        with ClockSampler(local) as clk:
+            ms = timed(self.step, steps) / steps
+            attn_ms = timed(lambda: self.step(True), steps) / steps
+        ms = max_over_ranks(ms, world, dev)
+        attn_ms = max_over_ranks(attn_ms, world, dev)
+        flops = prefill_flops(w, n)
+        peak, peak_kind = load_tensor_peak()
+        achieved = flops / (attn_ms * 1e-3) / 1e12
+        tokens = float(n * w.B)
+        return {
+            "metric": "prefill tokens/s", "value": tokens * world / (ms * 1e-3),
+            "unit": "tokens/s", "ms_per_step": ms, "higher_is_better": True,
+            "config": {"workload": f"qwen3-8b-prefill-{n // 1024}k-b{w.B}", "layers": w.layers,
+                       "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "head_dim": 128, "prompt": n,
+                       "sinks": w.sinks, "window": w.window,
+                       "retrieval_pairs": int(w.ret_mask.sum()),
+                       "step": "per layer: rtp_append_kv of the prompt, then rtp_prefill",
+                       "flush": "inputs larger than L2 (%.0f MB of q / k / v / out per layer)"
+                                % ((self.q.numel() + self.k.numel() + self.v.numel() +
+                                    self.out.numel()) * 2 / 1e6)},
+            "attention_ms_per_step": attn_ms,
+            "roofline": {"kernel": "rtp_prefill", "bound": "tensor", "achieved": achieved,
+                         "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
+                         "peak_kind": peak_kind, "traffic": None,
+                         "flops_per_step": flops,
+                         "note": "algorithmic FLOPs (4 * 128 per attended query-key pair) over "
+                                 "the time of rtp_prefill (RoPE'd-key pre-pass + attention); "
+                                 "the kernel issues twice as many tensor-core FLOPs (query and "
+                                 "probabilities as two bf16 terms each)"},
+            "gpu_launches": per_step_launches * steps,
+            "clocks": clk.summary(),
+            "setup_s": self.setup_s,
+        }
+
+    def close(self):
+        import torch
+        del self.layers, self.q, self.k, self.v, self.out, self.ws
+        torch.cuda.empty_cache()
+
+
+def oracle_prefill_sample(w, n, n_sample=2048):
+    """The CPU oracle on a bounded sample of the prefill: prefill_head of one retrieval and
+    one local query head over the first n_sample prompt tokens, scaled to a whole n-token,
+    36-layer step by the algorithmic FLOPs of each head kind."""
+    from oracle import rtp_oracle as O
+    from synth import gen
+    l_ret = int(np.nonzero(w.ret_mask.any(axis=1))[0][0])
+    g_ret = int(np.nonzero(w.ret_mask[l_ret])[0][0])
+    g_loc = int(np.nonzero(~w.ret_mask[l_ret])[0][0])
+    f64 = lambda bits: gen.bf16_bits_to_f32(bits).astype(np.float64)
+    spent = {}
+    for kind, g in (("retrieval", g_ret), ("local", g_loc)):
+        q = f64(w.prompt_q_bits(0, 0, g * w.G, 0, n_sample, 2.0))
+        k = f64(w.kpre_bits(0, 0, g, 0, n_sample))
+        v = f64(w.v_bits(0, 0, g, 0, n_sample))
+        t0 = time.perf_counter()
+        O.prefill_head(q, k, v, kind == "local", w.sinks, w.window, w.rope_base)
+        spent[kind] = time.perf_counter() - t0
+    m_s = np.arange(n_sample, dtype=np.float64)
+    m_f = np.arange(n, dtype=np.float64)
+    cap = w.sinks + w.window
+    scale = {"retrieval": (m_f + 1).sum() / (m_s + 1).sum(),
+             "local": np.minimum(m_f + 1, cap).sum() / np.minimum(m_s + 1, cap).sum()}
+    n_ret = int(w.ret_mask.sum()) * w.G * w.B
+    n_loc = int((~w.ret_mask).sum()) * w.G * w.B
+    step_s = (n_ret * spent["retrieval"] * scale["retrieval"] +
+              n_loc * spent["local"] * scale["local"])
+    return {"value": float(n * w.B / step_s), "unit": "tokens/s", "cores": cpu_threads(),
+            "kind": "oracle",
+            "sample": f"prefill_head of one retrieval and one local query head over the first "
+                      f"{n_sample} prompt tokens ({spent['retrieval'] + spent['local']:.2f} s of "
+                      f"float64 NumPy), scaled to {n_ret} retrieval + {n_loc} local query heads "
+                      f"of a {n}-token step by each kind's algorithmic FLOPs"}
+
+
 def _cpu_baseline(w, budget_s):
     """The oracle on the host cores: whole layer-steps (alternating a layer with retrieval
     heads and one without) up to budget_s seconds, or, for contexts beyond 64K tokens, the
@@ -683,6 +862,17 @@ def run_ours(args, w):
             extra[f"{we.name}@topk={args.topk}"] = gw.measure(we.p, args, world, topk=args.topk)
         gw.close()
         del gw
+    if args.prefill > 0:                       # the causal prefill of a prompt (f1)
+        wp = workloads.workload(2)
+        if args.layers:
+            wp.layers = min(wp.layers, args.layers)
+        pw = PrefillWorkload(wp, args.prefill, dev)
+        me = pw.measure(args, world)
+        pw.close()
+        del pw
+        if rank == 0 and world == 1 and not args.no_cpu:
+            me["cpu_baseline"] = oracle_prefill_sample(wp, args.prefill)
+        extra[me["config"]["workload"]] = me
     if extra:
         line["extra"] = extra
     if rank == 0 and world == 1 and not args.no_cpu:
@@ -720,6 +910,10 @@ def main(argv=None):
     ap.add_argument("--topk", type=int, default=2048,
                     help="k of the fixed-budget top-k variant measured on the 32K workload "
                          "(0: skip)")
+    ap.add_argument("--prefill", type=int, default=32768,
+                    help="prompt length of the prefill measured under 'extra' (0: skip)")
+    ap.add_argument("--prefill-steps", type=int, default=3,
+                    help="timed 36-layer prefill steps")
     ap.add_argument("--p", type=float, default=None)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--cpu-budget", type=float, default=12.0)

@@ -5,17 +5,19 @@
 // prefill_rope_keys: the prompt's keys rotated by R(j) with the append's arithmetic (double
 // angles and rotation, one rounding to bf16), so they equal the cache rows the append writes;
 // local heads need them because their ring keeps only the last window.
-// prefill_kernel: one CTA of 4 warps per (128 query rows, query head, sequence), two CTAs per
-// SM; thread t owns query row t. Over the 64-key tiles the rows can see (causal; local heads
-// skip the tiles between the sinks and the window), with K and V tiles staged by cp.async in
-// the 128-byte-swizzled operand layout:
+// prefill_kernel: one CTA of 8 warps per (128 query rows, query head, sequence), two CTAs per
+// SM; thread t owns query row t % 128 (its tensor-memory lane) and half t / 128 of the row's
+// keys in the softmax and of its output dims. Over the 64-key tiles the rows can see (causal;
+// local heads skip the tiles between the sinks and the window), with K and V tiles staged by
+// cp.async in the 128-byte-swizzled operand layout:
 //   S = Q K^T on the fifth-generation tensor cores (tcgen05.mma, 128 x 64, fp32 in tensor
 //   memory), the query as two bf16 terms (the rounded value and its rounded remainder) so the
 //   logits keep fp32-level accuracy;
-//   masked online softmax in the log2 domain (the query carries log2(e) / sqrt(128)), the
+//   online softmax in the log2 domain (the query carries log2(e) / sqrt(128)), keys checked
+//   one by one only where a tile crosses the row's diagonal, window edge or prompt end; the
 //   probabilities written back to tensor memory as two bf16 terms;
-//   the tile's P V from tensor memory (TS form, 128 x 128), added to the thread's fp32 output
-//   row in registers after the running-maximum rescale.
+//   the tile's P V from tensor memory (TS form, 128 x 128), added to the thread's 64 fp32
+//   output dims in registers after the running-maximum rescale.
 // The next K tile loads while the softmax runs, the next V tile while the next S is computed.
 #pragma once
 
@@ -26,7 +28,8 @@
 
 namespace rtp {
 
-constexpr int kPfThreads = 128;      // 4 warps: thread t owns query row t (tensor-memory lane t)
+constexpr int kPfThreads = 256;      // 8 warps: thread t owns row t % 128 (tensor-memory lane),
+                                     // the columns and output dims of half t / 128
 constexpr int kPfQ = 128;            // query rows per CTA (the MMA's M)
 constexpr int kPfK = 64;             // keys per tile
 constexpr uint32_t kPfQBlock = kPfQ * 128;                // one 64-dim block of the query tile
@@ -34,7 +37,8 @@ constexpr uint32_t kPfBlock = kPfK * 128;                 // one 64-dim block of
 constexpr uint32_t kPfQHi = 0, kPfQLo = 2 * kPfQBlock;    // query terms: 2 blocks each
 constexpr uint32_t kPfKt = 4 * kPfQBlock, kPfVt = kPfKt + 2 * kPfBlock;
 constexpr uint32_t kPfBar = kPfVt + 2 * kPfBlock;         // two mbarriers, the tensor-memory word
-constexpr int kPfSmem = (int)kPfBar + 64 + 1024;          // + slack to align the base to 1024
+constexpr uint32_t kPfLsum = kPfBar + 64;                 // [2][128] row-sum halves
+constexpr int kPfSmem = (int)kPfLsum + 1024 + 1024;       // + slack to align the base to 1024
 constexpr uint32_t kPfTmemCols = 256;  // S, then P hi / lo, in [0, 64); the PV tile in [128, 256)
 constexpr uint32_t kPfColO = 128;
 
@@ -174,15 +178,15 @@ __global__ void __launch_bounds__(kPfThreads, 2) prefill_kernel(PrefillParams P)
   __syncthreads();
   tmem_fence_after_sync();
   const uint32_t tm = *reinterpret_cast<volatile uint32_t*>(sm + kPfBar + 16);
-  const uint32_t tl = tm + ((uint32_t)(warp * 32) << 16);     // this thread's lane (row t)
+  const uint32_t tl = tm + ((uint32_t)((warp & 3) * 32) << 16);   // this thread's lane (row)
   constexpr uint32_t idS = umma_idesc_bf16(kPfQ, kPfK, 0);   // S = Q K^T: 128 x 64, K-major B
   constexpr uint32_t idO = umma_idesc_bf16(kPfQ, kD, 1);     // O = P V: 128 x 128, MN-major B
 
-  float o[kD];
+  float o[kD / 2];                                          // output dims 64 hf .. 64 hf + 63
 #pragma unroll
-  for (int d = 0; d < kD; ++d) o[d] = 0.f;
+  for (int d = 0; d < kD / 2; ++d) o[d] = 0.f;
   float m_run = -INFINITY, l_run = 0.f;
-  const int row = q0 + t;
+  const int row = q0 + (t & (kPfQ - 1)), hf = t >> 7;
   int j = 0, pend = 0;                                      // pend: 1 S, 2 PV in flight at an abort
 #pragma unroll 1
   while (kt >= 0) {
@@ -208,22 +212,32 @@ __global__ void __launch_bounds__(kPfThreads, 2) prefill_kernel(PrefillParams P)
     tmem_fence_after_sync();
     if (kn >= 0) pf_load_tile(sK, kbase, kD, kn, nb);       // the K buffer is free again
     cp_async_commit();
-    // masked online softmax of row `row` over the tile's 64 keys, 32 columns at a time: the
-    // maximum first, then the probabilities, each half's two bf16 terms written over its own
-    // scores (hi, then lo: columns 32 half + [0, 16) and + [16, 32))
-    const int k0 = kt * kPfK;
+    // online softmax of row `row`: the maximum over the tile's 64 keys (both halves of the
+    // row read it whole), then the probabilities of this thread's 32 keys, 16 at a time, each
+    // 16-key group's two bf16 terms written over its own scores (hi in the first 8 columns,
+    // lo in the next 8). Keys are checked one by one only in a tile this row does not see whole
+    // (the diagonal, the window's edge, the prompt's end); the tensor-memory accesses stay
+    // outside the per-row branch (they are warp-wide).
+    const int k0 = kt * kPfK, k1 = k0 + kPfK - 1;
     const int lo_ok = local ? row - L.window : -1;          // local: keys > lo_ok or < sinks
+    const bool whole = k1 <= row && k1 < nb && (k0 > lo_ok || k1 < L.sinks);
     float mx = -INFINITY;
 #pragma unroll
-    for (int half = 0; half < 2; ++half) {
+    for (int h2 = 0; h2 < 2; ++h2) {
       uint32_t sr[32];
-      tmem_ld32(tl + 32 * half, sr);
+      __syncwarp();
+      tmem_ld32(tl + 32 * h2, sr);
       tmem_wait_ld();
+      if (whole) {
 #pragma unroll
-      for (int i = 0; i < 32; ++i) {
-        const int key = k0 + 32 * half + i;
-        const bool ok = key <= row && key < nb && (key > lo_ok || key < L.sinks);
-        mx = ok ? fmaxf(mx, __uint_as_float(sr[i])) : mx;
+        for (int i = 0; i < 32; ++i) mx = fmaxf(mx, __uint_as_float(sr[i]));
+      } else {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          const int key = k0 + 32 * h2 + i;
+          const bool ok = key <= row && key < nb && (key > lo_ok || key < L.sinks);
+          mx = ok ? fmaxf(mx, __uint_as_float(sr[i])) : mx;
+        }
       }
     }
     const float mn = fmaxf(m_run, mx);
@@ -231,24 +245,38 @@ __global__ void __launch_bounds__(kPfThreads, 2) prefill_kernel(PrefillParams P)
     m_run = mn;
     float lsum = 0.f;
 #pragma unroll
-    for (int half = 0; half < 2; ++half) {
-      uint32_t sr[32], ph[16], pl[16];
-      tmem_ld32(tl + 32 * half, sr);
+    for (int q = 0; q < 2; ++q) {
+      const uint32_t col = 32 * hf + 16 * q;                // this 16-key group's columns
+      uint32_t sr[16], ph[8], pl[8];
+      __syncwarp();
+      tmem_ld16(tl + col, sr);
       tmem_wait_ld();
+      if (whole) {
 #pragma unroll
-      for (int c = 0; c < 16; ++c) {
-        const int key = k0 + 32 * half + 2 * c;
-        const bool ok0 = key <= row && key < nb && (key > lo_ok || key < L.sinks);
-        const bool ok1 = key + 1 <= row && key + 1 < nb && (key + 1 > lo_ok || key + 1 < L.sinks);
-        const float p0 = ok0 ? pf_ex2(__uint_as_float(sr[2 * c]) - mn) : 0.f;
-        const float p1 = ok1 ? pf_ex2(__uint_as_float(sr[2 * c + 1]) - mn) : 0.f;
-        lsum += p0 + p1;
-        split_bf2(p0, p1, ph[c], pl[c]);
+        for (int c = 0; c < 8; ++c) {
+          const float p0 = pf_ex2(__uint_as_float(sr[2 * c]) - mn);
+          const float p1 = pf_ex2(__uint_as_float(sr[2 * c + 1]) - mn);
+          lsum += p0 + p1;
+          split_bf2(p0, p1, ph[c], pl[c]);
+        }
+      } else {
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+          const int key = k0 + (int)col + 2 * c;
+          const bool ok0 = key <= row && key < nb && (key > lo_ok || key < L.sinks);
+          const bool ok1 = key + 1 <= row && key + 1 < nb && (key + 1 > lo_ok || key + 1 < L.sinks);
+          const float p0 = ok0 ? pf_ex2(__uint_as_float(sr[2 * c]) - mn) : 0.f;
+          const float p1 = ok1 ? pf_ex2(__uint_as_float(sr[2 * c + 1]) - mn) : 0.f;
+          lsum += p0 + p1;
+          split_bf2(p0, p1, ph[c], pl[c]);
+        }
       }
-      tmem_st16(tl + 32 * half, ph);
-      tmem_st16(tl + 32 * half + 16, pl);
+      __syncwarp();
+      tmem_st8(tl + col, ph);
+      tmem_st8(tl + col + 8, pl);
     }
     l_run = l_run * alpha + lsum;
+    __syncwarp();
     tmem_wait_st();
     cp_async_wait<1>();                                     // V tile kt landed
     fence_async_smem();
@@ -259,9 +287,9 @@ __global__ void __launch_bounds__(kPfThreads, 2) prefill_kernel(PrefillParams P)
 #pragma unroll
       for (int ks = 0; ks < kPfK / 16; ++ks) {
         const uint64_t bv = umma_desc_sw128(sV + (uint32_t)ks * 2048, kPfBlock, 1024);
-        const uint32_t pa = tm + 32 * (ks >> 1) + 8 * (ks & 1);   // P hi of keys 16 ks..
+        const uint32_t pa = tm + 16 * ks;                   // P hi of keys 16 ks .. 16 ks + 15
         umma_ts(tm + kPfColO, pa, bv, idO, ks > 0);
-        umma_ts(tm + kPfColO, pa + 16, bv, idO, 1);                // P lo
+        umma_ts(tm + kPfColO, pa + 8, bv, idO, 1);          // P lo
       }
       umma_commit(barO);
     }
@@ -271,9 +299,10 @@ __global__ void __launch_bounds__(kPfThreads, 2) prefill_kernel(PrefillParams P)
     if (kn >= 0) pf_load_tile(sV, vbase, vstride, kn, nb);  // the V buffer is free again
     cp_async_commit();
 #pragma unroll
-    for (int c = 0; c < kD / 32; ++c) {
+    for (int c = 0; c < 2; ++c) {
       uint32_t r[32];
-      tmem_ld32(tl + kPfColO + 32 * c, r);
+      __syncwarp();
+      tmem_ld32(tl + kPfColO + 64 * hf + 32 * c, r);
       tmem_wait_ld();
 #pragma unroll
       for (int i = 0; i < 32; ++i) o[32 * c + i] = fmaf(o[32 * c + i], alpha, __uint_as_float(r[i]));
@@ -286,11 +315,17 @@ __global__ void __launch_bounds__(kPfThreads, 2) prefill_kernel(PrefillParams P)
     // freed, and leave this CTA's rows unwritten
     if (t == 0) set_status(P.status, -5);
     mbar_wait(pend == 1 ? barS : barO, j & 1, 2000000000LL);
-  } else if (row <= q1) {
-    uint16_t* dst = P.out + (((int64_t)b * P.n_max + row) * L.Hq + h) * kD;
-    const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
+  }
+  // the row sum: this thread's half plus the other half's
+  float* lsh = reinterpret_cast<float*>(sm + kPfLsum);
+  lsh[t] = l_run;
+  __syncthreads();
+  if (!pend && row <= q1) {
+    const float l_all = lsh[t & (kPfQ - 1)] + lsh[kPfQ + (t & (kPfQ - 1))];
+    uint16_t* dst = P.out + (((int64_t)b * P.n_max + row) * L.Hq + h) * kD + 64 * hf;
+    const float inv = l_all > 0.f ? 1.f / l_all : 0.f;
 #pragma unroll
-    for (int c = 0; c < kD / 8; ++c) {
+    for (int c = 0; c < kD / 16; ++c) {
       uint4 w;
       w.x = pack_bf2(o[8 * c] * inv, o[8 * c + 1] * inv);
       w.y = pack_bf2(o[8 * c + 2] * inv, o[8 * c + 3] * inv);
