@@ -41,6 +41,7 @@ constexpr uint32_t kPfLsum = kPfBar + 64;                 // [2][128] row-sum ha
 constexpr int kPfSmem = (int)kPfLsum + 1024 + 1024;       // + slack to align the base to 1024
 constexpr uint32_t kPfTmemCols = 256;  // S, then P hi / lo, in [0, 64); the PV tile in [128, 256)
 constexpr uint32_t kPfColO = 128;
+constexpr float kPfSlack = 8.f;      // log2 units the softmax reference may lag a row's maximum
 
 __global__ void __launch_bounds__(128)
 prefill_rope_keys(LayerShape L, const uint16_t* __restrict__ k_pre, const int32_t* __restrict__ n_b,
@@ -182,11 +183,13 @@ __global__ void __launch_bounds__(kPfThreads, 2) prefill_kernel(PrefillParams P)
   constexpr uint32_t idS = umma_idesc_bf16(kPfQ, kPfK, 0);   // S = Q K^T: 128 x 64, K-major B
   constexpr uint32_t idO = umma_idesc_bf16(kPfQ, kD, 1);     // O = P V: 128 x 128, MN-major B
 
-  float o[kD / 2];                                          // output dims 64 hf .. 64 hf + 63
-#pragma unroll
-  for (int d = 0; d < kD / 2; ++d) o[d] = 0.f;
-  float m_run = -INFINITY, l_run = 0.f;
+  // The output accumulates in tensor memory across tiles (the PV MMAs add into it). The
+  // softmax reference m_ref of a row moves only when a tile's maximum exceeds it by more than
+  // kPfSlack (log2 units): then the row's accumulated output and sum are scaled by
+  // 2^(m_ref - m_new) in place; otherwise the probabilities 2^(s - m_ref) stay below 2^kPfSlack.
+  float m_ref = -INFINITY, l_run = 0.f;
   const int row = q0 + (t & (kPfQ - 1)), hf = t >> 7;
+  const uint32_t to = tl + kPfColO + 64 * hf;               // this thread's 64 output columns
   int j = 0, pend = 0;                                      // pend: 1 S, 2 PV in flight at an abort
 #pragma unroll 1
   while (kt >= 0) {
@@ -212,70 +215,102 @@ __global__ void __launch_bounds__(kPfThreads, 2) prefill_kernel(PrefillParams P)
     tmem_fence_after_sync();
     if (kn >= 0) pf_load_tile(sK, kbase, kD, kn, nb);       // the K buffer is free again
     cp_async_commit();
-    // online softmax of row `row`: the maximum over the tile's 64 keys (both halves of the
-    // row read it whole), then the probabilities of this thread's 32 keys, 16 at a time, each
-    // 16-key group's two bf16 terms written over its own scores (hi in the first 8 columns,
-    // lo in the next 8). Keys are checked one by one only in a tile this row does not see whole
-    // (the diagonal, the window's edge, the prompt's end); the tensor-memory accesses stay
-    // outside the per-row branch (they are warp-wide).
+    // softmax of row `row`: the maximum over the tile's 64 keys (both halves of the row read it
+    // whole), then the probabilities of this thread's 32 keys, each 16-key group's two bf16
+    // terms written over its own scores (hi in the first 8 columns, lo in the next 8). Keys are
+    // checked one by one only in a tile this row does not see whole (the diagonal, the window's
+    // edge, the prompt's end); tensor-memory accesses stay outside per-row branches (they are
+    // warp-wide).
     const int k0 = kt * kPfK, k1 = k0 + kPfK - 1;
     const int lo_ok = local ? row - L.window : -1;          // local: keys > lo_ok or < sinks
     const bool whole = k1 <= row && k1 < nb && (k0 > lo_ok || k1 < L.sinks);
     float mx = -INFINITY;
-#pragma unroll
-    for (int h2 = 0; h2 < 2; ++h2) {
-      uint32_t sr[32];
+    {
+      uint32_t sr[64];
       __syncwarp();
-      tmem_ld32(tl + 32 * h2, sr);
+      tmem_ld32(tl, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
+      tmem_ld32(tl + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
       tmem_wait_ld();
       if (whole) {
 #pragma unroll
-        for (int i = 0; i < 32; ++i) mx = fmaxf(mx, __uint_as_float(sr[i]));
+        for (int i = 0; i < 64; ++i) mx = fmaxf(mx, __uint_as_float(sr[i]));
       } else {
 #pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          const int key = k0 + 32 * h2 + i;
+        for (int i = 0; i < 64; ++i) {
+          const int key = k0 + i;
           const bool ok = key <= row && key < nb && (key > lo_ok || key < L.sinks);
           mx = ok ? fmaxf(mx, __uint_as_float(sr[i])) : mx;
         }
       }
     }
-    const float mn = fmaxf(m_run, mx);
-    const float alpha = mn == -INFINITY ? 1.f : pf_ex2(m_run - mn);
-    m_run = mn;
-    float lsum = 0.f;
+    // the row's other half (warp w ^ 4) reads these columns for its maximum too: both halves
+    // finish reading before either writes its probabilities over them
+    tmem_fence_before_sync();
+    switch (warp & 3) {                                     // named barrier of the warp pair
+      case 0: asm volatile("bar.sync 1, 64;" ::: "memory"); break;
+      case 1: asm volatile("bar.sync 2, 64;" ::: "memory"); break;
+      case 2: asm volatile("bar.sync 3, 64;" ::: "memory"); break;
+      default: asm volatile("bar.sync 4, 64;" ::: "memory"); break;
+    }
+    tmem_fence_after_sync();
+    const bool move = mx > m_ref + kPfSlack;                // also the first visible key
+    const float m_new = move ? mx : m_ref;
+    const float alpha = move ? pf_ex2(m_ref - m_new) : 1.f; // 0 while nothing was seen
+    m_ref = m_new;
+    l_run *= alpha;
+    if (j > 0 && __any_sync(0xffffffffu, move)) {          // scale the accumulated output
 #pragma unroll
-    for (int q = 0; q < 2; ++q) {
-      const uint32_t col = 32 * hf + 16 * q;                // this 16-key group's columns
-      uint32_t sr[16], ph[8], pl[8];
+      for (int c = 0; c < 2; ++c) {
+        uint32_t r[32];
+        __syncwarp();
+        tmem_ld32(to + 32 * c, r);
+        tmem_wait_ld();
+#pragma unroll
+        for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
+        __syncwarp();
+        tmem_st32(to + 32 * c, r);
+      }
+    }
+    {
+      const uint32_t col = 32 * hf;                         // this thread's 32 keys
+      uint32_t sr[32], ph[16], pl[16];
       __syncwarp();
-      tmem_ld16(tl + col, sr);
+      tmem_ld32(tl + col, sr);
       tmem_wait_ld();
+      float lsum = 0.f;
       if (whole) {
 #pragma unroll
-        for (int c = 0; c < 8; ++c) {
-          const float p0 = pf_ex2(__uint_as_float(sr[2 * c]) - mn);
-          const float p1 = pf_ex2(__uint_as_float(sr[2 * c + 1]) - mn);
+        for (int c = 0; c < 16; ++c) {
+          const float p0 = pf_ex2(__uint_as_float(sr[2 * c]) - m_ref);
+          const float p1 = pf_ex2(__uint_as_float(sr[2 * c + 1]) - m_ref);
           lsum += p0 + p1;
           split_bf2(p0, p1, ph[c], pl[c]);
         }
       } else {
 #pragma unroll
-        for (int c = 0; c < 8; ++c) {
+        for (int c = 0; c < 16; ++c) {
           const int key = k0 + (int)col + 2 * c;
           const bool ok0 = key <= row && key < nb && (key > lo_ok || key < L.sinks);
           const bool ok1 = key + 1 <= row && key + 1 < nb && (key + 1 > lo_ok || key + 1 < L.sinks);
-          const float p0 = ok0 ? pf_ex2(__uint_as_float(sr[2 * c]) - mn) : 0.f;
-          const float p1 = ok1 ? pf_ex2(__uint_as_float(sr[2 * c + 1]) - mn) : 0.f;
+          const float p0 = ok0 ? pf_ex2(__uint_as_float(sr[2 * c]) - m_ref) : 0.f;
+          const float p1 = ok1 ? pf_ex2(__uint_as_float(sr[2 * c + 1]) - m_ref) : 0.f;
           lsum += p0 + p1;
           split_bf2(p0, p1, ph[c], pl[c]);
         }
       }
+      l_run += lsum;
+      // groups g = 0, 1 of 16 keys: hi in columns col + 16 g + [0, 8), lo in + [8, 16)
+      uint32_t a[8], b[8];
+#pragma unroll
+      for (int c = 0; c < 8; ++c) { a[c] = ph[c]; b[c] = pl[c]; }
       __syncwarp();
-      tmem_st8(tl + col, ph);
-      tmem_st8(tl + col + 8, pl);
+      tmem_st8(tl + col, a);
+      tmem_st8(tl + col + 8, b);
+#pragma unroll
+      for (int c = 0; c < 8; ++c) { a[c] = ph[8 + c]; b[c] = pl[8 + c]; }
+      tmem_st8(tl + col + 16, a);
+      tmem_st8(tl + col + 24, b);
     }
-    l_run = l_run * alpha + lsum;
     __syncwarp();
     tmem_wait_st();
     cp_async_wait<1>();                                     // V tile kt landed
@@ -288,7 +323,7 @@ __global__ void __launch_bounds__(kPfThreads, 2) prefill_kernel(PrefillParams P)
       for (int ks = 0; ks < kPfK / 16; ++ks) {
         const uint64_t bv = umma_desc_sw128(sV + (uint32_t)ks * 2048, kPfBlock, 1024);
         const uint32_t pa = tm + 16 * ks;                   // P hi of keys 16 ks .. 16 ks + 15
-        umma_ts(tm + kPfColO, pa, bv, idO, ks > 0);
+        umma_ts(tm + kPfColO, pa, bv, idO, j > 0 || ks > 0);
         umma_ts(tm + kPfColO, pa + 8, bv, idO, 1);          // P lo
       }
       umma_commit(barO);
@@ -298,15 +333,6 @@ __global__ void __launch_bounds__(kPfThreads, 2) prefill_kernel(PrefillParams P)
     tmem_fence_after_sync();
     if (kn >= 0) pf_load_tile(sV, vbase, vstride, kn, nb);  // the V buffer is free again
     cp_async_commit();
-#pragma unroll
-    for (int c = 0; c < 2; ++c) {
-      uint32_t r[32];
-      __syncwarp();
-      tmem_ld32(tl + kPfColO + 64 * hf + 32 * c, r);
-      tmem_wait_ld();
-#pragma unroll
-      for (int i = 0; i < 32; ++i) o[32 * c + i] = fmaf(o[32 * c + i], alpha, __uint_as_float(r[i]));
-    }
     kt = kn;
     ++j;
   }
@@ -320,18 +346,25 @@ __global__ void __launch_bounds__(kPfThreads, 2) prefill_kernel(PrefillParams P)
   float* lsh = reinterpret_cast<float*>(sm + kPfLsum);
   lsh[t] = l_run;
   __syncthreads();
-  if (!pend && row <= q1) {
-    const float l_all = lsh[t & (kPfQ - 1)] + lsh[kPfQ + (t & (kPfQ - 1))];
-    uint16_t* dst = P.out + (((int64_t)b * P.n_max + row) * L.Hq + h) * kD + 64 * hf;
-    const float inv = l_all > 0.f ? 1.f / l_all : 0.f;
+  if (!pend) {
+    uint32_t r[64];
+    __syncwarp();
+    tmem_ld32(to, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
+    tmem_ld32(to + 32, *reinterpret_cast<uint32_t(*)[32]>(&r[32]));
+    tmem_wait_ld();
+    if (row <= q1) {
+      const float l_all = lsh[t & (kPfQ - 1)] + lsh[kPfQ + (t & (kPfQ - 1))];
+      uint16_t* dst = P.out + (((int64_t)b * P.n_max + row) * L.Hq + h) * kD + 64 * hf;
+      const float inv = l_all > 0.f ? 1.f / l_all : 0.f;
 #pragma unroll
-    for (int c = 0; c < kD / 16; ++c) {
-      uint4 w;
-      w.x = pack_bf2(o[8 * c] * inv, o[8 * c + 1] * inv);
-      w.y = pack_bf2(o[8 * c + 2] * inv, o[8 * c + 3] * inv);
-      w.z = pack_bf2(o[8 * c + 4] * inv, o[8 * c + 5] * inv);
-      w.w = pack_bf2(o[8 * c + 6] * inv, o[8 * c + 7] * inv);
-      *reinterpret_cast<uint4*>(dst + 8 * c) = w;
+      for (int c = 0; c < kD / 16; ++c) {
+        uint4 w;
+        w.x = pack_bf2(__uint_as_float(r[8 * c]) * inv, __uint_as_float(r[8 * c + 1]) * inv);
+        w.y = pack_bf2(__uint_as_float(r[8 * c + 2]) * inv, __uint_as_float(r[8 * c + 3]) * inv);
+        w.z = pack_bf2(__uint_as_float(r[8 * c + 4]) * inv, __uint_as_float(r[8 * c + 5]) * inv);
+        w.w = pack_bf2(__uint_as_float(r[8 * c + 6]) * inv, __uint_as_float(r[8 * c + 7]) * inv);
+        *reinterpret_cast<uint4*>(dst + 8 * c) = w;
+      }
     }
   }
   cp_async_wait<0>();
