@@ -741,7 +741,7 @@ class PrefillWorkload:
             "config": {"workload": f"qwen3-8b-prefill-{n // 1024}k-b{w.B}", "layers": w.layers,
                        "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "head_dim": 128, "prompt": n,
                        "sinks": w.sinks, "window": w.window,
-                       "retrieval_pairs": int(w.ret_mask.sum()),
+                       "retrieval_pairs": int(w.ret_mask[:w.layers].sum()),
                        "step": "per layer: rtp_append_kv of the prompt, then rtp_prefill",
                        "flush": "inputs larger than L2 (%.0f MB of q / k / v / out per layer)"
                                 % ((self.q.numel() + self.k.numel() + self.v.numel() +
@@ -789,8 +789,8 @@ def oracle_prefill_sample(w, n, n_sample=2048):
     cap = w.sinks + w.window
     scale = {"retrieval": (m_f + 1).sum() / (m_s + 1).sum(),
              "local": np.minimum(m_f + 1, cap).sum() / np.minimum(m_s + 1, cap).sum()}
-    n_ret = int(w.ret_mask.sum()) * w.G * w.B
-    n_loc = int((~w.ret_mask).sum()) * w.G * w.B
+    n_ret = int(w.ret_mask[:w.layers].sum()) * w.G * w.B
+    n_loc = int((~w.ret_mask[:w.layers]).sum()) * w.G * w.B
     step_s = (n_ret * spent["retrieval"] * scale["retrieval"] +
               n_loc * spent["local"] * scale["local"])
     return {"value": float(n * w.B / step_s), "unit": "tokens/s", "cores": cpu_threads(),
@@ -798,7 +798,7 @@ def oracle_prefill_sample(w, n, n_sample=2048):
             "sample": f"prefill_head of one retrieval and one local query head over the first "
                       f"{n_sample} prompt tokens ({spent['retrieval'] + spent['local']:.2f} s of "
                       f"float64 NumPy), scaled to {n_ret} retrieval + {n_loc} local query heads "
-                      f"of a {n}-token step by each kind's algorithmic FLOPs"}
+                      f"of a {n}-token, {w.layers}-layer step by each kind's algorithmic FLOPs"}
 
 
 def _cpu_baseline(w, budget_s):
