@@ -245,7 +245,8 @@ int32_t rtp_last_launch_count(void);
  *     raises an abort flag that ends the launch's other waits; the outputs of that call are
  *     undefined and its workspace must be re-initialised with rtp_workspace_init. Process-wide.
  *   rtp_debug_fail_next_call: the next call of rtp_append_kv, rtp_decode_step,
- *     rtp_decode_step_append or rtp_decode_step_static (on any thread) returns `status` (one
+ *     rtp_decode_step_append, rtp_decode_step_topk, rtp_decode_step_static or rtp_prefill (on
+ *     any thread) returns `status` (one
  *     of the negative RTP_E* codes; 0 cancels) before checking its arguments, and enqueues
  *     nothing. Process-wide, consumed by that one call.
  */

@@ -179,3 +179,27 @@ def test_wait_limit_hook_validates():
     assert lib.rtp_debug_set_wait_limit(-1) == _lib.RTP_EINVAL
     assert lib.rtp_debug_set_wait_limit(5000) == _lib.RTP_OK
     assert lib.rtp_debug_set_wait_limit(0) == _lib.RTP_OK            # default restored
+
+
+def test_prefill_workspace_and_argument_checks():
+    """rtp_prefill_workspace_bytes: the status header plus the rotated keys [B][Hkv][n][128];
+    rtp_prefill rejects bad arguments before any device call (n_max = 0 does nothing)."""
+    d = _desc(max_seq_len=4096)
+    lib = _lib.load()
+    need = rtp.rtp_prefill_workspace_bytes(d, 1000)
+    assert need == 256 + 2 * 8 * 1000 * 256                         # B = 2, Hkv = 8
+    assert rtp.rtp_prefill_workspace_bytes(d, 0) == 0
+    assert rtp.rtp_prefill_workspace_bytes(d, 4097) == 0
+    assert rtp.rtp_prefill_workspace_bytes(_desc(Hq=30), 100) == 0
+    x = 0x1000
+    call = lambda q, n, ws, wsb: lib.rtp_prefill(d.ref, q, x, x, x, n, x, ws, wsb, None)
+    assert call(None, 1000, x, need) == _lib.RTP_EINVAL
+    assert call(x, -1, x, need) == _lib.RTP_EINVAL
+    assert call(x, 4097, x, 1 << 30) == _lib.RTP_ESHAPE
+    assert call(x, 0, None, 0) == _lib.RTP_OK                       # nothing to do
+    assert call(x, 1000, x, need - 1) == _lib.RTP_EWORKSPACE
+    assert call(x, 1000, None, need) == _lib.RTP_EWORKSPACE
+    assert call(x, 1000, x + 16, need) == _lib.RTP_EWORKSPACE       # not 256-byte aligned
+    rtp.rtp_debug_fail_next_call(_lib.RTP_ECUDA)
+    assert call(None, 1000, x, need) == _lib.RTP_ECUDA               # before the checks
+    assert call(None, 1000, x, need) == _lib.RTP_EINVAL
