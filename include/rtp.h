@@ -44,7 +44,10 @@ enum {
   RTP_EWORKSPACE = -3,  /* workspace missing or smaller than rtp_workspace_bytes() */
   RTP_ECUDA = -4,       /* a CUDA launch or API call failed */
   RTP_ETIMEOUT = -5,    /* a device-side wait gave up (status word only) */
-  RTP_EDEVICE = -6      /* the device found bad data, e.g. seq_lens[b] > seq_cap[b] */
+  RTP_EDEVICE = -6,     /* the device found bad data, e.g. seq_lens[b] > seq_cap[b] */
+  RTP_ECHECK = -7       /* builds with -DRTP_CHECKS only: a gathered row, ring row, list slot or
+                           debug-list index fell outside its buffer (status word only; the access
+                           was redirected to a valid row that contributes nothing) */
 };
 
 /* Per-layer description. Host struct; the library reads it during the call only. */

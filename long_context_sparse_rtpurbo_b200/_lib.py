@@ -8,8 +8,8 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 # RTP_LIBRARY_PATH selects another build of the same library (for example a tracing build)
 LIB_PATH = os.environ.get("RTP_LIBRARY_PATH") or os.path.join(_HERE, "librtp.so")
 
-RTP_OK, RTP_EINVAL, RTP_ESHAPE, RTP_EWORKSPACE, RTP_ECUDA, RTP_ETIMEOUT, RTP_EDEVICE = \
-    0, -1, -2, -3, -4, -5, -6
+RTP_OK, RTP_EINVAL, RTP_ESHAPE, RTP_EWORKSPACE, RTP_ECUDA, RTP_ETIMEOUT, RTP_EDEVICE, RTP_ECHECK = \
+    0, -1, -2, -3, -4, -5, -6, -7
 
 EXPORTS = (
     "rtp_status_str", "rtp_build_slot_map", "rtp_workspace_bytes", "rtp_workspace_init",

@@ -28,5 +28,12 @@ def build(verbose: bool = False, extra_flags=(), out_name: str = "librtp.so") ->
     return out
 
 
+def build_checks(verbose: bool = False) -> str:
+    """librtp_checks.so: the library with -DRTP_CHECKS (bounds checks of data-dependent indices
+    that record RTP_ECHECK instead of touching memory outside a buffer), for debugging runs
+    selected with RTP_LIBRARY_PATH."""
+    return build(verbose, ["-DRTP_CHECKS"], "librtp_checks.so")
+
+
 if __name__ == "__main__":
     print(build(verbose=True))

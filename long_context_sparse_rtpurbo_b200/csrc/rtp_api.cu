@@ -278,6 +278,7 @@ const char* rtp_status_str(int status) {
     case RTP_ECUDA: return "CUDA launch or API call failed";
     case RTP_ETIMEOUT: return "device-side wait timed out";
     case RTP_EDEVICE: return "device found bad data (sequence length or position outside capacity)";
+    case RTP_ECHECK: return "bounds check failed on the device (RTP_CHECKS build)";
     default: return "unknown status";
   }
 }

@@ -67,4 +67,14 @@ __device__ __forceinline__ void set_status(int* status, int code) {
   if (status) atomicCAS(status, 0, code);
 }
 
+// Bounds checks of data-dependent indices (the debug build that stands in for a memory checker,
+// compiled with -DRTP_CHECKS): true when `cond` holds; otherwise records RTP_ECHECK (-7) in the
+// status word and returns false, and the caller redirects the access to a valid location that
+// contributes nothing. Release builds compile every check to `true`.
+#ifdef RTP_CHECKS
+#define RTP_CHECK(cond, status) ((cond) ? true : (::rtp::set_status((status), -7), false))
+#else
+#define RTP_CHECK(cond, status) true
+#endif
+
 }  // namespace rtp

@@ -742,13 +742,17 @@ struct DecodeCta {
     int pre_off;                   // byte offset of pre[17] in rtp_smem
     int stride;                    // > 0: fixed per-warp stride; 0: WSel slots
     int N, nc, j, ntl;
+    int64_t cap;                   // entries the list holds
+    int* status;
     __device__ __forceinline__ void operator()(int i, const uint16_t*& kp, const uint16_t*& vp,
                                                uint32_t& mk) const {
       const int* pre = smem_at<int>(pre_off);
       const int w = upper_index(pre, kWarps, i);
       const int q = i - pre[w];
       const int at = stride > 0 ? w * stride + q : tile_row(N, nc, j, ntl, q / kWRows, w) + q % kWRows;
+      if (!RTP_CHECK(at >= 0 && at < cap, status)) { kp = kb; vp = vb; mk = 0u; return; }
       const uint32_t e = list[at];
+      if (!RTP_CHECK((int)(e >> 8) < N, status)) { kp = kb; vp = vb; mk = 0u; return; }
       kp = kb + (int64_t)(e >> 8) * kD;
       vp = vb + (int64_t)(e >> 8) * kD;
       mk = e & 0xffu;
@@ -757,8 +761,11 @@ struct DecodeCta {
   struct RangeRows {
     const uint16_t* kb;
     const uint16_t* vb;
+    int n;                         // rows in range
+    int* status;
     __device__ __forceinline__ void operator()(int i, const uint16_t*& kp, const uint16_t*& vp,
                                                uint32_t& mk) const {
+      if (!RTP_CHECK(i >= 0 && i < n, status)) { kp = kb; vp = vb; mk = 0u; return; }
       kp = kb + (int64_t)i * kD;
       vp = vb + (int64_t)i * kD;
       mk = 0xffu;
@@ -1066,7 +1073,8 @@ struct DecodeCta {
     if (tcol >= 0) {
       uint32_t* list = smem_at<uint32_t>(tail(kTailList));
       uint32_t* wl = list + warp * kWListCap;
-      const WarpListRows rows{list, kb, vb, P.sm_int + kIntPre * 4, kWListCap, N, S, j, ntl};
+      const WarpListRows rows{list, kb, vb, P.sm_int + kIntPre * 4, kWListCap, N, S, j, ntl,
+                              (int64_t)kWarps * kWListCap, P.status};
       trace(kEvW1);
       const uint32_t ta = chunk_taddr(tcol);
 #pragma unroll 1
@@ -1104,7 +1112,8 @@ struct DecodeCta {
       __threadfence_block();
       const int total = list_prefix(wsel.nw);
       trace(kEvWl);
-      const WarpListRows rows{gl, kb, vb, P.sm_int + kIntPre * 4, 0, N, S, j, ntl};
+      const WarpListRows rows{gl, kb, vb, P.sm_int + kIntPre * 4, 0, N, S, j, ntl,
+                              P.cand_stride, P.status};
       attn_tiles<G>(W, total, rows, sm.stage(), nwa, false);
     }
     attn_end<G>(W, nwa, sm.res(), reinterpret_cast<float*>(sm.stage()), kFThreads);
@@ -1161,7 +1170,7 @@ struct DecodeCta {
     const int nwa = min(kFThreads / 32, P.free_bytes / kTileBytes);
     const uint16_t* kb = P.cache.k_loc + ring0 * kD;
     const uint16_t* vb = P.cache.v_loc + ring0 * kD;
-    const RangeRows rowfn{kb, vb};
+    const RangeRows rowfn{kb, vb, nrows, P.status};
     attn_first_copy(nrows, rowfn, sm.stage(), nwa);
     rope_query<G>(P, b, kvh, N, sm.q());
     __syncthreads();
@@ -1296,7 +1305,8 @@ __global__ void __launch_bounds__(kFThreads) emit_sel_kernel(DecodeParams P, int
     const int s1 = min(N, P.L.sinks);
     const int w0 = max(P.L.sinks, N - P.L.window);
     const int cnt = s1 + max(0, N - w0);
-    for (int k = t; k < cnt; k += kFThreads) dst[k] = k < s1 ? k : w0 + (k - s1);
+    for (int k = t; k < cnt; k += kFThreads)
+      if (RTP_CHECK(k < sel_stride, P.status)) dst[k] = k < s1 ? k : w0 + (k - s1);
     return;
   }
   const int g = b * P.L.n_ret + slot;
@@ -1335,7 +1345,7 @@ __global__ void __launch_bounds__(kFThreads) emit_sel_kernel(DecodeParams P, int
     int before, total;
     block_flag_prefix(keep, wc + par * 16, before, total);
     par ^= 1;
-    if (keep) dst[base + before] = rb + lane;
+    if (keep && RTP_CHECK(base + before < sel_stride, P.status)) dst[base + before] = rb + lane;
     base += total;
     __syncwarp();                          // rows_s / keep_s are rewritten next round
   }
