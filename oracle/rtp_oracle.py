@@ -15,6 +15,11 @@ Sources, named by page and section:
   head) that fuses scoring and selection.
 * [GS] gist.science explainer of the same paper, "Dynamische Top-p-Auswahl": the selector
   accumulates attention mass in the low-dimensional space until the cumulative share p.
+* [V2] RTPurboV2 article, finding 3 ("adaptive clustering on high-quality features"): the N
+  tokens of a retrieval head are grouped into K semantic clusters in the low-rank space (K = 128
+  in the article), the query is first matched against the K centroids, and the full attention
+  runs only inside the hit clusters; the architecture summary pairs this clustering index with
+  the dynamic top-p of V1.
 
 Readings where the pages are silent (each is repeated where it is used):
 
@@ -354,6 +359,77 @@ def prefill_head(q_pre, k_pre, v, local: bool, sinks: int, window: int,
     z = np.where(allowed, z, -np.inf)
     w = np.exp(z - z.max(axis=1, keepdims=True))
     return (w @ v) / w.sum(axis=1, keepdims=True)
+
+
+# ----------------------------------------------------------- [V2] centroid pre-filter (f3)
+def kmeans_index_keys(kidx, K: int = 128, iters: int = 10):
+    """Lloyd's k-means of one retrieval KV head's stored index keys ([V2] finding 3: the tokens
+    grouped into K clusters in the 16-dim low-rank space, K = 128 in the article).
+
+    Readings: (R-f3a) the initial centroids are the keys at positions floor(i N / K), i < K
+    (deterministic, spread over the sequence); K > N is clamped to N. (R-f3b) an iteration
+    assigns every key to its nearest centroid in squared Euclidean distance (ties to the lower
+    cluster id), then moves every non-empty cluster's centroid to the mean of its keys (an empty
+    cluster keeps its centroid); at most `iters` iterations, fewer when an assignment repeats.
+
+    kidx: [N][r] (bf16 values as float64). Returns (centroids [K][r] float64, assign [N] int64).
+    """
+    x = np.asarray(kidx, np.float64)
+    N = x.shape[0]
+    K = min(K, N)
+    mu = x[(np.arange(K) * N) // K].copy()
+    assign = None
+    for _ in range(iters):
+        d = ((x[:, None, :] - mu[None, :, :]) ** 2).sum(axis=2)     # [N][K]
+        new = d.argmin(axis=1)                                        # first minimum: lower id
+        if assign is not None and np.array_equal(new, assign):
+            break
+        assign = new
+        for k in range(K):
+            members = assign == k
+            if members.any():
+                mu[k] = x[members].mean(axis=0)
+    return mu, assign
+
+
+def cluster_mass(q_idx, centroids, assign):
+    """Coarse match ([V2] finding 3, step 1): centroid scores c_k = q_idx . mu_k and the
+    estimated mass of each cluster, |C_k| exp(c_k - max c) (R-f3c: a cluster's members stand at
+    their centroid's score, with the token mass of R1). Returns (c [K], mass [K])."""
+    c = np.asarray(centroids, np.float64) @ np.asarray(q_idx, np.float64)
+    counts = np.bincount(np.asarray(assign), minlength=c.shape[0]).astype(np.float64)
+    return c, counts * np.exp(c - c.max())
+
+
+def cluster_select(q_idx, centroids, assign, p: float) -> np.ndarray:
+    """The hit clusters ([V2] finding 3 with the dynamic top-p of V1; R-f3d): clusters in
+    descending estimated mass (ties to the lower id), the smallest prefix whose mass reaches p
+    of the total; p >= 1 hits every non-empty cluster. Returns the bool mask of hit tokens."""
+    _, mass = cluster_mass(q_idx, centroids, assign)
+    K = mass.shape[0]
+    if p >= 1.0:
+        hit = mass > 0
+    else:
+        order = np.lexsort((np.arange(K), -mass))
+        cum = np.cumsum(mass[order])
+        n = int(np.searchsorted(cum, p * cum[-1], side="left")) + 1
+        hit = np.zeros(K, bool)
+        hit[order[:min(n, K)]] = True
+    return hit[np.asarray(assign)]
+
+
+def clustered_head(q_pre, w_qidx_h, k_pre, v, w_kidx_g, centroids, assign, p: float,
+                   base: float = 1e6) -> HeadResult:
+    """A retrieval query head at m = N - 1 through the centroid pre-filter ([V2] finding 3,
+    step 2; R-f3e): exact softmax attention (R9) over every token of the hit clusters."""
+    k_pre = np.asarray(k_pre, np.float64)
+    N = k_pre.shape[0]
+    mask = cluster_select(index_query(q_pre, w_qidx_h), centroids, assign, p)
+    idx = np.nonzero(mask)[0]
+    K = bf16_round(rope_rotate(k_pre[idx], idx, base))
+    out = attend(rope_rotate(q_pre, N - 1, base), K, np.asarray(v, np.float64)[idx])
+    s = index_scores(index_query(q_pre, w_qidx_h), index_keys(k_pre, w_kidx_g))
+    return HeadResult(out, int(idx.size), idx, None, s)
 
 
 def append_rows(k_pre, v, w_kidx_g, positions, base: float = 1e6):

@@ -569,3 +569,107 @@ def test_prefill_rows_equal_the_decode_step(local):
             ref = O.attend(O.rope_rotate(q[m], m), O.bf16_round(O.rope_rotate(k[: m + 1], pos)),
                            v[: m + 1])
         np.testing.assert_allclose(got[m], ref, rtol=1e-10, atol=1e-12)
+
+
+# ------------------------------------------------------------- centroid pre-filter (f3)
+def _blobs(rng, n_blobs, per, r=16, spread=0.05):
+    centres = rng.standard_normal((n_blobs, r)) * 3.0
+    x = np.concatenate([c + spread * rng.standard_normal((per, r)) for c in centres])
+    return x[rng.permutation(x.shape[0])]
+
+
+@pytest.mark.parametrize("seed", [0, 1, 2])
+def test_kmeans_matches_sklearn_lloyd_from_the_same_start(seed):
+    """The k-means of the index keys against scikit-learn's Lloyd k-means started from the same
+    centroids (positions floor(i N / K)), run to convergence: the same clusters and centroids."""
+    from sklearn.cluster import KMeans
+    rng = np.random.default_rng(seed)
+    x = rng.standard_normal((300, 16))
+    K = 12
+    mu, assign = O.kmeans_index_keys(x, K, iters=300)
+    init = x[(np.arange(K) * 300) // K]
+    km = KMeans(n_clusters=K, init=init, n_init=1, algorithm="lloyd", max_iter=300, tol=0.0)
+    km.fit(x)
+    assert np.array_equal(assign, km.labels_)
+    np.testing.assert_allclose(mu, km.cluster_centers_, rtol=1e-10, atol=1e-12)
+
+
+def test_kmeans_fixed_point_and_separated_blobs():
+    """At convergence every key sits in its nearest centroid's cluster and every centroid is
+    the mean of its keys. Runs of consecutive tokens drawn around separated centres (one run
+    per initial position floor(i N / K)) come out as exactly the runs."""
+    rng = np.random.default_rng(4)
+    x = _blobs(rng, 8, 40)
+    mu, assign = O.kmeans_index_keys(x, 8, iters=100)
+    d = ((x[:, None, :] - mu[None]) ** 2).sum(axis=2)
+    assert np.array_equal(d.argmin(axis=1), assign)
+    for k in range(8):
+        np.testing.assert_allclose(mu[k], x[assign == k].mean(axis=0), rtol=0, atol=1e-12)
+    centres = rng.standard_normal((8, 16)) * 3.0
+    runs = np.concatenate([c + 0.05 * rng.standard_normal((40, 16)) for c in centres])
+    mu, assign = O.kmeans_index_keys(runs, 8, iters=100)
+    assert np.array_equal(assign, np.arange(320) // 40)
+    np.testing.assert_allclose(mu, runs.reshape(8, 40, 16).mean(axis=1), rtol=0, atol=1e-12)
+
+
+def test_kmeans_clamps_k_and_keeps_empty_centroids():
+    x = np.arange(5 * 16, dtype=np.float64).reshape(5, 16)
+    mu, assign = O.kmeans_index_keys(x, 128, iters=5)
+    assert mu.shape == (5, 16) and np.array_equal(assign, np.arange(5))
+    # duplicated keys: the second initial centroid equals the first, loses every tie and keeps
+    # its position as an empty cluster
+    y = np.zeros((4, 16))
+    y[2:] = 1.0
+    mu, assign = O.kmeans_index_keys(y, 2, iters=5)      # starts at rows 0 and 2
+    assert np.array_equal(assign, [0, 0, 1, 1])
+    z = np.zeros((4, 16))
+    mu, assign = O.kmeans_index_keys(z, 2, iters=5)      # both starts at 0: ties to cluster 0
+    assert np.array_equal(assign, [0, 0, 0, 0]) and np.array_equal(mu, np.zeros((2, 16)))
+
+
+def test_cluster_select_with_one_token_per_cluster_is_exact_top_p():
+    """K = N (every token its own cluster, the centroid its key): the estimated masses are the
+    token masses exp(s - max s), so the hit set is the exact sorted top-p set."""
+    rng = np.random.default_rng(5)
+    for _ in range(20):
+        n = int(rng.integers(1, 60))
+        kidx = rng.standard_normal((n, 16))
+        q = rng.standard_normal(16) * rng.uniform(0.2, 3.0)
+        p = float(rng.uniform(0.05, 0.999))
+        got = O.cluster_select(q, kidx, np.arange(n), p)
+        assert np.array_equal(got, O.topp_exact(O.index_scores(q, kidx), p))
+
+
+def test_cluster_select_hand_worked_case():
+    """Two clusters: 3 tokens at centroid score 0 and 1 token at centroid score ln 2. Masses
+    3 * exp(-ln 2) = 1.5 and 1: the three-token cluster leads; p = 0.6 of 2.5 = 1.5 is reached
+    by it alone, p = 0.61 needs both."""
+    cent = np.array([[0.0] * 16, [math.log(2.0)] + [0.0] * 15])
+    q = np.array([1.0] + [0.0] * 15)
+    assign = np.array([0, 0, 1, 0])
+    c, mass = O.cluster_mass(q, cent, assign)
+    np.testing.assert_allclose(c, [0.0, math.log(2.0)])
+    np.testing.assert_allclose(mass, [1.5, 1.0])
+    assert np.array_equal(O.cluster_select(q, cent, assign, 0.6), [True, True, False, True])
+    assert O.cluster_select(q, cent, assign, 0.61).all()
+
+
+def test_clustered_head_at_p1_is_dense_attention():
+    """p = 1 hits every cluster: the head's output is dense attention over all N tokens."""
+    rng = np.random.default_rng(6)
+    N = 200
+    k_pre = O.bf16_round(rng.standard_normal((N, 128)))
+    v = O.bf16_round(rng.standard_normal((N, 128)))
+    q_pre = O.bf16_round(rng.standard_normal(128))
+    wq = rng.standard_normal((128, 16)) / np.sqrt(128)
+    wk = rng.standard_normal((128, 16)) / np.sqrt(128)
+    mu, assign = O.kmeans_index_keys(O.index_keys(k_pre, wk), 16, iters=20)
+    r = O.clustered_head(q_pre, wq, k_pre, v, wk, mu, assign, 1.0)
+    pos = np.arange(N)
+    ref = O.attend(O.rope_rotate(q_pre, N - 1), O.bf16_round(O.rope_rotate(k_pre, pos)), v)
+    assert r.count == N
+    np.testing.assert_allclose(r.out, ref, rtol=1e-12, atol=1e-12)
+    # p < 1: the attended set is a union of whole clusters
+    r2 = O.clustered_head(q_pre, wq, k_pre, v, wk, mu, assign, 0.5)
+    hit = set(assign[r2.sel].tolist())
+    assert set(np.nonzero(np.isin(assign, list(hit)))[0].tolist()) == set(r2.sel.tolist())
