@@ -64,6 +64,23 @@ def test_algorithmic_bytes_closed_form():
     assert full - got == (512 + 32) + 512 + 8192
 
 
+def test_prefill_flops_counts_attended_pairs():
+    """The prefill roofline's FLOPs: 4 * 128 per attended (query head, row, key), counted here
+    pair by pair from the oracle's position sets on a tiny layout."""
+    import dataclasses
+    import numpy as np
+    from oracle import rtp_oracle as O
+    w = dataclasses.replace(workloads.workload(1), sinks=3, window=7)     # 1 retrieval, 1 local
+    n = 40
+    pairs = 0
+    for g in range(w.Hkv):
+        for m in range(n):
+            att = m + 1 if w.ret_mask[0, g] else O.local_positions(m + 1, w.sinks, w.window).size
+            pairs += att * w.G
+    assert bench.prefill_flops(w, n) == 4 * 128 * pairs * w.B
+    assert np.isclose(bench.prefill_flops(workloads.workload(2), 32768) / 1e12, 79.96, atol=0.01)
+
+
 def test_reference_arm_line_fields(capsys, monkeypatch):
     """--impl reference prints one JSON line with the oracle as the CPU baseline."""
     import json
