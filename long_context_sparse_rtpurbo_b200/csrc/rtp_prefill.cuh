@@ -16,8 +16,9 @@
 //   online softmax in the log2 domain (the query carries log2(e) / sqrt(128)), keys checked
 //   one by one only where a tile crosses the row's diagonal, window edge or prompt end; the
 //   probabilities written back to tensor memory as two bf16 terms;
-//   the tile's P V from tensor memory (TS form, 128 x 128), added to the thread's 64 fp32
-//   output dims in registers after the running-maximum rescale.
+//   the tile's P V from tensor memory (TS form, 128 x 128) accumulated into the output in
+//   tensor memory; a row's softmax reference moves only when a tile's maximum exceeds it by
+//   2^8, and only then is the row's accumulated output rescaled in place.
 // The next K tile loads while the softmax runs, the next V tile while the next S is computed.
 #pragma once
 
@@ -39,7 +40,7 @@ constexpr uint32_t kPfKt = 4 * kPfQBlock, kPfVt = kPfKt + 2 * kPfBlock;
 constexpr uint32_t kPfBar = kPfVt + 2 * kPfBlock;         // two mbarriers, the tensor-memory word
 constexpr uint32_t kPfLsum = kPfBar + 64;                 // [2][128] row-sum halves
 constexpr int kPfSmem = (int)kPfLsum + 1024 + 1024;       // + slack to align the base to 1024
-constexpr uint32_t kPfTmemCols = 256;  // S, then P hi / lo, in [0, 64); the PV tile in [128, 256)
+constexpr uint32_t kPfTmemCols = 256;  // S, then P hi / lo, in [0, 64); the output in [128, 256)
 constexpr uint32_t kPfColO = 128;
 constexpr float kPfSlack = 8.f;      // log2 units the softmax reference may lag a row's maximum
 
