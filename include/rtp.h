@@ -24,6 +24,12 @@
  *     rtp_read_device_status.
  *   - head_dim must be 128 and idx_dim 16; G = Hq / Hkv must be 1, 2, 4 or 8. Query head h
  *     reads KV head h / G.
+ *   - The bf16 row arrays (the caches k_ret, v_ret, idx, k_loc, v_loc; q_pre, k_pre, v,
+ *     k_new, v_new and out) are read and written in 16-byte pieces: their device pointers must
+ *     be 16-byte aligned (RTP_EINVAL otherwise, before anything is enqueued).
+ *
+ * Also: the causal prefill of a prompt (rtp_prefill, same paper §3.2: dense for retrieval heads,
+ * sinks + window for local heads) on the fifth-generation tensor cores.
  */
 #ifndef RTP_H
 #define RTP_H

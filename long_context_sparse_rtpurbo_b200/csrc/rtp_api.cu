@@ -30,6 +30,8 @@ std::atomic<int> g_fail_next{0};
 int take_injected() { return g_fail_next.exchange(0); }
 
 inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+// 16-byte aligned (or null): the kernels move bf16 rows in 16-byte pieces
+inline bool al16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
 inline int align16(int x) { return (x + 15) & ~15; }
 
 struct Plan {
@@ -319,6 +321,9 @@ int rtp_append_kv(const rtp_layer_desc* desc, const rtp_cache* cache, const uint
   if (n_new == 0) return RTP_OK;
   if (L.n_ret > 0 && (!cache->k_ret || !cache->v_ret || !cache->idx || !w_kidx)) return RTP_EINVAL;
   if (L.n_loc > 0 && (!cache->k_loc || !cache->v_loc)) return RTP_EINVAL;
+  if (!al16(k_pre) || !al16(v) || !al16(cache->k_ret) || !al16(cache->v_ret) ||
+      !al16(cache->idx) || !al16(cache->k_loc) || !al16(cache->v_loc))
+    return RTP_EINVAL;
   if (cache->T_total < 1 && L.n_ret > 0) return RTP_ESHAPE;
   L.T_total = cache->T_total;
   CachePtrs C{cache->k_ret, cache->v_ret, cache->idx, cache->k_loc, cache->v_loc, cache->seq_off,
@@ -387,6 +392,9 @@ int decode_impl(const rtp_layer_desc* desc, const rtp_cache* cache, const uint16
   if (L.n_loc > 0 && (!cache->k_loc || !cache->v_loc)) return RTP_EINVAL;
   if (L.n_ret > 0 && cache->T_total < 1) return RTP_ESHAPE;
   if (sel_idx && sel_stride < L.maxN) return RTP_EINVAL;
+  if (!al16(q_pre) || !al16(out) || !al16(k_new) || !al16(v_new) || !al16(cache->k_ret) ||
+      !al16(cache->v_ret) || !al16(cache->idx) || !al16(cache->k_loc) || !al16(cache->v_loc))
+    return RTP_EINVAL;
   if (!ws || ws_bytes < pl.total) return RTP_EWORKSPACE;
   if ((reinterpret_cast<uintptr_t>(ws) & 255) != 0) return RTP_EWORKSPACE;
   cudaStream_t st = (cudaStream_t)stream;
@@ -501,6 +509,7 @@ int rtp_prefill(const rtp_layer_desc* desc, const uint16_t* q_pre, const uint16_
   const int rc = check_desc(desc, L);
   if (rc != RTP_OK) return rc;
   if (!q_pre || !k_pre || !v || !n_b || !out || n_max < 0) return RTP_EINVAL;
+  if (!al16(q_pre) || !al16(k_pre) || !al16(v) || !al16(out)) return RTP_EINVAL;
   if (n_max > desc->max_seq_len) return RTP_ESHAPE;
   if (n_max == 0) return RTP_OK;
   if (!ws || ws_bytes < rtp_prefill_workspace_bytes(desc, n_max)) return RTP_EWORKSPACE;

@@ -203,3 +203,24 @@ def test_prefill_workspace_and_argument_checks():
     rtp.rtp_debug_fail_next_call(_lib.RTP_ECUDA)
     assert call(None, 1000, x, need) == _lib.RTP_ECUDA               # before the checks
     assert call(None, 1000, x, need) == _lib.RTP_EINVAL
+
+
+def test_misaligned_row_arrays_are_rejected_before_any_launch():
+    """Row arrays are moved in 16-byte pieces: a pointer off a 16-byte boundary is RTP_EINVAL
+    for the append, the decode step and the prefill (nothing reaches a device)."""
+    d = _desc()
+    lib = _lib.load()
+    x, bad = 0x1000, 0x1002
+    cache = rtp.make_cache(x, x, x, x, x, x, x, 65536)
+    rc = lib.rtp_append_kv(d.ref, ctypes.byref(cache), bad, x, x, x, None, 4, None, None)
+    assert rc == _lib.RTP_EINVAL
+    need = rtp.rtp_workspace_bytes(d)
+    for q, out, c in ((bad, x, cache), (x, bad, cache),
+                      (x, x, rtp.make_cache(x, bad, x, x, x, x, x, 65536))):
+        rc = lib.rtp_decode_step(d.ref, ctypes.byref(c), q, x, x, 0.9, out, x, None, 0, x,
+                                 need, None)
+        assert rc == _lib.RTP_EINVAL
+    pf = rtp.rtp_prefill_workspace_bytes(d, 100)
+    for args in ((bad, x, x, x), (x, bad, x, x), (x, x, bad, x), (x, x, x, bad)):
+        q, k, v, out = args
+        assert lib.rtp_prefill(d.ref, q, k, v, x, 100, out, x, pf, None) == _lib.RTP_EINVAL
