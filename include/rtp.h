@@ -1,5 +1,6 @@
 /*
- * rtp.h -- C ABI of the RTPurbo per-layer decode-step attention library (librtp.so, sm_100a).
+ * rtp.h -- C ABI of the RTPurbo per-layer decode-step and prefill attention library
+ * (librtp.so, sm_100a).
  *
  * What the library computes (sources named by page and section):
  *   "Full Attention Strikes Back: Transferring Full Attention into Sparse within Hundred
@@ -45,7 +46,7 @@ typedef struct CUstream_st* rtp_stream_t;   /* same type as cudaStream_t */
 
 enum {
   RTP_OK = 0,
-  RTP_EINVAL = -1,      /* a null pointer, or a scalar out of range */
+  RTP_EINVAL = -1,      /* a null or misaligned pointer, or a scalar out of range */
   RTP_ESHAPE = -2,      /* inconsistent or unsupported shape */
   RTP_EWORKSPACE = -3,  /* workspace missing or smaller than rtp_workspace_bytes() */
   RTP_ECUDA = -4,       /* a CUDA launch or API call failed */
