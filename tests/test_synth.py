@@ -101,3 +101,33 @@ def test_topk_vs_topp_budget_on_the_32k_workload():
     assert min(conc) > w.p and min(diff) < w.p
     k_all = max(r[2] for r in rows)
     assert len(rows) * k_all > sum(r[2] for r in rows)
+
+
+def test_cluster_prefilter_keeps_the_top_p_set_on_the_32k_workload():
+    """The centroid pre-filter of RTPurboV2 (oracle only, K = 128 clusters of one retrieval KV
+    head's index keys at 32K, cluster-level top-p at p = 0.9): a concentrated head hits a small
+    share of the tokens yet keeps almost all of its token-level top-p set; a diffuse head hits
+    more and still keeps most of it. The numbers are reported in the design notes."""
+    from oracle import rtp_oracle as O
+    w = workloads.workload(2)
+    layer = next(l for l in range(w.layers) if w.ret_mask[l].sum() >= 1)
+    g = int(np.nonzero(w.ret_mask[layer])[0][0])
+    N = int(w.seq_lens[0])
+    kp = gen.bf16_bits_to_f32(w.kpre_bits(layer, 0, g, 0, N)).astype(np.float64)
+    kidx = O.index_keys(kp, w.w_kidx(layer)[g])
+    mu, assign = O.kmeans_index_keys(kidx, 128, iters=10)
+    qb = w.q_pre_bits(layer)
+    seen = set()
+    for h in range(g * w.G, (g + 1) * w.G):
+        q_idx = O.index_query(gen.bf16_bits_to_f32(qb[0, h]).astype(np.float64),
+                              w.w_qidx(layer)[h])
+        v1 = O.topp_histogram(O.index_scores(q_idx, kidx), w.p).mask
+        hit = O.cluster_select(q_idx, mu, assign, w.p)
+        recall = v1[hit].sum() / v1.sum()
+        kind = w.group_layout(layer, 0, g).targets[h % w.G][0]
+        seen.add(kind)
+        if kind == "conc":
+            assert hit.mean() < 0.1 and recall > 0.95, (hit.mean(), recall)
+        else:
+            assert hit.mean() < 0.5 and recall > 0.85, (hit.mean(), recall)
+    assert seen == {"conc", "diff"}
